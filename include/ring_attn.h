@@ -1,0 +1,222 @@
+/*
+ * ring_attn.h -- C ABI of the single-GPU blockwise exact ("ring") attention
+ * forward for NVIDIA B200 (sm_100a).
+ *
+ * What is computed (per batch b, head h and query row i):
+ *
+ *     O[i]   = sum_{j in A(i)} exp(s_ij - m_i) v_j / l_i
+ *     lse[i] = m_i + ln(l_i),    s_ij = softmax_scale * <q_i, k_j>,
+ *     m_i = max_{j in A(i)} s_ij, l_i = sum_{j in A(i)} exp(s_ij - m_i)
+ *
+ * The sequence is split into N = n_ring_blocks "virtual devices" (ring
+ * blocks).  Query block r meets key/value block (r - step) mod N at ring step
+ * step = 0 .. N-1, and every block's partial result is folded into the output
+ * with the online-softmax rescale (running row max, running denominator,
+ * output rescaled by exp(m_old - m_new)); the division by l happens once at
+ * the end.  Sources: "Ring Attention" (Ultralytics glossary), section
+ * "Come funziona la ring attention" and its four-device demo; "Ring Attention
+ * simulation" (gist ring_attention_simulation.py), the flashattention()
+ * per-token update and Device.run ring loop.  On one GPU the ring is a block
+ * iteration order: no data moves between devices.
+ *
+ * Allowed set A(i).  Let pos(t) be the original token index of stored row t
+ * within its sequence (length L), rb(t) its ring block:
+ *   contiguous layout: pos(t) = t, rb(t) = floor(t * N / L)
+ *   striped layout   : ring block r holds tokens r, r+N, r+2N, ... stored
+ *                      consecutively, blocks stored in order r = 0..N-1
+ *                      ("Ring Attention" glossary: Striped Attention gives each
+ *                      device tokens spread evenly over the sequence; the
+ *                      issue thread below asks for striped causal masking to
+ *                      even out the work).
+ * j is in A(i) iff (1) i and j are in the same sequence, (2) causal == 0 or
+ * pos(j) <= pos(i), and (3) (rb(i) - rb(j)) mod N < min(max_ring_passes, N)
+ * (the issue thread's cap on ring passes: a query block sees its own block and
+ * the max_ring_passes - 1 blocks that precede it in the ring).
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    never frees or retains them.  The library allocates one 4-byte device
+ *    status word per device on first use and nothing per call.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy default
+ *    stream).  The return value reports host-side validation and launch
+ *    errors only; device-side errors (bad cu_seqlens contents, a pipeline wait
+ *    that exceeded its bound) are latched in the status word and reported by
+ *    ring_attn_status().
+ *  - Every tensor pointer must be 16-byte aligned (cu_seqlens: 4-byte).
+ *    Violations return RA_ERR_INVALID before anything is launched.
+ *  - Thread safety: calls on different streams may run concurrently; the
+ *    status word is shared per device.
+ */
+#ifndef RING_ATTN_H
+#define RING_ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RA_OK = 0,
+  RA_ERR_INVALID = 1,     /* bad argument; nothing was launched */
+  RA_ERR_UNSUPPORTED = 2, /* valid request this build has no kernel for */
+  RA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+  RA_ERR_TIMEOUT = 4      /* a bounded in-kernel wait expired (device side) */
+} ra_status;
+
+typedef enum { RA_LAYOUT_CONTIGUOUS = 0, RA_LAYOUT_STRIPED = 1 } ra_layout;
+
+typedef enum { RA_F32 = 0, RA_BF16 = 1 } ra_dtype;
+
+/*
+ * ring_attn_fwd -- exact attention forward, ring-ordered blockwise.
+ *
+ * Source: "Ring Attention" glossary, "Come funziona la ring attention" (query
+ * block kept in place, key/value blocks visited in ring order, partials
+ * combined by the running softmax); "Ring Attention simulation" gist,
+ * flashattention() update; issue thread "A ring attention with flash
+ * attention kernel implementation" (lse is returned so that blockwise results
+ * can be combined; maximum ring passes; striped masking; varlen variant).
+ *
+ * Arguments
+ *  q, k, v   dtype elements.  Dense: [batch, seqlen, heads, d_head]
+ *            contiguous (BSHD).  Varlen (cu_seqlens != NULL):
+ *            [seqlen, heads, d_head], seqlen = total rows = cu_seqlens[batch].
+ *  out       same shape and dtype as q; written for every valid row.
+ *  lse       float32.  Dense: [batch, heads, seqlen].  Varlen: [heads, seqlen].
+ *            Natural-log log-sum-exp of the scaled scores.
+ *  batch     number of sequences (>= 1).
+ *  heads     number of heads (>= 1).
+ *  seqlen    dense: tokens per sequence (multiple of n_ring_blocks).
+ *            varlen: total rows of q/k/v/out, which must equal
+ *            cu_seqlens[batch] (the host never reads cu_seqlens, so the call
+ *            stays asynchronous; the kernels check it).
+ *  d_head    head dimension: RA_F32 accepts 16, 32, 64, 128;
+ *            RA_BF16 accepts 64, 128.
+ *  n_ring_blocks  N >= 1, the number of virtual ring devices per sequence.
+ *  layout    ra_layout; buffers are in that stored order and out/lse are
+ *            returned in the same order.
+ *  causal    0 or 1; causal in ORIGINAL token positions.
+ *  softmax_scale  finite scale applied to q.k (the gist uses 1, the glossary
+ *            demo 1/sqrt(d_head)).
+ *  max_ring_passes  P >= 1; values above N are clamped to N.
+ *  cu_seqlens  NULL for dense, else DEVICE int32[batch + 1] (4-byte aligned),
+ *            cu_seqlens[0] = 0, non-decreasing, cu_seqlens[batch] = seqlen.
+ *            Sequence b is rows [cu_seqlens[b], cu_seqlens[b+1]); its ring
+ *            blocks follow its own length (any length >= 1, no divisibility
+ *            requirement).  A negative length or an offset beyond seqlen
+ *            latches RA_ERR_INVALID in the status word and that sequence's
+ *            rows are left unwritten; a wrong cu_seqlens[0] or
+ *            cu_seqlens[batch] latches RA_ERR_INVALID too.
+ *  dtype     ra_dtype of q, k, v and out.
+ *  stream    cudaStream_t to launch on.
+ *
+ * Errors: RA_ERR_INVALID for a null or misaligned pointer, a non-positive
+ * size, seqlen % n_ring_blocks != 0 (dense), max_ring_passes < 1, a
+ * non-finite softmax_scale, causal not in {0,1}, an unknown layout/dtype, or
+ * a d_head outside {16,32,64,128}; RA_ERR_UNSUPPORTED for a d_head the dtype
+ * has no kernel for; RA_ERR_CUDA when a launch fails.
+ */
+ra_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                        float* lse, int batch, int heads, int seqlen,
+                        int d_head, int n_ring_blocks, int layout, int causal,
+                        float softmax_scale, int max_ring_passes,
+                        const int32_t* cu_seqlens, int dtype, void* stream);
+
+/*
+ * ring_attn_qkvpacked_fwd -- same computation, q/k/v packed in one tensor.
+ *
+ * Source: issue thread "A ring attention with flash attention kernel
+ * implementation": ring_flash_attn_qkvpacked_func (mirrors
+ * flash_attn_qkvpacked_func) and its varlen variant; the cu_seqlens shape
+ * (batch_size + 1,) is stated on the "Tensorflow flash attention" page.
+ *
+ *  qkv   dense: [batch, seqlen, 3, heads, d_head]; varlen: [seqlen, 3, heads,
+ *        d_head] (seqlen = total rows).  Index 0/1/2 of the "3" axis is q/k/v.
+ *  out   dense: [batch, seqlen, heads, d_head]; varlen: [seqlen, heads, d_head].
+ *  lse   as ring_attn_fwd.
+ * All other arguments and errors as ring_attn_fwd.
+ */
+ra_status ring_attn_qkvpacked_fwd(const void* qkv, void* out, float* lse,
+                                  int batch, int heads, int seqlen, int d_head,
+                                  int n_ring_blocks, int layout, int causal,
+                                  float softmax_scale, int max_ring_passes,
+                                  const int32_t* cu_seqlens, int dtype,
+                                  void* stream);
+
+/*
+ * ring_attn_fwd_simt -- the same contract as ring_attn_fwd computed by the
+ * CUDA-core (SIMT, fp32 arithmetic) kernel for every dtype and d_head in
+ * {16,32,64,128}.  It is the kernel RA_F32 always uses; for RA_BF16 it is an
+ * independent second GPU path used to cross-check the tensor-core kernel on
+ * every row.  Arguments and errors as ring_attn_fwd.
+ */
+ra_status ring_attn_fwd_simt(const void* q, const void* k, const void* v,
+                             void* out, float* lse, int batch, int heads,
+                             int seqlen, int d_head, int n_ring_blocks,
+                             int layout, int causal, float softmax_scale,
+                             int max_ring_passes, const int32_t* cu_seqlens,
+                             int dtype, void* stream);
+
+/*
+ * ring_attn_merge -- fold partial result (out_b, lse_b) into (out_a, lse_a)
+ * in place:
+ *     lse = max(la, lb) + log1p(exp(min(la, lb) - max(la, lb)))
+ *     out = exp(la - lse) * out_a + exp(lb - lse) * out_b
+ * with lse = -inf and out = 0 when both sides are -inf, and the other side
+ * copied exactly when one side is -inf.
+ *
+ * Source: issue thread "A ring attention with flash attention kernel
+ * implementation": returning lse is what lets blockwise (per ring step)
+ * results be combined, and the KV-outer variant stores outputs and lse and
+ * passes them back in on the next ring pass.
+ *
+ *  out_a, out_b  dtype [batch, seqlen, heads, d_head] (varlen results: batch
+ *                = 1, seqlen = total rows).  out_a is overwritten.
+ *  lse_a, lse_b  float32 [batch, heads, seqlen].  lse_a is overwritten.
+ *  d_head        RA_F32: 4, 8, 16, 32, 64 or 128; RA_BF16: 8, 16, 32, 64,
+ *                128 or 256 (a row is 1 to 32 whole 16-byte chunks).
+ * Errors: RA_ERR_INVALID for null/misaligned pointers, non-positive sizes,
+ * an unsupported d_head or dtype; RA_ERR_CUDA when the launch fails.
+ */
+ra_status ring_attn_merge(void* out_a, float* lse_a, const void* out_b,
+                          const float* lse_b, int batch, int heads, int seqlen,
+                          int d_head, int dtype, void* stream);
+
+/*
+ * ring_attn_status -- synchronize `stream`, then return and clear the current
+ * device's status word (RA_OK when no device-side error was latched since the
+ * last call).  Returns RA_ERR_CUDA when the synchronization itself fails.
+ */
+ra_status ring_attn_status(void* stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* ring_attn_status_string(int status);
+
+/*
+ * ring_attn_schedule -- host-side view of the ring-step scheduler, the same
+ * code the kernels run on the device.  For one sequence of length seqlen it
+ * lists, for every q-tile of q_tile rows (in stored order), the kv-tiles of
+ * kv_tile rows it visits, in visit (ring) order, with their class:
+ *   1 = FULL (every query/key pair of the two tiles is allowed, no mask),
+ *   2 = PARTIAL (mixed; the element mask is applied).
+ * EMPTY pairs (no allowed pair) are not visited and not listed.
+ * The classification is exact whenever the two tiles together touch at most
+ * 64 (q-block, kv-block) pairs of ring blocks; beyond that a pair that is
+ * really EMPTY or FULL may be listed as PARTIAL (never the reverse).
+ *
+ *  out_q, out_kv  int32 tile indices; out_class int8.  HOST arrays of
+ *                 `capacity` entries (may be NULL when capacity is 0).
+ * Returns the total number of visited pairs (which may exceed capacity; only
+ * the first `capacity` are written), or -1 for invalid arguments.
+ */
+int64_t ring_attn_schedule(int seqlen, int n_ring_blocks, int layout,
+                           int causal, int max_ring_passes, int q_tile,
+                           int kv_tile, int32_t* out_q, int32_t* out_kv,
+                           int8_t* out_class, int64_t capacity);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RING_ATTN_H */

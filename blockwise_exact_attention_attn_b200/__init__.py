@@ -1,0 +1,31 @@
+"""Blockwise exact ("ring") attention forward for NVIDIA B200 (sm_100a).
+
+The compute lives in ``libringattn.so`` (C ABI: ``include/ring_attn.h``);
+this package is its thin ctypes binding.  The library is loaded on first use.
+"""
+
+from ._binding import (  # noqa: F401
+    BF16,
+    CONTIGUOUS,
+    EXPORTS,
+    F32,
+    RA_ERR_CUDA,
+    RA_ERR_INVALID,
+    RA_ERR_TIMEOUT,
+    RA_ERR_UNSUPPORTED,
+    RA_OK,
+    STRIPED,
+    RingAttnError,
+    library_path,
+    load_library,
+    ring_attn_func,
+    ring_attn_fwd,
+    ring_attn_fwd_simt,
+    ring_attn_merge,
+    ring_attn_qkvpacked_fwd,
+    ring_attn_qkvpacked_func,
+    ring_attn_schedule,
+    ring_attn_status,
+    ring_attn_status_string,
+    ring_attn_varlen_qkvpacked_func,
+)

@@ -1,0 +1,278 @@
+"""ctypes binding of libringattn.so (include/ring_attn.h).
+
+Argument marshalling only: tensors become device pointers, enums become
+ints, the stream defaults to torch's current CUDA stream.  Every step of the
+computation runs in the library's CUDA kernels; when the library is missing
+the calls raise (there is no fallback).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+from typing import Optional
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libringattn.so")
+
+RA_OK, RA_ERR_INVALID, RA_ERR_UNSUPPORTED, RA_ERR_CUDA, RA_ERR_TIMEOUT = range(5)
+CONTIGUOUS, STRIPED = 0, 1
+F32, BF16 = 0, 1
+
+EXPORTS = (
+    "ring_attn_fwd",
+    "ring_attn_qkvpacked_fwd",
+    "ring_attn_fwd_simt",
+    "ring_attn_merge",
+    "ring_attn_status",
+    "ring_attn_status_string",
+    "ring_attn_schedule",
+)
+
+
+class RingAttnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+
+
+_lib = None
+_lock = threading.Lock()
+
+_c_int = ctypes.c_int
+_c_float = ctypes.c_float
+_c_vp = ctypes.c_void_p
+_c_i64 = ctypes.c_int64
+
+_FWD_ARGS = [_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int, _c_int,
+             _c_int, _c_int, _c_float, _c_int, _c_vp, _c_int, _c_vp]
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load (once) and return the CUDA library; raise when it was not built."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"{path} is missing: build it with "
+                "`python -m blockwise_exact_attention_attn_b200.build`")
+        lib = ctypes.CDLL(path)
+        lib.ring_attn_fwd.argtypes = _FWD_ARGS
+        lib.ring_attn_fwd.restype = _c_int
+        lib.ring_attn_fwd_simt.argtypes = _FWD_ARGS
+        lib.ring_attn_fwd_simt.restype = _c_int
+        lib.ring_attn_qkvpacked_fwd.argtypes = [_c_vp, _c_vp, _c_vp] + _FWD_ARGS[5:]
+        lib.ring_attn_qkvpacked_fwd.restype = _c_int
+        lib.ring_attn_merge.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
+                                        _c_int, _c_int, _c_vp]
+        lib.ring_attn_merge.restype = _c_int
+        lib.ring_attn_status.argtypes = [_c_vp]
+        lib.ring_attn_status.restype = _c_int
+        lib.ring_attn_status_string.argtypes = [_c_int]
+        lib.ring_attn_status_string.restype = ctypes.c_char_p
+        lib.ring_attn_schedule.argtypes = [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                           _c_int, _c_vp, _c_vp, _c_vp, _c_i64]
+        lib.ring_attn_schedule.restype = _c_i64
+        _lib = lib
+        return lib
+
+
+def library_path() -> str:
+    return LIB_PATH
+
+
+def status_string(status: int) -> str:
+    return load_library().ring_attn_status_string(int(status)).decode()
+
+
+ring_attn_status_string = status_string
+
+
+# --------------------------------------------------------------------- helpers
+
+def _ptr(t, name: str) -> int:
+    if t is None:
+        return 0
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def _layout_code(layout) -> int:
+    if isinstance(layout, str):
+        return {"contiguous": CONTIGUOUS, "striped": STRIPED}[layout]
+    return int(layout)
+
+
+def _check(fn: str, st: int):
+    if st != RA_OK:
+        raise RingAttnError(fn, st)
+
+
+# --------------------------------------------------------------------- C ABI
+
+def ring_attn_fwd(q, k, v, out, lse, batch: int, heads: int, seqlen: int, d_head: int,
+                  n_ring_blocks: int, layout=CONTIGUOUS, causal: bool = False,
+                  softmax_scale: Optional[float] = None, max_ring_passes: Optional[int] = None,
+                  cu_seqlens=None, dtype: Optional[int] = None, stream=None) -> None:
+    """Exact ring-ordered blockwise attention forward (see ring_attn.h)."""
+    lib = load_library()
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d_head)
+    if max_ring_passes is None:
+        max_ring_passes = n_ring_blocks
+    st = lib.ring_attn_fwd(
+        _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _ptr(out, "out"), _ptr(lse, "lse"),
+        int(batch), int(heads), int(seqlen), int(d_head), int(n_ring_blocks),
+        _layout_code(layout), int(bool(causal)), float(softmax_scale), int(max_ring_passes),
+        _ptr(cu_seqlens, "cu_seqlens"), _dtype_code(q) if dtype is None else int(dtype),
+        _stream(stream))
+    _check("ring_attn_fwd", st)
+
+
+def ring_attn_fwd_simt(q, k, v, out, lse, batch: int, heads: int, seqlen: int, d_head: int,
+                       n_ring_blocks: int, layout=CONTIGUOUS, causal: bool = False,
+                       softmax_scale: Optional[float] = None,
+                       max_ring_passes: Optional[int] = None, cu_seqlens=None,
+                       dtype: Optional[int] = None, stream=None) -> None:
+    """Same contract as ring_attn_fwd on the CUDA-core kernel."""
+    lib = load_library()
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d_head)
+    if max_ring_passes is None:
+        max_ring_passes = n_ring_blocks
+    st = lib.ring_attn_fwd_simt(
+        _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _ptr(out, "out"), _ptr(lse, "lse"),
+        int(batch), int(heads), int(seqlen), int(d_head), int(n_ring_blocks),
+        _layout_code(layout), int(bool(causal)), float(softmax_scale), int(max_ring_passes),
+        _ptr(cu_seqlens, "cu_seqlens"), _dtype_code(q) if dtype is None else int(dtype),
+        _stream(stream))
+    _check("ring_attn_fwd_simt", st)
+
+
+def ring_attn_qkvpacked_fwd(qkv, out, lse, batch: int, heads: int, seqlen: int, d_head: int,
+                            n_ring_blocks: int, layout=CONTIGUOUS, causal: bool = False,
+                            softmax_scale: Optional[float] = None,
+                            max_ring_passes: Optional[int] = None, cu_seqlens=None,
+                            dtype: Optional[int] = None, stream=None) -> None:
+    """q/k/v packed as [..., 3, heads, d_head] (see ring_attn.h)."""
+    lib = load_library()
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d_head)
+    if max_ring_passes is None:
+        max_ring_passes = n_ring_blocks
+    st = lib.ring_attn_qkvpacked_fwd(
+        _ptr(qkv, "qkv"), _ptr(out, "out"), _ptr(lse, "lse"),
+        int(batch), int(heads), int(seqlen), int(d_head), int(n_ring_blocks),
+        _layout_code(layout), int(bool(causal)), float(softmax_scale), int(max_ring_passes),
+        _ptr(cu_seqlens, "cu_seqlens"), _dtype_code(qkv) if dtype is None else int(dtype),
+        _stream(stream))
+    _check("ring_attn_qkvpacked_fwd", st)
+
+
+def ring_attn_merge(out_a, lse_a, out_b, lse_b, batch: int, heads: int, seqlen: int,
+                    d_head: int, dtype: Optional[int] = None, stream=None) -> None:
+    """Fold (out_b, lse_b) into (out_a, lse_a) in place (see ring_attn.h)."""
+    lib = load_library()
+    st = lib.ring_attn_merge(
+        _ptr(out_a, "out_a"), _ptr(lse_a, "lse_a"), _ptr(out_b, "out_b"), _ptr(lse_b, "lse_b"),
+        int(batch), int(heads), int(seqlen), int(d_head),
+        _dtype_code(out_a) if dtype is None else int(dtype), _stream(stream))
+    _check("ring_attn_merge", st)
+
+
+def ring_attn_status(stream=None) -> int:
+    """Synchronize the stream; return and clear the device status word."""
+    return int(load_library().ring_attn_status(_stream(stream)))
+
+
+def ring_attn_schedule(seqlen: int, n_ring_blocks: int, layout=CONTIGUOUS,
+                       causal: bool = False, max_ring_passes: Optional[int] = None,
+                       q_tile: int = 128, kv_tile: int = 128):
+    """Visited (q_tile, kv_tile, class) triples of the ring scheduler, as
+    three numpy arrays in visit order (class 1 = FULL, 2 = PARTIAL)."""
+    lib = load_library()
+    if max_ring_passes is None:
+        max_ring_passes = n_ring_blocks
+    args = (int(seqlen), int(n_ring_blocks), _layout_code(layout), int(bool(causal)),
+            int(max_ring_passes), int(q_tile), int(kv_tile))
+    n = lib.ring_attn_schedule(*args, None, None, None, 0)
+    if n < 0:
+        raise RingAttnError("ring_attn_schedule", RA_ERR_INVALID)
+    qt = np.zeros(n, dtype=np.int32)
+    kt = np.zeros(n, dtype=np.int32)
+    cl = np.zeros(n, dtype=np.int8)
+    if n:
+        lib.ring_attn_schedule(*args, qt.ctypes.data, kt.ctypes.data, cl.ctypes.data, n)
+    return qt, kt, cl
+
+
+# --------------------------------------------------------------------- user API
+
+def _alloc_out(q_like, rows_shape, heads, d_head, lse_shape):
+    import torch
+    out = torch.empty(*rows_shape, heads, d_head, dtype=q_like.dtype, device=q_like.device)
+    lse = torch.empty(*lse_shape, dtype=torch.float32, device=q_like.device)
+    return out, lse
+
+
+def ring_attn_func(q, k, v, n_ring_blocks: int, causal: bool = False, layout=CONTIGUOUS,
+                   softmax_scale: Optional[float] = None, max_ring_passes: Optional[int] = None,
+                   stream=None):
+    """q, k, v: [batch, seqlen, heads, d_head] CUDA tensors -> (out, lse[batch, heads,
+    seqlen])."""
+    B, S, H, D = q.shape
+    out, lse = _alloc_out(q, (B, S), H, D, (B, H, S))
+    ring_attn_fwd(q, k, v, out, lse, B, H, S, D, n_ring_blocks, layout, causal, softmax_scale,
+                  max_ring_passes, None, None, stream)
+    return out, lse
+
+
+def ring_attn_qkvpacked_func(qkv, n_ring_blocks: int, causal: bool = False,
+                             layout=CONTIGUOUS, softmax_scale: Optional[float] = None,
+                             max_ring_passes: Optional[int] = None, stream=None):
+    """qkv: [batch, seqlen, 3, heads, d_head] -> (out, lse[batch, heads, seqlen])."""
+    B, S, _, H, D = qkv.shape
+    out, lse = _alloc_out(qkv, (B, S), H, D, (B, H, S))
+    ring_attn_qkvpacked_fwd(qkv, out, lse, B, H, S, D, n_ring_blocks, layout, causal,
+                            softmax_scale, max_ring_passes, None, None, stream)
+    return out, lse
+
+
+def ring_attn_varlen_qkvpacked_func(qkv, cu_seqlens, n_ring_blocks: int, causal: bool = False,
+                                    layout=CONTIGUOUS, softmax_scale: Optional[float] = None,
+                                    max_ring_passes: Optional[int] = None, stream=None):
+    """qkv: [total, 3, heads, d_head], cu_seqlens: int32 [batch + 1] (device) ->
+    (out [total, heads, d_head], lse [heads, total])."""
+    T, _, H, D = qkv.shape
+    B = cu_seqlens.numel() - 1
+    out, lse = _alloc_out(qkv, (T,), H, D, (H, T))
+    ring_attn_qkvpacked_fwd(qkv, out, lse, B, H, T, D, n_ring_blocks, layout, causal,
+                            softmax_scale, max_ring_passes, cu_seqlens, None, stream)
+    return out, lse

@@ -1,0 +1,257 @@
+// ra_api.cu -- the C ABI declared in include/ring_attn.h: argument
+// validation (before any CUDA call), the per-device status word, and the
+// choice of kernel (tensor-core kernel for bf16, CUDA-core kernel for fp32).
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include <cuda_runtime.h>
+
+#include "ra_params.h"
+#include "ra_sched.h"
+#include "ring_attn.h"
+
+namespace ra {
+cudaError_t launch_fwd_tc(const FwdParams& p, cudaStream_t stream);
+cudaError_t launch_fwd_simt(const FwdParams& p, int dtype, cudaStream_t stream);
+cudaError_t launch_merge(void* out_a, float* lse_a, const void* out_b, const float* lse_b,
+                         int batch, int heads, int seqlen, int d_head, int dtype, int num_sms,
+                         cudaStream_t stream);
+}  // namespace ra
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int* g_status[kMaxDevices] = {nullptr};
+int g_num_sms[kMaxDevices] = {0};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Current device, its status word (allocated and zeroed on first use) and SM
+// count.
+ra_status device_state(int** status, int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_status[dev]) {
+    int* p = nullptr;
+    if (cudaMalloc(&p, sizeof(int)) != cudaSuccess) return RA_ERR_CUDA;
+    if (cudaMemset(p, 0, sizeof(int)) != cudaSuccess) {
+      cudaFree(p);
+      return RA_ERR_CUDA;
+    }
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaFree(p);
+      return RA_ERR_CUDA;
+    }
+    g_status[dev] = p;
+    g_num_sms[dev] = sms;
+  }
+  *status = g_status[dev];
+  if (num_sms) *num_sms = g_num_sms[dev];
+  return RA_OK;
+}
+
+// Shared validation of the forward calls; fills everything but the tensor
+// pointers' derived fields.
+ra_status validate_fwd(int batch, int heads, int seqlen, int d_head, int n_ring, int layout,
+                       int causal, float scale, int passes, const int32_t* cu_seqlens,
+                       int dtype) {
+  if (batch < 1 || heads < 1 || seqlen < 1 || n_ring < 1) return RA_ERR_INVALID;
+  if (layout != RA_LAYOUT_CONTIGUOUS && layout != RA_LAYOUT_STRIPED) return RA_ERR_INVALID;
+  if (causal != 0 && causal != 1) return RA_ERR_INVALID;
+  if (!std::isfinite(scale)) return RA_ERR_INVALID;
+  if (passes < 1) return RA_ERR_INVALID;
+  if (dtype != RA_F32 && dtype != RA_BF16) return RA_ERR_INVALID;
+  if (d_head != 16 && d_head != 32 && d_head != 64 && d_head != 128) return RA_ERR_INVALID;
+  if (!cu_seqlens && seqlen % n_ring != 0) return RA_ERR_INVALID;
+  if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return RA_ERR_INVALID;
+  // every row index must fit in 32 bits
+  if (!cu_seqlens && (int64_t)batch * seqlen > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
+  if ((int64_t)batch * heads > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
+  return RA_OK;
+}
+
+ra_status run_fwd(const void* q, const void* k, const void* v, int64_t tok_stride, void* out,
+                  float* lse, int batch, int heads, int seqlen, int d_head, int n_ring,
+                  int layout, int causal, float scale, int passes, const int32_t* cu_seqlens,
+                  int dtype, void* stream, bool force_simt) {
+  ra::FwdParams p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.tok_stride = tok_stride;
+  p.out = out;
+  p.lse = lse;
+  p.cu_seqlens = cu_seqlens;
+  p.batch = batch;
+  p.heads = heads;
+  p.seqlen = seqlen;
+  p.d_head = d_head;
+  p.n_ring = n_ring;
+  p.layout = layout;
+  p.causal = causal;
+  p.passes = passes < n_ring ? passes : n_ring;
+  p.scale = scale;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  p.n_qranges = 0;
+  // heaviest query ranges first when later ranges see more keys
+  p.longest_first = (causal && layout == RA_LAYOUT_CONTIGUOUS) ? 1 : 0;
+  if (cu_seqlens) {
+    // varlen: seqlen is the total row count of the packed tensors
+    p.total_rows = seqlen;
+    p.lse_seq_stride = 0;
+    p.lse_head_stride = seqlen;
+  } else {
+    p.total_rows = batch * seqlen;
+    p.lse_seq_stride = (int64_t)heads * seqlen;
+    p.lse_head_stride = seqlen;
+  }
+  int* status = nullptr;
+  ra_status st = device_state(&status, nullptr);
+  if (st != RA_OK) return st;
+  p.status = status;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  // scale 0 (a plain average over the allowed keys) has no log2-domain
+  // reference on the tensor-core path; the CUDA-core kernel handles it
+  if (dtype == RA_BF16 && !force_simt && scale != 0.f) {
+    if (d_head != 64 && d_head != 128) return RA_ERR_UNSUPPORTED;
+    if (((tok_stride * 2) & 15) != 0) return RA_ERR_INVALID;
+    e = ra::launch_fwd_tc(p, s);
+  } else {
+    e = ra::launch_fwd_simt(p, dtype == RA_F32 ? 0 : 1, s);
+  }
+  if (e == cudaErrorInvalidValue) return RA_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+ra_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                        int batch, int heads, int seqlen, int d_head, int n_ring_blocks,
+                        int layout, int causal, float softmax_scale, int max_ring_passes,
+                        const int32_t* cu_seqlens, int dtype, void* stream) {
+  if (!q || !k || !v || !out || !lse) return RA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return RA_ERR_INVALID;
+  ra_status st = validate_fwd(batch, heads, seqlen, d_head, n_ring_blocks, layout, causal,
+                              softmax_scale, max_ring_passes, cu_seqlens, dtype);
+  if (st != RA_OK) return st;
+  return run_fwd(q, k, v, (int64_t)heads * d_head, out, lse, batch, heads, seqlen, d_head,
+                 n_ring_blocks, layout, causal, softmax_scale, max_ring_passes, cu_seqlens,
+                 dtype, stream, false);
+}
+
+ra_status ring_attn_fwd_simt(const void* q, const void* k, const void* v, void* out,
+                             float* lse, int batch, int heads, int seqlen, int d_head,
+                             int n_ring_blocks, int layout, int causal, float softmax_scale,
+                             int max_ring_passes, const int32_t* cu_seqlens, int dtype,
+                             void* stream) {
+  if (!q || !k || !v || !out || !lse) return RA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return RA_ERR_INVALID;
+  ra_status st = validate_fwd(batch, heads, seqlen, d_head, n_ring_blocks, layout, causal,
+                              softmax_scale, max_ring_passes, cu_seqlens, dtype);
+  if (st != RA_OK) return st;
+  return run_fwd(q, k, v, (int64_t)heads * d_head, out, lse, batch, heads, seqlen, d_head,
+                 n_ring_blocks, layout, causal, softmax_scale, max_ring_passes, cu_seqlens,
+                 dtype, stream, true);
+}
+
+ra_status ring_attn_qkvpacked_fwd(const void* qkv, void* out, float* lse, int batch, int heads,
+                                  int seqlen, int d_head, int n_ring_blocks, int layout,
+                                  int causal, float softmax_scale, int max_ring_passes,
+                                  const int32_t* cu_seqlens, int dtype, void* stream) {
+  if (!qkv || !out || !lse) return RA_ERR_INVALID;
+  if (!aligned16(qkv) || !aligned16(out) || !aligned16(lse)) return RA_ERR_INVALID;
+  ra_status st = validate_fwd(batch, heads, seqlen, d_head, n_ring_blocks, layout, causal,
+                              softmax_scale, max_ring_passes, cu_seqlens, dtype);
+  if (st != RA_OK) return st;
+  const int esize = dtype == RA_F32 ? 4 : 2;
+  const int64_t hd = (int64_t)heads * d_head;
+  const char* base = static_cast<const char*>(qkv);
+  return run_fwd(base, base + hd * esize, base + 2 * hd * esize, 3 * hd, out, lse, batch,
+                 heads, seqlen, d_head, n_ring_blocks, layout, causal, softmax_scale,
+                 max_ring_passes, cu_seqlens, dtype, stream, false);
+}
+
+ra_status ring_attn_merge(void* out_a, float* lse_a, const void* out_b, const float* lse_b,
+                          int batch, int heads, int seqlen, int d_head, int dtype,
+                          void* stream) {
+  if (!out_a || !lse_a || !out_b || !lse_b) return RA_ERR_INVALID;
+  if (!aligned16(out_a) || !aligned16(out_b) || !aligned16(lse_a) || !aligned16(lse_b))
+    return RA_ERR_INVALID;
+  if (batch < 1 || heads < 1 || seqlen < 1 || d_head < 1) return RA_ERR_INVALID;
+  if (dtype != RA_F32 && dtype != RA_BF16) return RA_ERR_INVALID;
+  const int esize = dtype == RA_F32 ? 4 : 2;
+  if ((d_head * esize) % 16 != 0) return RA_ERR_INVALID;
+  const int chunks = d_head * esize / 16;
+  if (chunks > 32 || (chunks & (chunks - 1)) != 0) return RA_ERR_INVALID;
+  if ((int64_t)batch * seqlen * heads > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
+  int* status = nullptr;
+  int sms = 0;
+  ra_status st = device_state(&status, &sms);
+  if (st != RA_OK) return st;
+  cudaError_t e = ra::launch_merge(out_a, lse_a, out_b, lse_b, batch, heads, seqlen, d_head,
+                                   dtype == RA_F32 ? 0 : 1, sms,
+                                   reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+ra_status ring_attn_status(void* stream) {
+  int* status = nullptr;
+  ra_status st = device_state(&status, nullptr);
+  if (st != RA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return RA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return RA_ERR_CUDA;
+  if (v != 0 && cudaMemset(status, 0, sizeof(int)) != cudaSuccess) return RA_ERR_CUDA;
+  return static_cast<ra_status>(v);
+}
+
+const char* ring_attn_status_string(int status) {
+  switch (status) {
+    case RA_OK: return "RA_OK";
+    case RA_ERR_INVALID: return "RA_ERR_INVALID";
+    case RA_ERR_UNSUPPORTED: return "RA_ERR_UNSUPPORTED";
+    case RA_ERR_CUDA: return "RA_ERR_CUDA";
+    case RA_ERR_TIMEOUT: return "RA_ERR_TIMEOUT";
+  }
+  return "RA_ERR_UNKNOWN";
+}
+
+int64_t ring_attn_schedule(int seqlen, int n_ring_blocks, int layout, int causal,
+                           int max_ring_passes, int q_tile, int kv_tile, int32_t* out_q,
+                           int32_t* out_kv, int8_t* out_class, int64_t capacity) {
+  if (seqlen < 1 || n_ring_blocks < 1 || max_ring_passes < 1 || q_tile < 1 || kv_tile < 1)
+    return -1;
+  if (layout != RA_LAYOUT_CONTIGUOUS && layout != RA_LAYOUT_STRIPED) return -1;
+  if (causal != 0 && causal != 1) return -1;
+  if (capacity > 0 && (!out_q || !out_kv || !out_class)) return -1;
+  const ra::RingGeom g = ra::make_geom(seqlen, n_ring_blocks, layout, causal, max_ring_passes);
+  int64_t n = 0;
+  for (int q0 = 0; q0 < seqlen; q0 += q_tile) {
+    const int q1 = q0 + q_tile < seqlen ? q0 + q_tile : seqlen;
+    ra::TileWalk w;
+    w.init(g, q0, q1, q1, kv_tile);
+    int kt, c0, c1;
+    while (w.next(&kt, &c0, &c1)) {
+      if (n < capacity) {
+        out_q[n] = q0 / q_tile;
+        out_kv[n] = kt;
+        out_class[n] = (int8_t)c0;
+      }
+      ++n;
+    }
+  }
+  return n;
+}
+
+}  // extern "C"

@@ -1,0 +1,201 @@
+// ra_fwd_simt.cu -- ring-ordered blockwise attention forward on CUDA cores
+// (fp32 arithmetic), for fp32 inputs and as an independent cross-check of
+// the tensor-core kernel for bf16 inputs.
+//
+// Each CTA owns one range of query rows of one (sequence, head) and walks the
+// key/value tiles in ring order (ra_sched.h).  Every tile is folded into the
+// running state of each query row with the online-softmax rescale: new row
+// max, old output and denominator scaled by exp(m_old - m_new), then the
+// tile's exponentials added ("Ring Attention simulation" gist, the
+// flashattention() update of output, maxima and denominators; "Ring
+// Attention" glossary, "Come funziona la ring attention": a running sum of
+// exponentiated scores and of weighted values, divided at the end).  Here the
+// division by the denominator is deferred to the end, as in the glossary.
+//
+// A query row is served by TPR = d_head / DPT threads, each holding DPT of its
+// dimensions; the dot products are completed with warp shuffles.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "ra_common.cuh"
+#include "ra_params.h"
+#include "ra_sched.h"
+#include "ra_work.cuh"
+
+namespace ra {
+
+constexpr int kSimtThreads = 128;
+constexpr int kSimtBN = 64;
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kSimtThreads)
+    fwd_simt_kernel(const FwdParams p) {
+  constexpr int DPT = D < 32 ? D : 32;     // dims per thread
+  constexpr int TPR = D / DPT;             // threads per row
+  constexpr int ROWS = kSimtThreads / TPR; // query rows per CTA
+  constexpr int BN = kSimtBN;
+
+  extern __shared__ float smem_f[];
+  float* Ks = smem_f;            // [BN][D]
+  float* Vs = smem_f + BN * D;   // [BN][D]
+
+  const SeqWork it = find_work(p, ROWS);
+  if (!it.live) return;  // uniform across the CTA
+  const int base = it.base, L = it.L;
+  const int q0 = it.qr * ROWS;
+  const int q1 = min(q0 + ROWS, L);
+
+  const int tid = threadIdx.x;
+  const int rloc = tid / TPR;
+  const int part = tid % TPR;
+  const int sq = q0 + rloc;          // stored row of this thread's query
+  const bool valid = sq < L;
+
+  const RingGeom g = make_geom(L, p.n_ring, p.layout, p.causal, p.passes);
+  int rq = 0, tq = 0;
+  if (valid) {
+    rq = block_of(g, sq);
+    tq = token_of(g, sq, rq);
+  }
+
+  const T* qg = static_cast<const T*>(p.q);
+  const T* kg = static_cast<const T*>(p.k);
+  const T* vg = static_cast<const T*>(p.v);
+
+  float qr[DPT], o[DPT];
+#pragma unroll
+  for (int d = 0; d < DPT; ++d) {
+    qr[d] = valid ? to_f32(qg[(int64_t)(base + sq) * p.tok_stride + (int64_t)it.h * D +
+                              part * DPT + d])
+                  : 0.f;
+    o[d] = 0.f;
+  }
+  float m = -INFINITY;  // running max, log2 domain (score * scale * log2 e)
+  float l = 0.f;        // running denominator relative to m
+
+  TileWalk walk;
+  walk.init(g, q0, q1, q1, BN);
+  int kt, c0, c1;
+  while (walk.next(&kt, &c0, &c1)) {
+    const int k0 = kt * BN;
+    const int nk = min(BN, L - k0);
+    __syncthreads();  // previous tile fully consumed
+    for (int e = tid; e < BN * D; e += kSimtThreads) {
+      const int c = e / D, d = e % D;
+      float kv = 0.f, vv = 0.f;
+      if (c < nk) {
+        const int64_t off =
+            (int64_t)(base + k0 + c) * p.tok_stride + (int64_t)it.h * D + d;
+        kv = to_f32(kg[off]);
+        vv = to_f32(vg[off]);
+      }
+      Ks[e] = kv;
+      Vs[e] = vv;
+    }
+    __syncthreads();
+
+    float s[BN];
+    float tile_max = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < BN; ++c) {
+      const float* kr = Ks + c * D + part * DPT;
+      float acc = 0.f;
+#pragma unroll
+      for (int d = 0; d < DPT; ++d) acc = fmaf(qr[d], kr[d], acc);
+#pragma unroll
+      for (int off = 1; off < TPR; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      float x = acc * p.scale_log2;
+      bool ok = c < nk;
+      if (ok && c0 == CLS_PARTIAL && valid) ok = allowed(g, sq, rq, tq, k0 + c);
+      x = ok ? x : -INFINITY;
+      s[c] = x;
+      tile_max = fmaxf(tile_max, x);
+    }
+    const float m_new = fmaxf(m, tile_max);
+    if (m_new == -INFINITY) continue;  // nothing allowed for this row yet
+    const float alpha = exp2f(m - m_new);  // 0 when m == -inf
+    l *= alpha;
+#pragma unroll
+    for (int d = 0; d < DPT; ++d) o[d] *= alpha;
+#pragma unroll
+    for (int c = 0; c < BN; ++c) {
+      const float pc = exp2f(s[c] - m_new);
+      l += pc;
+      const float* vr = Vs + c * D + part * DPT;
+#pragma unroll
+      for (int d = 0; d < DPT; ++d) o[d] = fmaf(pc, vr[d], o[d]);
+    }
+    m = m_new;
+  }
+
+  if (!valid) return;
+  T* og = static_cast<T*>(p.out);
+  const float inv_l = 1.f / l;
+  const int64_t orow = (int64_t)(base + sq) * p.heads * D + (int64_t)it.h * D + part * DPT;
+#pragma unroll
+  for (int d = 0; d < DPT; ++d) og[orow + d] = from_f32<T>(o[d] * inv_l);
+  if (part == 0) {
+    const int64_t li = (int64_t)it.b * p.lse_seq_stride + (int64_t)it.h * p.lse_head_stride +
+                       (p.cu_seqlens ? base : 0) + sq;
+    // lse = ln(l) + m / log2(e), with m in the log2 domain
+    p.lse[li] = (m + log2f(l)) * 0.69314718055994530942f;
+  }
+}
+
+template <typename T, int D>
+static cudaError_t launch_simt_t(const FwdParams& p, cudaStream_t stream) {
+  constexpr int DPT = D < 32 ? D : 32;
+  constexpr int ROWS = kSimtThreads / (D / DPT);
+  FwdParams pp = p;
+  pp.n_qranges = (p.seqlen + ROWS - 1) / ROWS;
+  const int64_t grid = work_grid(pp, ROWS);
+  if (grid == 0) return cudaSuccess;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  const size_t smem = 2 * kSimtBN * D * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(fwd_simt_kernel<T, D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  fwd_simt_kernel<T, D><<<(unsigned)grid, kSimtThreads, smem, stream>>>(pp);
+  return cudaGetLastError();
+}
+
+// dtype: 0 = fp32, 1 = bf16.  Returns cudaErrorInvalidValue for an
+// unsupported head dimension.
+cudaError_t launch_fwd_simt(const FwdParams& p, int dtype, cudaStream_t stream) {
+  if (dtype == 0) {
+    switch (p.d_head) {
+      case 16: return launch_simt_t<float, 16>(p, stream);
+      case 32: return launch_simt_t<float, 32>(p, stream);
+      case 64: return launch_simt_t<float, 64>(p, stream);
+      case 128: return launch_simt_t<float, 128>(p, stream);
+    }
+  } else {
+    switch (p.d_head) {
+      case 16: return launch_simt_t<__nv_bfloat16, 16>(p, stream);
+      case 32: return launch_simt_t<__nv_bfloat16, 32>(p, stream);
+      case 64: return launch_simt_t<__nv_bfloat16, 64>(p, stream);
+      case 128: return launch_simt_t<__nv_bfloat16, 128>(p, stream);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ra

@@ -1,0 +1,648 @@
+// ra_fwd_tc.cu -- ring-ordered blockwise attention forward on the sm_100a
+// tensor cores (tcgen05 + TMEM), bf16 inputs, fp32 accumulation.
+//
+// The method: the sequence is split into N ring blocks; a query block keeps
+// its queries in place and meets the key/value blocks in ring order, folding
+// each block into its output with the running softmax ("Ring Attention"
+// glossary, "Come funziona la ring attention"; "Ring Attention simulation"
+// gist, flashattention() update: running row max, running denominator,
+// output rescaled by exp(m_old - m_new)).  Production kernels subtract the
+// running maximum before exponentiating (same glossary page).  The blockwise
+// evaluation inside one device is the flash-attention tiling of the
+// "Attention的分块计算" blog (local softmax of a block in fast on-chip memory,
+// combined into the global softmax through per-block max and sum).
+//
+// CTA organisation (one CTA per SM, 384 threads):
+//   warps 0-3  softmax for query tile 0 (one TMEM lane = one query row each)
+//   warps 4-7  softmax for query tile 1
+//   warp  8    TMA producer: Q tiles once, then K and V tiles through an
+//              NS-slot shared-memory ring guarded by mbarriers
+//   warp  9    MMA issuer: S_i = Q_i K^T and O_i += P_i V as tcgen05.mma,
+//              completion signalled with tcgen05.commit
+//   warp  10   schedule builder: runs the ring-order tile walk (ra_sched.h)
+//              and publishes the visited kv tiles with their per-query-tile
+//              class into a double-buffered shared-memory list
+//   warp  11   idle (completes the control warpgroup, whose register budget
+//              is handed to the softmax warpgroups with setmaxnreg)
+// Tensor memory (512 columns): S_0 | S_1 | O_0 | O_1; P_i (bf16) is written
+// over the first BN/2 columns of S_i once its scores are in registers.
+//
+// Issue order of the MMA warp for consecutive kv tiles t-1, t:
+//   PV_0(t-1), S_0(t), PV_1(t-1), S_1(t)
+// so the tensor core computes S of one query tile while the softmax warps of
+// the other tile work, and a finished S_i(t) implies PV_i(t-1) finished
+// (commits track all earlier MMAs), which makes the O rescale safe.
+//
+// The running max is only moved when it grows by more than kRescaleLog2
+// (in log2 units); until then exponentials are taken against the stale max
+// (values <= 2^kRescaleLog2), which is exact up to rounding because the same
+// reference is used for O and l.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "ra_common.cuh"
+#include "ra_params.h"
+#include "ra_sched.h"
+#include "ra_work.cuh"
+
+namespace ra {
+
+constexpr int kTcBM = 128;          // rows per query tile (TMEM lanes)
+constexpr int kTcQT = 2;            // query tiles per CTA
+constexpr int kTcBN = 128;          // keys per kv tile
+constexpr int kTcThreads = 384;     // 2 softmax warpgroups + 1 control warpgroup
+constexpr int kTcProducerWarp = 8;
+constexpr int kTcMmaWarp = 9;
+constexpr int kTcListWarp = 10;
+constexpr int kListChunk = 1024;    // entries per schedule-list buffer (2 buffers)
+constexpr int kListConsumers = 10;  // producer, MMA, 8 softmax warps
+// Register split.  Launch: 384 threads x 168 = 64512 registers.  After the
+// split: 256 softmax threads x 176 + 128 control threads x 152 = 64512.
+constexpr int kRegsSoftmax = 176;
+constexpr int kRegsControl = 152;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleLog2 = 8.0f;
+
+template <int D>
+struct TcCfg {
+  static constexpr int kPanels = D / 64;                    // 128-byte swizzle panels
+  static constexpr int kPanelBytes = kTcBM * 128;           // 128 rows x 128 B
+  static constexpr int kTileBytes = kPanels * kPanelBytes;  // one Q/K/V tile
+  static constexpr int kStages = D == 128 ? 4 : 8;          // K/V slots
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = kTcQT * kTileBytes;
+  static constexpr int kListOff = kKVOff + kStages * kTileBytes;
+  static constexpr int kCtrlOff = kListOff + 2 * kListChunk * 4;
+  static constexpr int kSmemBytes = kCtrlOff + 1024 + 1024;  // + ctrl + align slack
+  static constexpr uint32_t kColS = 0;                      // S_i at i * 128
+  static constexpr uint32_t kColO = 256;                    // O_i at 256 + i * D
+};
+
+struct TcCtrl {
+  uint64_t q_full;
+  uint64_t kv_full[8];
+  uint64_t kv_empty[8];
+  uint64_t s_full[kTcQT];
+  uint64_t p_full[kTcQT];
+  uint64_t o_full[kTcQT];
+  uint64_t list_full[2];
+  uint64_t list_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct TcMaps {
+  CUtensorMap q, k, v;
+};
+
+// Number of leading columns of kv tile [k0, k0 + nk) allowed for query (rq,
+// tq) when the whole tile lies in ring block rk (the allowed keys of one
+// block always form a prefix in stored order).
+__device__ __forceinline__ int single_block_limit(const RingGeom& g, int rq, int tq, int rk,
+                                                  int k0, int nk) {
+  if (!pass_ok(g, rq, rk)) return 0;
+  if (!g.causal) return nk;
+  int last;  // last allowed stored key of block rk
+  if (g.layout == LAYOUT_CONTIGUOUS) {
+    last = tq;
+  } else {
+    if (tq < rk) return 0;
+    last = block_start(g, rk) + (tq - rk) / g.N;
+  }
+  const int lim = last - k0 + 1;
+  return lim < 0 ? 0 : (lim > nk ? nk : lim);
+}
+
+// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  __syncwarp();
+  return ok;
+}
+
+// S = Q K^T for one query tile: M = 128 rows, N = 128 keys, K = D in steps of
+// 16.  Both operands K-major in 128-byte-swizzled panels of 64 elements.
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t qbase, uint32_t kbase,
+                                         uint32_t idesc) {
+  using C = TcCfg<D>;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+    umma_ss(d_tmem, smem_desc_sw128(qbase + off, 16, 1024),
+            smem_desc_sw128(kbase + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// O (+)= P V for one query tile: A = P from tensor memory (128 x 128 bf16,
+// 8 columns per 16 keys), B = V tile MN-major (N = D split in 64-element
+// panels, LBO = panel stride; 8-key groups 1024 bytes apart).
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t vbase,
+                                         uint32_t idesc, bool accumulate) {
+  using C = TcCfg<D>;
+#pragma unroll
+  for (int kk = 0; kk < kTcBN / 16; ++kk) {
+    umma_ts(d_tmem, p_tmem + kk * 8, smem_desc_sw128(vbase + kk * 16 * 128, C::kPanelBytes, 1024),
+            idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// Replace the scores of disallowed keys by -inf.  Keys at or beyond L (the
+// next sequence, or rows past the tensor) are always disallowed; on PARTIAL
+// tiles the ring mask is applied too.
+__device__ __forceinline__ void apply_mask(float* x, const FwdParams& p, int L, bool valid,
+                                           int cls, int sq, int rq, int tq, int k0, int nk) {
+  int lim;
+  const RingGeom g = make_geom(L, p.n_ring, p.layout, p.causal, p.passes);
+  if (!valid || cls == CLS_FULL) {
+    lim = nk;
+  } else {
+    const int rk0 = block_of(g, k0), rk1 = block_of(g, k0 + nk - 1);
+    lim = rk0 == rk1 ? single_block_limit(g, rq, tq, rk0, k0, nk) : -1;
+  }
+  // allowed columns as 4 x 32-bit masks (indices stay compile-time)
+  uint32_t mw[kTcBN / 32];
+#pragma unroll
+  for (int w = 0; w < kTcBN / 32; ++w) {
+    if (lim >= 0) {
+      const int n = min(max(lim - 32 * w, 0), 32);
+      mw[w] = n >= 32 ? 0xffffffffu : ((1u << n) - 1u);
+    } else {
+      uint32_t bits = 0;
+      for (int bit = 0; bit < 32; ++bit) {
+        const int c = 32 * w + bit;
+        if (c < nk && allowed(g, sq, rq, tq, k0 + c)) bits |= 1u << bit;
+      }
+      mw[w] = bits;
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < kTcBN; ++c) x[c] = ((mw[c >> 5] >> (c & 31)) & 1u) ? x[c] : -INFINITY;
+}
+
+// Schedule-list entries: (kt << 4) | (class of query tile 1 << 2) | class of
+// query tile 0; -1 ends the list.
+__device__ __forceinline__ int entry_tile(int e) { return e >> 4; }
+__device__ __forceinline__ int entry_cls(int e, int i) { return (e >> (2 * i)) & 3; }
+
+// Sequential reader of the schedule list for a single thread (producer, MMA).
+struct ListReader {
+  const int* list;
+  uint64_t* full;
+  uint64_t* empty;
+  int n;
+  // Next entry into *e; false when a wait gave up.
+  __device__ __forceinline__ bool next(int* e, volatile int* abort) {
+    const int pos = n & (kListChunk - 1);
+    const int c = n / kListChunk;
+    if (pos == 0 && !mbar_wait(&full[c & 1], (c >> 1) & 1, abort)) return false;
+    *e = list[(c & 1) * kListChunk + pos];
+    ++n;
+    if (pos == kListChunk - 1 || *e < 0) mbar_arrive(&empty[c & 1]);
+    return true;
+  }
+  // Same for a whole warp: lane 0 waits and releases, every lane reads.
+  __device__ __forceinline__ bool next_warp(int* e, volatile int* abort) {
+    const int pos = n & (kListChunk - 1);
+    const int c = n / kListChunk;
+    if (pos == 0 && !warp_wait(&full[c & 1], (c >> 1) & 1, abort)) return false;
+    *e = list[(c & 1) * kListChunk + pos];
+    ++n;
+    if (pos == kListChunk - 1 || *e < 0) {
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[c & 1]);
+    }
+    return true;
+  }
+};
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    fwd_tc_kernel(const FwdParams p, const __grid_constant__ TcMaps maps) {
+  using C = TcCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  TcCtrl* ctrl = reinterpret_cast<TcCtrl*>(smem + C::kCtrlOff);
+  volatile int* abort_flag = &ctrl->abort;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const SeqWork it = find_work(p, kTcBM * kTcQT);
+  if (!it.live) return;  // uniform across the CTA
+  const int base = it.base, L = it.L;
+  const int q0 = it.qr * (kTcBM * kTcQT);
+  const int qm = min(q0 + kTcBM, L);
+  const int q1 = min(q0 + kTcBM * kTcQT, L);
+
+  // ------------------------------------------------------------ set-up
+  int* list = reinterpret_cast<int*>(smem + C::kListOff);
+  if (threadIdx.x == 0) {
+    mbar_init(&ctrl->q_full, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&ctrl->kv_full[s], 1);
+      mbar_init(&ctrl->kv_empty[s], 1);
+    }
+    for (int i = 0; i < kTcQT; ++i) {
+      mbar_init(&ctrl->s_full[i], 1);
+      mbar_init(&ctrl->p_full[i], kTcBM);
+      mbar_init(&ctrl->o_full[i], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctrl->list_full[b], 1);
+      mbar_init(&ctrl->list_empty[b], kListConsumers);
+    }
+    mbar_init(&ctrl->drain, 1);
+    ctrl->abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == kTcMmaWarp) {
+    tmem_alloc(&ctrl->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem_base;
+  ListReader rd;
+  rd.list = list;
+  rd.full = ctrl->list_full;
+  rd.empty = ctrl->list_empty;
+  rd.n = 0;
+
+  if (warp >= 8) {
+   regs_dec<kRegsControl>();
+   if (warp == kTcListWarp) {
+    // ---------------------------------------------------------- schedule
+    if (lane == 0) {
+      const RingGeom g = make_geom(L, p.n_ring, p.layout, p.causal, p.passes);
+      TileWalk walk;
+      walk.init(g, q0, qm, q1, kTcBN);
+      bool done = false, ok = true;
+      for (int c = 0; !done; ++c) {
+        const int b = c & 1;
+        if (c >= 2 && !mbar_wait(&ctrl->list_empty[b], ((c >> 1) - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        int* dst = list + b * kListChunk;
+        for (int pos = 0; pos < kListChunk; ++pos) {
+          int kt, c0, c1;
+          if (walk.next(&kt, &c0, &c1)) {
+            dst[pos] = (kt << 4) | (c1 << 2) | c0;
+          } else {
+            dst[pos] = -1;
+            done = true;
+            break;
+          }
+        }
+        mbar_arrive(&ctrl->list_full[b]);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        latch_status(p.status, ST_TIMEOUT);
+      }
+    }
+    __syncwarp();
+   } else if (warp == kTcProducerWarp) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      tma_prefetch_desc(&maps.q);
+      tma_prefetch_desc(&maps.k);
+      tma_prefetch_desc(&maps.v);
+      uint8_t* qs = smem + C::kQOff;
+      mbar_arrive_expect_tx(&ctrl->q_full, kTcQT * C::kTileBytes);
+      for (int i = 0; i < kTcQT; ++i)
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_3d(qs + i * C::kTileBytes + pn * C::kPanelBytes, &maps.q, &ctrl->q_full,
+                      pn * 64, it.h, base + q0 + i * kTcBM);
+      int n = 0;
+      bool ok = true;
+      int e;
+      while (true) {
+        ok = rd.next(&e, abort_flag);
+        if (!ok || e < 0) break;
+        const int kt = entry_tile(e);
+        for (int which = 0; which < 2 && ok; ++which) {
+          const int slot = n % C::kStages;
+          if (n >= C::kStages) {
+            ok = mbar_wait(&ctrl->kv_empty[slot], ((n / C::kStages) - 1) & 1, abort_flag);
+            if (!ok) break;
+          }
+          uint8_t* dst = smem + C::kKVOff + slot * C::kTileBytes;
+          mbar_arrive_expect_tx(&ctrl->kv_full[slot], C::kTileBytes);
+          const CUtensorMap* map = which == 0 ? &maps.k : &maps.v;
+          for (int pn = 0; pn < C::kPanels; ++pn)
+            tma_load_3d(dst + pn * C::kPanelBytes, map, &ctrl->kv_full[slot], pn * 64, it.h,
+                        base + kt * kTcBN);
+          ++n;
+        }
+        if (!ok) break;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        latch_status(p.status, ST_TIMEOUT);
+        // let the copies already issued land before the CTA can exit
+        for (int u = (n > C::kStages ? n - C::kStages : 0); u < n; ++u)
+          mbar_wait(&ctrl->kv_full[u % C::kStages], (u / C::kStages) & 1, nullptr);
+        mbar_wait(&ctrl->q_full, 0, nullptr);
+      }
+    }
+    __syncwarp();
+   } else if (warp == kTcMmaWarp) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      // a negative softmax scale is applied as S = (-Q) K^T times |scale|
+      const uint32_t idesc_s =
+          idesc_bf16_f32(kTcBM, kTcBN, 0) | (p.scale_log2 < 0.f ? (1u << 13) : 0u);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(kTcBM, D, 1);
+      const uint32_t qs = smem_u32(smem + C::kQOff);
+      const uint32_t kvs = smem_u32(smem + C::kKVOff);
+      bool ok = mbar_wait(&ctrl->q_full, 0, abort_flag);
+      tc_fence_after();
+      uint32_t pphase[kTcQT] = {0, 0};
+      bool started[kTcQT] = {false, false};
+      int n = 0;
+      bool issued_any = false;
+      int e = -1, ep = -1;
+      if (ok) ok = rd.next(&e, abort_flag);
+      if (ok && e >= 0) {
+        const int slot = n % C::kStages;
+        ok = mbar_wait(&ctrl->kv_full[slot], (n / C::kStages) & 1, abort_flag);
+        ++n;
+        if (ok) {
+          tc_fence_after();
+          for (int i = 0; i < kTcQT; ++i)
+            if (entry_cls(e, i) != CLS_EMPTY) {
+              issue_qk<D>(tmem + C::kColS + i * kTcBN, qs + i * C::kTileBytes,
+                          kvs + slot * C::kTileBytes, idesc_s);
+              umma_commit(&ctrl->s_full[i]);
+            }
+          umma_commit(&ctrl->kv_empty[slot]);
+          issued_any = true;
+        }
+        ep = e;
+        while (ok) {
+          const int slot_v = n % C::kStages;
+          ok = mbar_wait(&ctrl->kv_full[slot_v], (n / C::kStages) & 1, abort_flag);
+          ++n;
+          if (!ok) break;
+          ok = rd.next(&e, abort_flag);
+          if (!ok) break;
+          const bool has = e >= 0;
+          int slot_k = 0;
+          if (has) {
+            slot_k = n % C::kStages;
+            ok = mbar_wait(&ctrl->kv_full[slot_k], (n / C::kStages) & 1, abort_flag);
+            ++n;
+            if (!ok) break;
+          }
+          tc_fence_after();
+          for (int i = 0; i < kTcQT && ok; ++i) {
+            if (entry_cls(ep, i) != CLS_EMPTY) {
+              ok = mbar_wait(&ctrl->p_full[i], pphase[i], abort_flag);
+              pphase[i] ^= 1;
+              if (!ok) break;
+              tc_fence_after();
+              issue_pv<D>(tmem + C::kColO + i * D, tmem + C::kColS + i * kTcBN,
+                          kvs + slot_v * C::kTileBytes, idesc_o, started[i]);
+              started[i] = true;
+            }
+            if (has && entry_cls(e, i) != CLS_EMPTY) {
+              issue_qk<D>(tmem + C::kColS + i * kTcBN, qs + i * C::kTileBytes,
+                          kvs + slot_k * C::kTileBytes, idesc_s);
+              umma_commit(&ctrl->s_full[i]);
+            }
+          }
+          if (!ok) break;
+          umma_commit(&ctrl->kv_empty[slot_v]);
+          if (!has) break;
+          umma_commit(&ctrl->kv_empty[slot_k]);
+          ep = e;
+        }
+      }
+      if (ok) {
+        for (int i = 0; i < kTcQT; ++i) umma_commit(&ctrl->o_full[i]);
+      } else {
+        *abort_flag = 1;
+        latch_status(p.status, ST_TIMEOUT);
+        if (issued_any) {
+          // wait (bounded) for the MMAs already issued before TMEM is freed
+          umma_commit(&ctrl->drain);
+          mbar_wait(&ctrl->drain, 0, nullptr);
+        }
+      }
+    }
+    __syncwarp();
+   }
+  } else {
+    regs_inc<kRegsSoftmax>();
+    // ---------------------------------------------------------- softmax
+    const int tile = warp >> 2;          // query tile handled by this warp
+    const int quad = warp & 3;           // TMEM lane quadrant
+    const int r = quad * 32 + lane;      // row within the query tile
+    const int sq = q0 + tile * kTcBM + r;
+    const bool valid = sq < L;
+    int rq = 0, tq = 0;
+    if (valid) {
+      const RingGeom g = make_geom(L, p.n_ring, p.layout, p.causal, p.passes);
+      rq = block_of(g, sq);
+      tq = token_of(g, sq, rq);
+    }
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::kColS + tile * kTcBN;
+    const uint32_t tO = tmem + lane_off + C::kColO + tile * D;
+    const float sl2 = fabsf(p.scale_log2);  // > 0; the sign is folded into the MMA
+
+    float m_ref = -INFINITY;  // reference max, log2 domain
+    float l = 0.f;
+    uint32_t sphase = 0;
+    bool first = true;
+    bool ok = true;
+
+    while (true) {
+      int e;
+      ok = rd.next_warp(&e, abort_flag);
+      if (!ok || e < 0) break;
+      const int cls = entry_cls(e, tile);
+      if (cls == CLS_EMPTY) continue;
+      ok = warp_wait(&ctrl->s_full[tile], sphase, abort_flag);
+      sphase ^= 1;
+      if (!ok) break;
+      tc_fence_after();
+
+      float x[kTcBN];
+      {
+        uint32_t* xr = reinterpret_cast<uint32_t*>(x);
+#pragma unroll
+        for (int c = 0; c < kTcBN; c += 32) RA_TMEM_LD32(tS + c, (xr + c));
+        tmem_wait_ld();
+      }
+      const int k0 = entry_tile(e) * kTcBN;
+      const int nk = min(kTcBN, L - k0);
+      if (cls == CLS_PARTIAL || nk < kTcBN) {
+        apply_mask(x, p, L, valid, cls, sq, rq, tq, k0, nk);
+      }
+      float mx = x[0];
+#pragma unroll
+      for (int c = 1; c < kTcBN; ++c) mx = fmaxf(mx, x[c]);
+      const float m_tile = mx * sl2;  // -inf stays -inf (sl2 > 0)
+      const bool need = m_tile > m_ref + kRescaleLog2;
+      float alpha = 1.f;
+      if (need) {
+        alpha = ex2_approx(m_ref - m_tile);  // 0 when m_ref == -inf
+        m_ref = m_tile;
+      }
+      const float msub = m_ref == -INFINITY ? 0.f : m_ref;
+      float rs = 0.f;
+#pragma unroll
+      for (int q = 0; q < kTcBN / 32; ++q) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float a = ex2_approx(fmaf(x[q * 32 + 2 * j], sl2, -msub));
+          const float b = ex2_approx(fmaf(x[q * 32 + 2 * j + 1], sl2, -msub));
+          rs += a + b;
+          pk[j] = pack_bf16x2(a, b);
+        }
+        RA_TMEM_ST16(tS + q * 16, pk);
+      }
+      l = l * alpha + rs;
+      if (!first && __any_sync(0xffffffffu, need)) {
+        // O_row *= alpha (exactly 1.0 for rows that keep their reference)
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t o[32];
+          RA_TMEM_LD32(tO + c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+          RA_TMEM_ST32(tO + c, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&ctrl->p_full[tile]);
+      first = false;
+    }
+
+    if (ok && !first) {
+      ok = warp_wait(&ctrl->o_full[tile], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        const float inv_l = valid ? 1.f / l : 0.f;
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) +
+                              ((int64_t)(base + sq) * p.heads + it.h) * D;
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t o[32];
+          RA_TMEM_LD32(tO + c, o);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            pk[j] = pack_bf16x2(__uint_as_float(o[2 * j]) * inv_l,
+                                __uint_as_float(o[2 * j + 1]) * inv_l);
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          }
+        }
+        if (valid) {
+          const int64_t li = (int64_t)it.b * p.lse_seq_stride +
+                             (int64_t)it.h * p.lse_head_stride + (p.cu_seqlens ? base : 0) + sq;
+          p.lse[li] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
+        }
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) latch_status(p.status, ST_TIMEOUT);
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kTcMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) !=
+            cudaSuccess ||
+        qres != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// [rows, heads, D] bf16 view with the given row stride; box 64 x 1 x 128.
+static bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int heads, int D,
+                     int64_t tok_stride) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)tok_stride * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)kTcBM};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D>
+static cudaError_t launch_tc_t(const FwdParams& p, cudaStream_t stream) {
+  using C = TcCfg<D>;
+  FwdParams pp = p;
+  pp.n_qranges = (p.seqlen + kTcBM * kTcQT - 1) / (kTcBM * kTcQT);
+  const int64_t grid = work_grid(pp, kTcBM * kTcQT);
+  if (grid == 0) return cudaSuccess;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  TcMaps maps;
+  if (!make_map(&maps.q, p.q, p.total_rows, p.heads, D, p.tok_stride) ||
+      !make_map(&maps.k, p.k, p.total_rows, p.heads, D, p.tok_stride) ||
+      !make_map(&maps.v, p.v, p.total_rows, p.heads, D, p.tok_stride))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  fwd_tc_kernel<D><<<(unsigned)grid, kTcThreads, C::kSmemBytes, stream>>>(pp, maps);
+  return cudaGetLastError();
+}
+
+// bf16 inputs, d_head 64 or 128.
+cudaError_t launch_fwd_tc(const FwdParams& p, cudaStream_t stream) {
+  switch (p.d_head) {
+    case 64: return launch_tc_t<64>(p, stream);
+    case 128: return launch_tc_t<128>(p, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ra

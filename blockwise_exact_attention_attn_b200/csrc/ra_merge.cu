@@ -1,0 +1,199 @@
+// ra_merge.cu -- fold a partial attention result (out_b, lse_b) into
+// (out_a, lse_a) in place.
+//
+// The issue thread "A ring attention with flash attention kernel
+// implementation" explains that the returned log-sum-exp is what makes
+// blockwise evaluation possible (partial results over disjoint key sets are
+// combined through it), and that a key/value-outer ring pass stores outputs
+// and lse and passes them back in.  The combination used here is the stable
+// log-add-exp:
+//     lse = hi + log1p(exp(lo - hi)),   hi/lo = max/min(lse_a, lse_b)
+//     out = exp(lse_a - lse) * out_a + exp(lse_b - lse) * out_b
+// with the empty-side cases handled exactly.
+//
+// Memory-bound: every 16-byte chunk of out_a/out_b is read once and out_a
+// written once; one warp covers whole rows (d_head * sizeof(T) / 16 chunks per
+// row divides 32), so the row's lse is read by its lanes before lane 0 of the
+// row overwrites it (separated by __syncwarp).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "ra_common.cuh"
+
+namespace ra {
+
+// Division of 32-bit unsigned n by a fixed divisor d >= 1 with one high
+// multiply (Granlund & Montgomery, "Division by invariant integers using
+// multiplication", PLDI 1994): with l = ceil(log2 d) and
+// m = floor(2^32 (2^l - d) / d) + 1, n / d = (t + ((n - t) >> 1)) >> (l - 1)
+// where t = mulhi(m, n) (l = 0, i.e. d = 1, is handled separately).
+struct FastDiv {
+  uint32_t d, m, sh;
+  void init(uint32_t div) {
+    d = div;
+    uint32_t l = 0;
+    while ((1ull << l) < div) ++l;
+    sh = l;
+    m = l == 0 ? 0u : (uint32_t)((((1ull << l) - div) << 32) / div + 1);
+  }
+  __device__ __forceinline__ uint32_t div(uint32_t n) const {
+    if (sh == 0) return n;
+    const uint32_t t = __umulhi(m, n);
+    return (t + ((n - t) >> 1)) >> (sh - 1);
+  }
+};
+
+struct MergeParams {
+  void* out_a;
+  float* lse_a;
+  const void* out_b;
+  const float* lse_b;
+  int batch, heads, seqlen, d_head;
+  int64_t rows;     // batch * seqlen * heads (< 2^31, checked by the host)
+  int log2_chunks;  // 16-byte chunks per row = 1 << log2_chunks (divides 32)
+  FastDiv div_heads, div_seqlen;
+};
+
+__device__ __forceinline__ void merge_weights(float la, float lb, float* wa, float* wb,
+                                              float* lse) {
+  const bool ea = la == -INFINITY, eb = lb == -INFINITY;
+  if (ea && eb) { *wa = 0.f; *wb = 0.f; *lse = -INFINITY; return; }
+  if (ea) { *wa = 0.f; *wb = 1.f; *lse = lb; return; }
+  if (eb) { *wa = 1.f; *wb = 0.f; *lse = la; return; }
+  const float hi = fmaxf(la, lb), lo = fminf(la, lb);
+  const float s = hi + log1pf(expf(lo - hi));
+  *wa = expf(la - s);
+  *wb = expf(lb - s);
+  *lse = s;
+}
+
+// fp32: a chunk is 4 floats
+__device__ __forceinline__ void combine_chunk(float4* a, const float4* b, float wa, float wb,
+                                              bool b_only, bool a_only) {
+  float4 x = *a;
+  const float4 y = __ldcs(b);
+  float4 r;
+  if (b_only) {
+    r = y;
+  } else if (a_only) {
+    r = x;
+  } else {
+    r.x = wa * x.x + wb * y.x;
+    r.y = wa * x.y + wb * y.y;
+    r.z = wa * x.z + wb * y.z;
+    r.w = wa * x.w + wb * y.w;
+  }
+  __stcs(a, r);
+}
+
+// bf16: a chunk is 8 values held in a uint4
+__device__ __forceinline__ void combine_chunk_bf16(uint4* a, const uint4* b, float wa, float wb,
+                                                   bool b_only, bool a_only) {
+  uint4 x = *a;
+  const uint4 y = __ldcs(b);
+  uint4 r;
+  if (b_only) {
+    r = y;
+  } else if (a_only) {
+    r = x;
+  } else {
+    const __nv_bfloat162* xa = reinterpret_cast<const __nv_bfloat162*>(&x);
+    const __nv_bfloat162* yb = reinterpret_cast<const __nv_bfloat162*>(&y);
+    __nv_bfloat162* rr = reinterpret_cast<__nv_bfloat162*>(&r);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 fa = __bfloat1622float2(xa[i]);
+      const float2 fb = __bfloat1622float2(yb[i]);
+      rr[i] = __floats2bfloat162_rn(wa * fa.x + wb * fb.x, wa * fa.y + wb * fb.y);
+    }
+  }
+  __stcs(a, r);
+}
+
+template <bool kBf16>
+__global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
+  const int64_t total = p.rows << p.log2_chunks;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t wbase = warp0 * 32; wbase < total; wbase += nwarps * 32) {
+    const int64_t chunk = wbase + lane;
+    const bool live = chunk < total;
+    int c = 0;
+    int64_t li = 0;
+    float la = 0.f, lb = 0.f;
+    if (live) {
+      const uint32_t row = (uint32_t)(chunk >> p.log2_chunks);
+      c = (int)(chunk & ((1 << p.log2_chunks) - 1));
+      // out rows are [batch, seqlen, heads]; lse is [batch, heads, seqlen]
+      const uint32_t bs = p.div_heads.div(row);
+      const uint32_t h = row - bs * (uint32_t)p.heads;
+      const uint32_t b = p.div_seqlen.div(bs);
+      const uint32_t s = bs - b * (uint32_t)p.seqlen;
+      li = ((int64_t)b * p.heads + h) * p.seqlen + s;
+      la = p.lse_a[li];
+      lb = __ldcs(p.lse_b + li);
+    }
+    __syncwarp();
+    if (live) {
+      float wa, wb, lse;
+      merge_weights(la, lb, &wa, &wb, &lse);
+      const bool b_only = la == -INFINITY && lb != -INFINITY;
+      const bool a_only = lb == -INFINITY;
+      if (kBf16) {
+        uint4* a = reinterpret_cast<uint4*>(p.out_a) + chunk;
+        const uint4* b = reinterpret_cast<const uint4*>(p.out_b) + chunk;
+        if (la == -INFINITY && lb == -INFINITY) {
+          __stcs(a, make_uint4(0u, 0u, 0u, 0u));
+        } else {
+          combine_chunk_bf16(a, b, wa, wb, b_only, a_only);
+        }
+      } else {
+        float4* a = reinterpret_cast<float4*>(p.out_a) + chunk;
+        const float4* b = reinterpret_cast<const float4*>(p.out_b) + chunk;
+        if (la == -INFINITY && lb == -INFINITY) {
+          __stcs(a, make_float4(0.f, 0.f, 0.f, 0.f));
+        } else {
+          combine_chunk(a, b, wa, wb, b_only, a_only);
+        }
+      }
+      if (c == 0) p.lse_a[li] = lse;
+    }
+  }
+}
+
+// dtype: 0 = fp32, 1 = bf16.  The host checks that the chunks per row are a
+// power of two dividing 32 and that rows < 2^31.
+cudaError_t launch_merge(void* out_a, float* lse_a, const void* out_b, const float* lse_b,
+                         int batch, int heads, int seqlen, int d_head, int dtype,
+                         int num_sms, cudaStream_t stream) {
+  MergeParams p;
+  p.out_a = out_a;
+  p.lse_a = lse_a;
+  p.out_b = out_b;
+  p.lse_b = lse_b;
+  p.batch = batch;
+  p.heads = heads;
+  p.seqlen = seqlen;
+  p.d_head = d_head;
+  p.rows = (int64_t)batch * seqlen * heads;
+  const int chunks = d_head * (dtype == 0 ? 4 : 2) / 16;
+  p.log2_chunks = 0;
+  while ((1 << p.log2_chunks) < chunks) ++p.log2_chunks;
+  p.div_heads.init((uint32_t)heads);
+  p.div_seqlen.init((uint32_t)seqlen);
+  const int64_t total = p.rows * chunks;
+  if (total == 0) return cudaSuccess;
+  const int threads = 256;
+  // a few resident blocks per SM, whole grid a multiple of the SM count
+  int64_t blocks = (int64_t)num_sms * 8;
+  const int64_t need = (total + threads - 1) / threads;
+  if (need < blocks) blocks = need;
+  if (dtype == 0)
+    merge_kernel<false><<<(unsigned)blocks, threads, 0, stream>>>(p);
+  else
+    merge_kernel<true><<<(unsigned)blocks, threads, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace ra

@@ -1,0 +1,55 @@
+// ra_params.h -- launch parameters shared by the host API and the kernels.
+#pragma once
+
+#include <stdint.h>
+
+namespace ra {
+
+// One forward call, in the form every forward kernel consumes.  Rows of all
+// sequences are addressed as one token axis: token row r of sequence b is
+// global row seq_base(b) + r, with seq_base(b) = b * seqlen (dense) or
+// cu_seqlens[b] (varlen).
+struct FwdParams {
+  const void* q;            // element (row, h, d) at q + row*tok_stride + h*d_head + d
+  const void* k;
+  const void* v;
+  int64_t tok_stride;       // elements between consecutive rows of q/k/v
+  void* out;                // [rows, heads, d_head], same dtype as q
+  float* lse;               // see lse_seq_stride / lse_head_stride
+  int64_t lse_seq_stride;   // dense: heads*seqlen; varlen: 0
+  int64_t lse_head_stride;  // dense: seqlen;       varlen: total rows
+  const int32_t* cu_seqlens;  // NULL for dense
+  int batch, heads, seqlen, d_head;
+  int n_ring, layout, causal, passes;
+  int total_rows;           // rows of q/k/v/out (dense: batch*seqlen)
+  int n_qranges;            // query ranges per sequence (ceil(seqlen / rows per CTA))
+  int longest_first;        // visit query ranges from the last to the first
+  float scale;              // softmax scale
+  float scale_log2;         // scale * log2(e)
+  int* status;              // device status word (never NULL at launch)
+};
+
+// Map a linear CTA index to (query range, batch, head).  The query range is
+// the slowest index so that, with longest_first, the heaviest causal ranges of
+// every (batch, head) are dispatched first.
+struct WorkItem {
+  int qr, b, h;
+};
+
+#if defined(__CUDACC__)
+__host__ __device__ __forceinline__
+#else
+inline
+#endif
+WorkItem decode_work(const FwdParams& p, int64_t w) {
+  WorkItem it;
+  const int64_t bh = (int64_t)p.batch * p.heads;
+  int qr = (int)(w / bh);
+  const int64_t rem = w - (int64_t)qr * bh;
+  it.b = (int)(rem / p.heads);
+  it.h = (int)(rem - (int64_t)it.b * p.heads);
+  it.qr = p.longest_first ? (p.n_qranges - 1 - qr) : qr;
+  return it;
+}
+
+}  // namespace ra

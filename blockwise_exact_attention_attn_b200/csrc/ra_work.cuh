@@ -1,0 +1,101 @@
+// ra_work.cuh -- map a CTA to its work item (sequence, query range, head).
+//
+// Dense inputs: CTA index w -> (query range, batch, head) with the query
+// range slowest, so that with longest_first the heaviest causal ranges of
+// every (batch, head) start first.
+// Varlen inputs (cu_seqlens, "Tensorflow flash attention" page: cumulative
+// sequence lengths of shape (batch_size + 1,) index ragged, unpadded
+// tensors): CTA index w -> (flat range, head) with the head fastest; the flat
+// range is located among the sequences by a warp-wide scan of their range
+// counts ceil(L_b / rows_per_cta), and inside a sequence the ranges run from
+// the last to the first when longest_first.
+#pragma once
+
+#include <stdint.h>
+
+#include "ra_common.cuh"
+#include "ra_params.h"
+
+namespace ra {
+
+struct SeqWork {
+  int b, qr, h;   // sequence, query range within it, head
+  int base;       // global row of the sequence's first token
+  int L;          // sequence length
+  bool live;      // false: nothing to do for this CTA
+};
+
+// Must be called by all 32 lanes of a warp (any warp; every warp of a CTA
+// computes the same answer).  Latches ST_INVALID for malformed cu_seqlens.
+__device__ __forceinline__ SeqWork find_work(const FwdParams& p, int rows_per_cta) {
+  SeqWork w;
+  w.live = false;
+  w.b = w.qr = w.h = w.base = w.L = 0;
+  const int lane = threadIdx.x & 31;
+  if (!p.cu_seqlens) {
+    const WorkItem it = decode_work(p, blockIdx.x);
+    w.b = it.b;
+    w.qr = it.qr;
+    w.h = it.h;
+    w.base = it.b * p.seqlen;
+    w.L = p.seqlen;
+    w.live = (int64_t)it.qr * rows_per_cta < p.seqlen;
+    return w;
+  }
+  const int flat = blockIdx.x / p.heads;
+  w.h = blockIdx.x - flat * p.heads;
+  if (lane == 0 && threadIdx.x == 0 && blockIdx.x == 0 &&
+      (p.cu_seqlens[0] != 0 || p.cu_seqlens[p.batch] != p.total_rows))
+    latch_status(p.status, ST_INVALID);
+  int acc = 0;
+  for (int b0 = 0; b0 < p.batch; b0 += 32) {
+    const int b = b0 + lane;
+    int n = 0, s0 = 0, len = 0;
+    if (b < p.batch) {
+      s0 = p.cu_seqlens[b];
+      const int s1 = p.cu_seqlens[b + 1];
+      len = s1 - s0;
+      if (s0 < 0 || len < 0 || s1 > p.total_rows) {
+        if (w.h == 0 && flat == 0) latch_status(p.status, ST_INVALID);
+        len = 0;
+      }
+      n = (len + rows_per_cta - 1) / rows_per_cta;
+    }
+    int incl = n;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    const int excl = incl - n;
+    const bool mine = n > 0 && flat >= acc + excl && flat < acc + incl;
+    const unsigned hit = __ballot_sync(0xffffffffu, mine);
+    if (hit) {
+      const int src = __ffs(hit) - 1;
+      w.b = __shfl_sync(0xffffffffu, b, src);
+      w.base = __shfl_sync(0xffffffffu, s0, src);
+      w.L = __shfl_sync(0xffffffffu, len, src);
+      const int nq = __shfl_sync(0xffffffffu, n, src);
+      const int qi = flat - acc - __shfl_sync(0xffffffffu, excl, src);
+      w.qr = p.longest_first ? nq - 1 - qi : qi;
+      w.live = true;
+      return w;
+    }
+    acc += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  return w;
+}
+
+// Launch size: dense n_qranges * batch * heads; varlen (ceil(total /
+// rows_per_cta) + batch) * heads, an upper bound of the ranges of all
+// sequences.
+inline int64_t work_grid(const FwdParams& p, int rows_per_cta) {
+  if (!p.cu_seqlens) {
+    const int64_t nq = ((int64_t)p.seqlen + rows_per_cta - 1) / rows_per_cta;
+    return nq * p.batch * p.heads;
+  }
+  const int64_t nq = ((int64_t)p.total_rows + rows_per_cta - 1) / rows_per_cta + p.batch;
+  return nq * p.heads;
+}
+
+}  // namespace ra

@@ -1,0 +1,92 @@
+"""The C-ABI library loads, exports every entry point include/ring_attn.h
+declares, and rejects bad arguments on the host before touching CUDA (these
+calls never reach a kernel, so they run without a GPU)."""
+
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+import blockwise_exact_attention_attn_b200 as ra
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                      "include", "ring_attn.h")
+
+# an aligned, never-dereferenced fake device address
+FAKE = 0x10000
+
+
+def declared_functions():
+    with open(HEADER) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ring_attn_\w+)\s*\(", text)))
+
+
+def test_header_and_export_list_agree():
+    assert declared_functions() == sorted(ra.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code, name in enumerate(["RA_OK", "RA_ERR_INVALID", "RA_ERR_UNSUPPORTED", "RA_ERR_CUDA",
+                                 "RA_ERR_TIMEOUT"]):
+        assert lib.ring_attn_status_string(code).decode() == name
+    assert lib.ring_attn_status_string(99).decode() == "RA_ERR_UNKNOWN"
+
+
+def fwd(lib, **over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, batch=1, heads=2, seqlen=256, d_head=128,
+             n=4, layout=0, causal=1, scale=0.1, passes=4, cu=None, dtype=1, stream=None)
+    a.update(over)
+    return lib.ring_attn_fwd(a["q"], a["k"], a["v"], a["out"], a["lse"], a["batch"], a["heads"],
+                             a["seqlen"], a["d_head"], a["n"], a["layout"], a["causal"],
+                             a["scale"], a["passes"], a["cu"], a["dtype"], a["stream"])
+
+
+@pytest.mark.parametrize("over", [
+    dict(q=None), dict(k=None), dict(v=None), dict(out=None), dict(lse=None),
+    dict(q=FAKE + 4), dict(out=FAKE + 8), dict(lse=FAKE + 2),
+    dict(batch=0), dict(heads=0), dict(seqlen=0), dict(n=0), dict(passes=0),
+    dict(seqlen=250),                    # dense seqlen not a multiple of N
+    dict(d_head=48), dict(d_head=0), dict(layout=2), dict(causal=2), dict(dtype=5),
+    dict(scale=math.inf), dict(scale=math.nan), dict(cu=FAKE + 2),
+])
+def test_fwd_rejects_invalid_arguments(lib, over):
+    assert fwd(lib, **over) == ra.RA_ERR_INVALID
+
+
+def test_qkvpacked_and_simt_reject_invalid_arguments(lib):
+    st = lib.ring_attn_qkvpacked_fwd(None, FAKE, FAKE, 1, 2, 256, 128, 4, 0, 1, 0.1, 4, None, 1,
+                                     None)
+    assert st == ra.RA_ERR_INVALID
+    st = lib.ring_attn_fwd_simt(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 256, 100, 4, 0, 1, 0.1, 4,
+                                None, 0, None)
+    assert st == ra.RA_ERR_INVALID
+
+
+@pytest.mark.parametrize("args", [
+    (None, FAKE, FAKE, FAKE, 1, 1, 8, 128, 0),         # null
+    (FAKE, FAKE + 4, FAKE, FAKE, 1, 1, 8, 128, 0),     # misaligned lse
+    (FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 3, 0),           # row not whole 16-byte chunks
+    (FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 256, 0),         # fp32 row of 64 chunks (> 32)
+    (FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 24, 1),          # 3 chunks: not a power of two
+    (FAKE, FAKE, FAKE, FAKE, 0, 1, 8, 128, 0),         # empty batch
+    (FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 128, 7),         # dtype
+])
+def test_merge_rejects_invalid_arguments(lib, args):
+    assert lib.ring_attn_merge(*args, None) == ra.RA_ERR_INVALID
+
+
+def test_binding_refuses_host_tensors():
+    import torch
+    x = torch.zeros(1, 128, 1, 64, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 1, 128)
+    with pytest.raises(ValueError):
+        ra.ring_attn_fwd(x, x, x, x, lse, 1, 1, 128, 64, 1)

@@ -221,22 +221,42 @@ def make_step(w, dev):
     return step, lens, in_bytes, out_bytes, (inp, out, lse)
 
 
-def time_steps(step, steps, warmup, dist, dev):
+def time_steps(step, steps, warmup, dist, dev, graph=False):
+    """Device time of `steps` calls (CUDA events on the launching stream,
+    synchronized and barriered on both sides, max over ranks).  With graph,
+    the calls are captured once into a CUDA graph that is replayed for the
+    timed region, so host launch overhead does not pace small kernels."""
     for _ in range(warmup):
         step()
     torch.cuda.synchronize(dev)
+    g = None
+    if graph:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                for _ in range(steps):
+                    step()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        g.replay()  # one untimed replay
+        torch.cuda.synchronize(dev)
     dist.barrier()
     torch.cuda.synchronize(dev)
     stream = torch.cuda.current_stream(dev)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(steps):
-        step()
+    if g is not None:
+        g.replay()
+    else:
+        for _ in range(steps):
+            step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     dist.barrier()
     ms = e0.elapsed_time(e1)
+    del g
     return dist.max(ms)
 
 
@@ -246,7 +266,7 @@ def measure_workload(name, steps, warmup, dist, dev, peaks):
     w = gen.WORKLOADS[name]
     step, lens, in_bytes, out_bytes, keep = make_step(w, dev)
     flops = workload_flops(w, lens)
-    ms = time_steps(step, steps, warmup, dist, dev)
+    ms = time_steps(step, steps, warmup, dist, dev, graph=True)
     st = ra.ring_attn_status()
     if st != ra.RA_OK:
         raise RuntimeError(f"{name}: device status {ra.ring_attn_status_string(st)}")
@@ -276,7 +296,7 @@ def measure_merge(steps, warmup, dist, dev, peaks):
     def step():
         ra.ring_attn_merge(oa, la, ob, lb, B, H, S, D)
 
-    ms = time_steps(step, max(steps, 20), warmup, dist, dev)
+    ms = time_steps(step, max(steps, 20), warmup, dist, dev, graph=True)
     per = ms / max(steps, 20)
     nbytes = 3 * oa.numel() * 4 + 3 * la.numel() * 4
     gbs = nbytes / (per * 1e-3) / 1e9
@@ -467,7 +487,8 @@ def run_ours(args, dist):
                    "n_ring_blocks": w.n_ring, "layout": "striped" if w.layout else "contiguous",
                    "max_ring_passes": w.passes,
                    "parallelism": f"{dist.world} independent replicas",
-                   "l2": f"no flush: inputs {in_bytes / 2**20:.0f} MiB > L2 126 MiB"},
+                   "l2": f"no flush: inputs {in_bytes / 2**20:.0f} MiB > L2 126 MiB",
+                   "timing": "CUDA graph of the timed launches, CUDA events"},
         "pct_of_peak": 100.0 * value / dist.world / peak if peak else None,
         "roofline": {"bound": "tensor", "achieved": value / dist.world, "peak": peak,
                      "unit": "TFLOP/s", "frac": value / dist.world / peak if peak else None,

@@ -125,30 +125,31 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // S = Q K^T for one query tile: M = 128 rows, N = 128 keys, K = D in steps of
-// 16.  Both operands K-major in 128-byte-swizzled panels of 64 elements.
+// 16.  Both operands K-major in 128-byte-swizzled panels of 64 elements; the
+// descriptors of step kk are the tile's base descriptors plus a constant
+// (start address field, in 16-byte units: panel * 1024 + 2 * (kk % 4)).
 template <int D>
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t qbase, uint32_t kbase,
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t qdesc, uint64_t kdesc,
                                          uint32_t idesc) {
   using C = TcCfg<D>;
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-    umma_ss(d_tmem, smem_desc_sw128(qbase + off, 16, 1024),
-            smem_desc_sw128(kbase + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+    const uint64_t off = (uint64_t)((kk >> 2) * (C::kPanelBytes >> 4) + (kk & 3) * 2);
+    umma_ss(d_tmem, qdesc + off, kdesc + off, idesc, kk > 0 ? 1u : 0u);
   }
 }
 
 // O (+)= P V for one query tile: A = P from tensor memory (128 x 128 bf16,
 // 8 columns per 16 keys), B = V tile MN-major (N = D split in 64-element
-// panels, LBO = panel stride; 8-key groups 1024 bytes apart).
+// panels, LBO = panel stride; 8-key groups 1024 bytes apart); step kk starts
+// 16 keys (2048 bytes, 128 units) further.
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t vbase,
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t vdesc,
                                          uint32_t idesc, bool accumulate) {
-  using C = TcCfg<D>;
 #pragma unroll
   for (int kk = 0; kk < kTcBN / 16; ++kk) {
-    umma_ts(d_tmem, p_tmem + kk * 8, smem_desc_sw128(vbase + kk * 16 * 128, C::kPanelBytes, 1024),
-            idesc, (accumulate || kk > 0) ? 1u : 0u);
+    umma_ts(d_tmem, p_tmem + kk * 8, vdesc + (uint64_t)(kk * 128), idesc,
+            (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -362,8 +363,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint32_t idesc_s =
           idesc_bf16_f32(kTcBM, kTcBN, 0) | (p.scale_log2 < 0.f ? (1u << 13) : 0u);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kTcBM, D, 1);
+      // base descriptors: K-major tiles (Q, K) and MN-major tiles (V)
       const uint32_t qs = smem_u32(smem + C::kQOff);
       const uint32_t kvs = smem_u32(smem + C::kKVOff);
+      uint64_t qdesc[kTcQT];
+#pragma unroll
+      for (int i = 0; i < kTcQT; ++i) qdesc[i] = smem_desc_sw128(qs + i * C::kTileBytes, 16, 1024);
+      const uint64_t kdesc0 = smem_desc_sw128(kvs, 16, 1024);
+      const uint64_t vdesc0 = smem_desc_sw128(kvs, C::kPanelBytes, 1024);
+      constexpr uint64_t kSlotStep = (uint64_t)(C::kTileBytes >> 4);
       bool ok = mbar_wait(&ctrl->q_full, 0, abort_flag);
       tc_fence_after();
       uint32_t pphase[kTcQT] = {0, 0};
@@ -380,8 +388,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tc_fence_after();
           for (int i = 0; i < kTcQT; ++i)
             if (entry_cls(e, i) != CLS_EMPTY) {
-              issue_qk<D>(tmem + C::kColS + i * kTcBN, qs + i * C::kTileBytes,
-                          kvs + slot * C::kTileBytes, idesc_s);
+              issue_qk<D>(tmem + C::kColS + i * kTcBN, qdesc[i], kdesc0 + slot * kSlotStep,
+                          idesc_s);
               umma_commit(&ctrl->s_full[i]);
             }
           umma_commit(&ctrl->kv_empty[slot]);
@@ -411,12 +419,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               if (!ok) break;
               tc_fence_after();
               issue_pv<D>(tmem + C::kColO + i * D, tmem + C::kColS + i * kTcBN,
-                          kvs + slot_v * C::kTileBytes, idesc_o, started[i]);
+                          vdesc0 + slot_v * kSlotStep, idesc_o, started[i]);
               started[i] = true;
             }
             if (has && entry_cls(e, i) != CLS_EMPTY) {
-              issue_qk<D>(tmem + C::kColS + i * kTcBN, qs + i * C::kTileBytes,
-                          kvs + slot_k * C::kTileBytes, idesc_s);
+              issue_qk<D>(tmem + C::kColS + i * kTcBN, qdesc[i], kdesc0 + slot_k * kSlotStep,
+                          idesc_s);
               umma_commit(&ctrl->s_full[i]);
             }
           }
@@ -489,9 +497,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (cls == CLS_PARTIAL || nk < kTcBN) {
         apply_mask(x, p, L, valid, cls, sq, rq, tq, k0, nk);
       }
-      float mx = x[0];
+      // row max as a tree of independent maxima (short dependency chains)
+      float mx8[8];
 #pragma unroll
-      for (int c = 1; c < kTcBN; ++c) mx = fmaxf(mx, x[c]);
+      for (int j = 0; j < 8; ++j) mx8[j] = x[j];
+#pragma unroll
+      for (int c = 8; c < kTcBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_tile = mx * sl2;  // -inf stays -inf (sl2 > 0)
       const bool need = m_tile > m_ref + kRescaleLog2;
       float alpha = 1.f;
@@ -500,7 +513,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         m_ref = m_tile;
       }
       const float msub = m_ref == -INFINITY ? 0.f : m_ref;
-      float rs = 0.f;
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial row sums
 #pragma unroll
       for (int q = 0; q < kTcBN / 32; ++q) {
         uint32_t pk[16];
@@ -508,12 +521,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int j = 0; j < 16; ++j) {
           const float a = ex2_approx(fmaf(x[q * 32 + 2 * j], sl2, -msub));
           const float b = ex2_approx(fmaf(x[q * 32 + 2 * j + 1], sl2, -msub));
-          rs += a + b;
+          rs4[j & 3] += a + b;
           pk[j] = pack_bf16x2(a, b);
         }
         RA_TMEM_ST16(tS + q * 16, pk);
       }
-      l = l * alpha + rs;
+      l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
       if (!first && __any_sync(0xffffffffu, need)) {
         // O_row *= alpha (exactly 1.0 for rows that keep their reference)
 #pragma unroll

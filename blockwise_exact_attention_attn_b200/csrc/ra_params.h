@@ -29,9 +29,10 @@ struct FwdParams {
   int* status;              // device status word (never NULL at launch)
 };
 
-// Map a linear CTA index to (query range, batch, head).  The query range is
-// the slowest index so that, with longest_first, the heaviest causal ranges of
-// every (batch, head) are dispatched first.
+// Map a linear CTA index to (query range, batch, head).  The (batch, head)
+// pair is the slowest index, so the CTAs resident at one time share the K/V
+// of a few heads in L2; inside a head the query ranges run from the last to
+// the first with longest_first (heaviest causal ranges first).
 struct WorkItem {
   int qr, b, h;
 };
@@ -43,11 +44,10 @@ inline
 #endif
 WorkItem decode_work(const FwdParams& p, int64_t w) {
   WorkItem it;
-  const int64_t bh = (int64_t)p.batch * p.heads;
-  int qr = (int)(w / bh);
-  const int64_t rem = w - (int64_t)qr * bh;
-  it.b = (int)(rem / p.heads);
-  it.h = (int)(rem - (int64_t)it.b * p.heads);
+  const int64_t bh = w / p.n_qranges;
+  const int qr = (int)(w - bh * p.n_qranges);
+  it.b = (int)(bh / p.heads);
+  it.h = (int)(bh - (int64_t)it.b * p.heads);
   it.qr = p.longest_first ? (p.n_qranges - 1 - qr) : qr;
   return it;
 }

@@ -56,18 +56,25 @@ RA_HD RingGeom make_geom(int L, int N, int layout, int causal, int P) {
   return g;
 }
 
+// floor((a * b + c) / d) for non-negative a, b, c and positive d; 32-bit
+// arithmetic whenever the numerator fits (64-bit division is slow on the GPU).
+RA_HD int muladd_div(int a, int b, int c, int d) {
+  const uint64_t num = (uint64_t)(uint32_t)a * (uint32_t)b + (uint32_t)c;
+  if (num <= 0xffffffffull) return (int)((uint32_t)num / (uint32_t)d);
+  return (int)(num / (uint64_t)d);
+}
+
 // First stored row of ring block r (r in [0, N]; r == N gives L).
 //   contiguous: block r = rows t with floor(t*N/L) == r, i.e. [ceil(rL/N), ..)
 //   striped   : blocks hold ceil((L - r)/N) rows each, stored in order.
 RA_HD int block_start(const RingGeom& g, int r) {
-  if (g.layout == LAYOUT_CONTIGUOUS)
-    return (int)(((int64_t)r * g.L + g.N - 1) / g.N);
+  if (g.layout == LAYOUT_CONTIGUOUS) return muladd_div(r, g.L, g.N - 1, g.N);
   return r * g.q + (r < g.rem ? r : g.rem);
 }
 
 // Ring block of stored row s (0 <= s < L).
 RA_HD int block_of(const RingGeom& g, int s) {
-  if (g.layout == LAYOUT_CONTIGUOUS) return (int)(((int64_t)s * g.N) / g.L);
+  if (g.layout == LAYOUT_CONTIGUOUS) return muladd_div(s, g.N, 0, g.L);
   const int big = g.rem * (g.q + 1);  // rows held by the blocks of q+1 rows
   if (s < big) return s / (g.q + 1);
   return g.rem + (s - big) / g.q;     // here q >= 1 because s < L
@@ -152,9 +159,62 @@ RA_HD bool allowed(const RingGeom& g, int sq, int rq, int tq, int sk) {
 // [q0, qm) and [qm, q1)) are classified per tile, so a CTA that owns two
 // q-tiles can share one walk; a tile is emitted when it is non-EMPTY for at
 // least one sub-range.
+// Query segments (one per ring block) of a query sub-range, cached by the
+// walk so that the tiles lying inside one key block are classified without
+// any division.
+constexpr int kMaxQSegs = 4;
+struct QSegs {
+  int n;                      // segments, or -1 when there are too many
+  int r[kMaxQSegs];           // ring block
+  int a[kMaxQSegs], b[kMaxQSegs];  // stored rows [a, b)
+  int start[kMaxQSegs];       // first stored row of block r
+};
+
+RA_HD void make_qsegs(const RingGeom& g, int lo, int hi, QSegs* s) {
+  s->n = 0;
+  if (lo >= hi) return;
+  const int r0 = block_of(g, lo), r1 = block_of(g, hi - 1);
+  if (r1 - r0 + 1 > kMaxQSegs) { s->n = -1; return; }
+  for (int r = r0; r <= r1; ++r) {
+    const int bs = block_start(g, r), be = block_start(g, r + 1);
+    const int a = lo > bs ? lo : bs, b = hi < be ? hi : be;
+    if (a >= b) continue;
+    s->r[s->n] = r;
+    s->a[s->n] = a;
+    s->b[s->n] = b;
+    s->start[s->n] = bs;
+    ++s->n;
+  }
+}
+
+// Class of query segments `s` against key rows [c, d) that lie inside key
+// block rk starting at row ks (same rules as classify_segment).
+RA_HD int classify_in_block(const RingGeom& g, const QSegs& s, int rk, int ks, int c, int d) {
+  bool any = false, all = true;
+  for (int i = 0; i < s.n; ++i) {
+    const int rq = s.r[i];
+    if (!pass_ok(g, rq, rk)) { all = false; continue; }
+    if (!g.causal) { any = true; continue; }
+    if (g.layout == LAYOUT_CONTIGUOUS) {
+      if (c <= s.b[i] - 1) any = true;
+      if (!(d - 1 <= s.a[i])) all = false;
+    } else {
+      const int delta = rk > rq ? 1 : 0;
+      const int ia = s.a[i] - s.start[i], ib = s.b[i] - s.start[i];
+      const int ja = c - ks, jb = d - ks;
+      if (ja <= ib - 1 - delta) any = true;
+      if (!(jb - 1 <= ia - delta)) all = false;
+    }
+  }
+  if (!any) return CLS_EMPTY;
+  return all ? CLS_FULL : CLS_PARTIAL;
+}
+
 struct TileWalk {
   RingGeom g;
   int q0, qm, q1;   // sub-range 0 = [q0, qm), sub-range 1 = [qm, q1)
+  QSegs seg0, seg1; // their per-block segments
+  int kbs, kbe;     // stored rows of the current key block
   int BN;
   int rq_ref;       // ring block of q0
   int rqa, rqb;     // ring blocks spanned by [q0, q1)
@@ -169,6 +229,9 @@ struct TileWalk {
     g = geom;
     q0 = q_begin; qm = q_mid; q1 = q_end;
     BN = kv_tile;
+    make_qsegs(g, q0, qm, &seg0);
+    make_qsegs(g, qm, q1, &seg1);
+    kbs = kbe = 0;
     rq_ref = block_of(g, q0);
     rqa = rq_ref;
     rqb = block_of(g, q1 - 1);
@@ -215,6 +278,8 @@ struct TileWalk {
       if (rk < 0) rk += g.N;
       const int bs = block_start(g, rk), be = block_start(g, rk + 1);
       if (bs >= be) continue;
+      kbs = bs;
+      kbe = be;
       kt = (bs + BN - 1) / BN;
       const int kt_all = (be + BN - 1) / BN;  // tiles starting in [bs, be)
       if (kt >= kt_all) continue;
@@ -249,19 +314,29 @@ struct TileWalk {
   RA_HD bool next(int* tile, int* cls0, int* cls1) {
     while (true) {
       int t;
+      bool inner;
       if (kt < kt_end) {
         t = kt++;
+        inner = true;
       } else if (kt_cross >= 0) {
         t = kt_cross;
         kt_cross = -1;
+        inner = false;
       } else {
         if (!next_block()) return false;
         continue;
       }
       const int k0 = t * BN;
       const int k1 = (k0 + BN < g.L) ? k0 + BN : g.L;
-      const int c0 = classify(g, q0, qm, k0, k1);
-      const int c1 = classify(g, qm, q1, k0, k1);
+      int c0, c1;
+      if (inner && seg0.n >= 0 && seg1.n >= 0) {
+        // tile inside key block rk: division-free classification
+        c0 = classify_in_block(g, seg0, rk, kbs, k0, k1);
+        c1 = classify_in_block(g, seg1, rk, kbs, k0, k1);
+      } else {
+        c0 = classify(g, q0, qm, k0, k1);
+        c1 = classify(g, qm, q1, k0, k1);
+      }
       if (c0 == CLS_EMPTY && c1 == CLS_EMPTY) continue;
       *tile = t;
       *cls0 = c0;

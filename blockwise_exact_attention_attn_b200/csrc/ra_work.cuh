@@ -1,8 +1,8 @@
 // ra_work.cuh -- map a CTA to its work item (sequence, query range, head).
 //
-// Dense inputs: CTA index w -> (query range, batch, head) with the query
-// range slowest, so that with longest_first the heaviest causal ranges of
-// every (batch, head) start first.
+// Dense inputs: CTA index w -> (batch, head, query range) with the query
+// range fastest, so the CTAs running together share a few heads' K/V in L2;
+// with longest_first a head's heaviest causal ranges start first.
 // Varlen inputs (cu_seqlens, "Tensorflow flash attention" page: cumulative
 // sequence lengths of shape (batch_size + 1,) index ragged, unpadded
 // tensors): CTA index w -> (flat range, head) with the head fastest; the flat

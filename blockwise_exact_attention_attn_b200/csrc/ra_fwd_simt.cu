@@ -12,8 +12,9 @@
 // exponentiated scores and of weighted values, divided at the end).  Here the
 // division by the denominator is deferred to the end, as in the glossary.
 //
-// A query row is served by TPR = d_head / DPT threads, each holding DPT of its
-// dimensions; the dot products are completed with warp shuffles.
+// A query row is served by 8 threads: the row's dimensions are split over
+// d_head / min(d_head, 32) of them (dot products completed with warp
+// shuffles) and its keys over the rest (key lanes merged at the end).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -45,17 +46,31 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
 }
 
+// Thread layout: 8 threads serve one query row, 16 rows per CTA.  The row's
+// dimensions are split over TPRD = D / min(D, 32) threads and its keys over
+// KL = 8 / TPRD key lanes; lane index within the row = kl * TPRD + part.  A
+// thread keeps its own online-softmax state (m, l, O) over the keys of its
+// lane; the lanes are merged at the end (max of m, rescale, sum).
+template <typename T, int D>
+struct SimtShape {
+  static constexpr int DPT = D < 32 ? D : 32;           // dims per thread
+  static constexpr int TPRD = D / DPT;                  // threads per row (dims)
+  static constexpr int KL = 8 / TPRD;                   // key lanes per row
+  static constexpr int ROWS = kSimtThreads / 8;         // query rows per CTA
+  static constexpr int KPL = kSimtBN / KL;              // keys per lane per tile
+  static constexpr int STRIDE = D + 4;                  // smem row stride (floats)
+};
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kSimtThreads)
     fwd_simt_kernel(const FwdParams p) {
-  constexpr int DPT = D < 32 ? D : 32;     // dims per thread
-  constexpr int TPR = D / DPT;             // threads per row
-  constexpr int ROWS = kSimtThreads / TPR; // query rows per CTA
-  constexpr int BN = kSimtBN;
+  using Sh = SimtShape<T, D>;
+  constexpr int DPT = Sh::DPT, TPRD = Sh::TPRD, KL = Sh::KL, ROWS = Sh::ROWS, KPL = Sh::KPL;
+  constexpr int BN = kSimtBN, ST = Sh::STRIDE;
 
   extern __shared__ float smem_f[];
-  float* Ks = smem_f;            // [BN][D]
-  float* Vs = smem_f + BN * D;   // [BN][D]
+  float* Ks = smem_f;             // [BN][ST]
+  float* Vs = smem_f + BN * ST;   // [BN][ST]
 
   const SeqWork it = find_work(p, ROWS);
   if (!it.live) return;  // uniform across the CTA
@@ -64,8 +79,9 @@ __global__ void __launch_bounds__(kSimtThreads)
   const int q1 = min(q0 + ROWS, L);
 
   const int tid = threadIdx.x;
-  const int rloc = tid / TPR;
-  const int part = tid % TPR;
+  const int rloc = tid >> 3;
+  const int part = tid & (TPRD - 1);
+  const int kl = (tid & 7) / TPRD;
   const int sq = q0 + rloc;          // stored row of this thread's query
   const bool valid = sq < L;
 
@@ -88,7 +104,7 @@ __global__ void __launch_bounds__(kSimtThreads)
                   : 0.f;
     o[d] = 0.f;
   }
-  float m = -INFINITY;  // running max, log2 domain (score * scale * log2 e)
+  float m = -INFINITY;  // running max of this lane's keys, log2 domain
   float l = 0.f;        // running denominator relative to m
 
   TileWalk walk;
@@ -107,46 +123,63 @@ __global__ void __launch_bounds__(kSimtThreads)
         kv = to_f32(kg[off]);
         vv = to_f32(vg[off]);
       }
-      Ks[e] = kv;
-      Vs[e] = vv;
+      Ks[c * ST + d] = kv;
+      Vs[c * ST + d] = vv;
     }
     __syncthreads();
 
-    float s[BN];
+    float s[KPL];
     float tile_max = -INFINITY;
 #pragma unroll
-    for (int c = 0; c < BN; ++c) {
-      const float* kr = Ks + c * D + part * DPT;
+    for (int j = 0; j < KPL; ++j) {
+      const int c = kl + KL * j;
+      const float* kr = Ks + c * ST + part * DPT;
       float acc = 0.f;
 #pragma unroll
       for (int d = 0; d < DPT; ++d) acc = fmaf(qr[d], kr[d], acc);
 #pragma unroll
-      for (int off = 1; off < TPR; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      for (int off = 1; off < TPRD; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
       float x = acc * p.scale_log2;
       bool ok = c < nk;
       if (ok && c0 == CLS_PARTIAL && valid) ok = allowed(g, sq, rq, tq, k0 + c);
       x = ok ? x : -INFINITY;
-      s[c] = x;
+      s[j] = x;
       tile_max = fmaxf(tile_max, x);
     }
     const float m_new = fmaxf(m, tile_max);
-    if (m_new == -INFINITY) continue;  // nothing allowed for this row yet
+    if (m_new == -INFINITY) continue;  // nothing allowed for this lane yet
     const float alpha = exp2f(m - m_new);  // 0 when m == -inf
     l *= alpha;
 #pragma unroll
     for (int d = 0; d < DPT; ++d) o[d] *= alpha;
 #pragma unroll
-    for (int c = 0; c < BN; ++c) {
-      const float pc = exp2f(s[c] - m_new);
+    for (int j = 0; j < KPL; ++j) {
+      const float pc = exp2f(s[j] - m_new);
       l += pc;
-      const float* vr = Vs + c * D + part * DPT;
+      const float* vr = Vs + (kl + KL * j) * ST + part * DPT;
 #pragma unroll
       for (int d = 0; d < DPT; ++d) o[d] = fmaf(pc, vr[d], o[d]);
     }
     m = m_new;
   }
 
-  if (!valid) return;
+  // merge the KL key lanes of the row: common maximum, rescale, sum
+  float m_all = m;
+#pragma unroll
+  for (int off = TPRD; off < 8; off <<= 1)
+    m_all = fmaxf(m_all, __shfl_xor_sync(0xffffffffu, m_all, off));
+  const float f = (m == -INFINITY) ? 0.f : exp2f(m - m_all);
+  l *= f;
+#pragma unroll
+  for (int d = 0; d < DPT; ++d) o[d] *= f;
+#pragma unroll
+  for (int off = TPRD; off < 8; off <<= 1) {
+    l += __shfl_xor_sync(0xffffffffu, l, off);
+#pragma unroll
+    for (int d = 0; d < DPT; ++d) o[d] += __shfl_xor_sync(0xffffffffu, o[d], off);
+  }
+
+  if (!valid || kl != 0) return;
   T* og = static_cast<T*>(p.out);
   const float inv_l = 1.f / l;
   const int64_t orow = (int64_t)(base + sq) * p.heads * D + (int64_t)it.h * D + part * DPT;
@@ -156,20 +189,19 @@ __global__ void __launch_bounds__(kSimtThreads)
     const int64_t li = (int64_t)it.b * p.lse_seq_stride + (int64_t)it.h * p.lse_head_stride +
                        (p.cu_seqlens ? base : 0) + sq;
     // lse = ln(l) + m / log2(e), with m in the log2 domain
-    p.lse[li] = (m + log2f(l)) * 0.69314718055994530942f;
+    p.lse[li] = (m_all + log2f(l)) * 0.69314718055994530942f;
   }
 }
 
 template <typename T, int D>
 static cudaError_t launch_simt_t(const FwdParams& p, cudaStream_t stream) {
-  constexpr int DPT = D < 32 ? D : 32;
-  constexpr int ROWS = kSimtThreads / (D / DPT);
+  using Sh = SimtShape<T, D>;
   FwdParams pp = p;
-  pp.n_qranges = (p.seqlen + ROWS - 1) / ROWS;
-  const int64_t grid = work_grid(pp, ROWS);
+  pp.n_qranges = (p.seqlen + Sh::ROWS - 1) / Sh::ROWS;
+  const int64_t grid = work_grid(pp, Sh::ROWS);
   if (grid == 0) return cudaSuccess;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  const size_t smem = 2 * kSimtBN * D * sizeof(float);
+  const size_t smem = 2 * kSimtBN * Sh::STRIDE * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(fwd_simt_kernel<T, D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -161,10 +161,11 @@ RA_HD bool allowed(const RingGeom& g, int sq, int rq, int tq, int sk) {
 // least one sub-range.
 // Query segments (one per ring block) of a query sub-range, cached by the
 // walk so that the tiles lying inside one key block are classified without
-// any division.
+// any division.  Slot k holds ring block r0 + k (empty when a >= b); all
+// loops over slots are unrolled so the arrays stay in registers.
 constexpr int kMaxQSegs = 4;
 struct QSegs {
-  int n;                      // segments, or -1 when there are too many
+  int n;                      // slots in use, or -1 when there are too many blocks
   int r[kMaxQSegs];           // ring block
   int a[kMaxQSegs], b[kMaxQSegs];  // stored rows [a, b)
   int start[kMaxQSegs];       // first stored row of block r
@@ -172,18 +173,27 @@ struct QSegs {
 
 RA_HD void make_qsegs(const RingGeom& g, int lo, int hi, QSegs* s) {
   s->n = 0;
+#pragma unroll
+  for (int k = 0; k < kMaxQSegs; ++k) {
+    s->r[k] = 0;
+    s->a[k] = 0;
+    s->b[k] = 0;
+    s->start[k] = 0;
+  }
   if (lo >= hi) return;
   const int r0 = block_of(g, lo), r1 = block_of(g, hi - 1);
   if (r1 - r0 + 1 > kMaxQSegs) { s->n = -1; return; }
-  for (int r = r0; r <= r1; ++r) {
-    const int bs = block_start(g, r), be = block_start(g, r + 1);
-    const int a = lo > bs ? lo : bs, b = hi < be ? hi : be;
-    if (a >= b) continue;
-    s->r[s->n] = r;
-    s->a[s->n] = a;
-    s->b[s->n] = b;
-    s->start[s->n] = bs;
-    ++s->n;
+  s->n = r1 - r0 + 1;
+#pragma unroll
+  for (int k = 0; k < kMaxQSegs; ++k) {
+    const int r = r0 + k;
+    if (k < s->n) {
+      const int bs = block_start(g, r), be = block_start(g, r + 1);
+      s->r[k] = r;
+      s->a[k] = lo > bs ? lo : bs;
+      s->b[k] = hi < be ? hi : be;
+      s->start[k] = bs;
+    }
   }
 }
 
@@ -191,7 +201,9 @@ RA_HD void make_qsegs(const RingGeom& g, int lo, int hi, QSegs* s) {
 // block rk starting at row ks (same rules as classify_segment).
 RA_HD int classify_in_block(const RingGeom& g, const QSegs& s, int rk, int ks, int c, int d) {
   bool any = false, all = true;
-  for (int i = 0; i < s.n; ++i) {
+#pragma unroll
+  for (int i = 0; i < kMaxQSegs; ++i) {
+    if (i >= s.n || s.a[i] >= s.b[i]) continue;
     const int rq = s.r[i];
     if (!pass_ok(g, rq, rk)) { all = false; continue; }
     if (!g.causal) { any = true; continue; }

@@ -22,9 +22,15 @@ cudaError_t launch_merge(void* out_a, float* lse_a, const void* out_b, const flo
 namespace {
 
 constexpr int kMaxDevices = 64;
+// Per device, one allocation: the status word at [0] and, from
+// [kCounterBase], a ring of work counters handed one per persistent launch
+// (distinct launches in flight on different streams use distinct counters).
+constexpr int kCounterBase = 32;
+constexpr int kCounterSlots = 256;
 std::mutex g_mu;
 int* g_status[kMaxDevices] = {nullptr};
 int g_num_sms[kMaxDevices] = {0};
+unsigned g_next_slot[kMaxDevices] = {0};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -36,8 +42,9 @@ ra_status device_state(int** status, int* num_sms) {
   std::lock_guard<std::mutex> lock(g_mu);
   if (!g_status[dev]) {
     int* p = nullptr;
-    if (cudaMalloc(&p, sizeof(int)) != cudaSuccess) return RA_ERR_CUDA;
-    if (cudaMemset(p, 0, sizeof(int)) != cudaSuccess) {
+    const size_t bytes = sizeof(int) * (kCounterBase + kCounterSlots);
+    if (cudaMalloc(&p, bytes) != cudaSuccess) return RA_ERR_CUDA;
+    if (cudaMemset(p, 0, bytes) != cudaSuccess) {
       cudaFree(p);
       return RA_ERR_CUDA;
     }
@@ -52,6 +59,15 @@ ra_status device_state(int** status, int* num_sms) {
   *status = g_status[dev];
   if (num_sms) *num_sms = g_num_sms[dev];
   return RA_OK;
+}
+
+// A work counter for one persistent launch on the current device.
+int* next_counter(int* status) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(g_mu);
+  const unsigned slot = g_next_slot[dev]++ % kCounterSlots;
+  return status + kCounterBase + slot;
 }
 
 // Shared validation of the forward calls; fills everything but the tensor
@@ -97,8 +113,9 @@ ra_status run_fwd(const void* q, const void* k, const void* v, int64_t tok_strid
   p.scale = scale;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   p.n_qranges = 0;
-  // heaviest query ranges first when later ranges see more keys
-  p.longest_first = (causal && layout == RA_LAYOUT_CONTIGUOUS) ? 1 : 0;
+  // heaviest query ranges first (the kernel launchers refine this per tile size)
+  p.order = (causal && layout == RA_LAYOUT_CONTIGUOUS) ? 1 : 0;
+  p.qr_per_block = 0;
   if (cu_seqlens) {
     // varlen: seqlen is the total row count of the packed tensors
     p.total_rows = seqlen;
@@ -113,6 +130,7 @@ ra_status run_fwd(const void* q, const void* k, const void* v, int64_t tok_strid
   ra_status st = device_state(&status, nullptr);
   if (st != RA_OK) return st;
   p.status = status;
+  p.work_counter = nullptr;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
   // scale 0 (a plain average over the allowed keys) has no log2-domain
@@ -120,6 +138,8 @@ ra_status run_fwd(const void* q, const void* k, const void* v, int64_t tok_strid
   if (dtype == RA_BF16 && !force_simt && scale != 0.f) {
     if (d_head != 64 && d_head != 128) return RA_ERR_UNSUPPORTED;
     if (((tok_stride * 2) & 15) != 0) return RA_ERR_INVALID;
+    p.work_counter = next_counter(status);
+    if (cudaMemsetAsync(p.work_counter, 0, sizeof(int), s) != cudaSuccess) return RA_ERR_CUDA;
     e = ra::launch_fwd_tc(p, s);
   } else {
     e = ra::launch_fwd_simt(p, dtype == RA_F32 ? 0 : 1, s);

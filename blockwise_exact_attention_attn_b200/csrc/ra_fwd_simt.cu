@@ -198,6 +198,7 @@ static cudaError_t launch_simt_t(const FwdParams& p, cudaStream_t stream) {
   using Sh = SimtShape<T, D>;
   FwdParams pp = p;
   pp.n_qranges = (p.seqlen + Sh::ROWS - 1) / Sh::ROWS;
+  set_striped_order(pp, Sh::ROWS);
   const int64_t grid = work_grid(pp, Sh::ROWS);
   if (grid == 0) return cudaSuccess;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;

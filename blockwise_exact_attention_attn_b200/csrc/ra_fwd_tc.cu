@@ -12,7 +12,13 @@
 // "Attention的分块计算" blog (local softmax of a block in fast on-chip memory,
 // combined into the global softmax through per-block max and sum).
 //
-// CTA organisation (one CTA per SM, 384 threads):
+// Persistent CTAs (one per SM, 384 threads) claim work items (two query
+// tiles of one (sequence, head)) from a per-launch counter, in item order
+// (heaviest causal ranges first); the pipelines run across item boundaries:
+// the next item's Q is loaded
+// as soon as the last S MMA of the current one is done (q_free), and its
+// first PV MMA waits only until the softmax warps have read O out (o_free).
+// Warp roles:
 //   warps 0-3  softmax for query tile 0 (one TMEM lane = one query row each)
 //   warps 4-7  softmax for query tile 1
 //   warp  8    TMA producer: Q tiles once, then K and V tiles through an
@@ -21,7 +27,8 @@
 //              completion signalled with tcgen05.commit
 //   warp  10   schedule builder: runs the ring-order tile walk (ra_sched.h)
 //              and publishes the visited kv tiles with their per-query-tile
-//              class into a double-buffered shared-memory list
+//              class into a shared-memory ring of small list chunks (the
+//              first chunk is ready after a few entries)
 //   warp  11   idle (completes the control warpgroup, whose register budget
 //              is handed to the softmax warpgroups with setmaxnreg)
 // Tensor memory (512 columns): S_0 | S_1 | O_0 | O_1; P_i (bf16) is written
@@ -55,7 +62,8 @@ constexpr int kTcThreads = 384;     // 2 softmax warpgroups + 1 control warpgrou
 constexpr int kTcProducerWarp = 8;
 constexpr int kTcMmaWarp = 9;
 constexpr int kTcListWarp = 10;
-constexpr int kListChunk = 1024;    // entries per schedule-list buffer (2 buffers)
+constexpr int kListChunk = 16;      // entries per schedule-list chunk (published at once)
+constexpr int kListBufs = 32;       // chunks in the shared-memory ring
 constexpr int kListConsumers = 10;  // producer, MMA, 8 softmax warps
 // Register split.  Launch: 384 threads x 168 = 64512 registers.  After the
 // split: 256 softmax threads x 176 + 128 control threads x 152 = 64512.
@@ -73,7 +81,7 @@ struct TcCfg {
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = kTcQT * kTileBytes;
   static constexpr int kListOff = kKVOff + kStages * kTileBytes;
-  static constexpr int kCtrlOff = kListOff + 2 * kListChunk * 4;
+  static constexpr int kCtrlOff = kListOff + kListBufs * kListChunk * 4;
   static constexpr int kSmemBytes = kCtrlOff + 1024 + 1024;  // + ctrl + align slack
   static constexpr uint32_t kColS = 0;                      // S_i at i * 128
   static constexpr uint32_t kColO = 256;                    // O_i at 256 + i * D
@@ -81,13 +89,15 @@ struct TcCfg {
 
 struct TcCtrl {
   uint64_t q_full;
+  uint64_t q_free;
   uint64_t kv_full[8];
   uint64_t kv_empty[8];
   uint64_t s_full[kTcQT];
   uint64_t p_full[kTcQT];
   uint64_t o_full[kTcQT];
-  uint64_t list_full[2];
-  uint64_t list_empty[2];
+  uint64_t o_free[kTcQT];
+  uint64_t list_full[kListBufs];
+  uint64_t list_empty[kListBufs];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -187,7 +197,15 @@ __device__ __forceinline__ void apply_mask(float* x, const FwdParams& p, int L, 
 }
 
 // Schedule-list entries: (kt << 4) | (class of query tile 1 << 2) | class of
-// query tile 0; -1 ends the list.
+// query tile 0 for a visited kv tile; kItemEnd ends a work item, kAllDone ends
+// the stream, kPad fills a chunk published early, and -(item + 8) starts work
+// item `item`.  Chunks are released by every consumer after it read their
+// last entry.
+constexpr int kItemEnd = -1;
+constexpr int kAllDone = -2;
+constexpr int kPad = -3;
+__device__ __forceinline__ int item_header(int item) { return -(item + 8); }
+__device__ __forceinline__ int header_item(int e) { return -e - 8; }
 __device__ __forceinline__ int entry_tile(int e) { return e >> 4; }
 __device__ __forceinline__ int entry_cls(int e, int i) { return (e >> (2 * i)) & 3; }
 
@@ -197,26 +215,40 @@ struct ListReader {
   uint64_t* full;
   uint64_t* empty;
   int n;
-  // Next entry into *e; false when a wait gave up.
+  // Next entry other than padding into *e; false when a wait gave up.
   __device__ __forceinline__ bool next(int* e, volatile int* abort) {
-    const int pos = n & (kListChunk - 1);
+    do {
+      if (!next_raw(e, abort)) return false;
+    } while (*e == kPad);
+    return true;
+  }
+  __device__ __forceinline__ bool next_warp(int* e, volatile int* abort) {
+    do {
+      if (!next_warp_raw(e, abort)) return false;
+    } while (*e == kPad);
+    return true;
+  }
+  __device__ __forceinline__ bool next_raw(int* e, volatile int* abort) {
+    const int pos = n % kListChunk;
     const int c = n / kListChunk;
-    if (pos == 0 && !mbar_wait(&full[c & 1], (c >> 1) & 1, abort)) return false;
-    *e = list[(c & 1) * kListChunk + pos];
+    const int b = c % kListBufs;
+    if (pos == 0 && !mbar_wait(&full[b], (c / kListBufs) & 1, abort)) return false;
+    *e = list[b * kListChunk + pos];
     ++n;
-    if (pos == kListChunk - 1 || *e < 0) mbar_arrive(&empty[c & 1]);
+    if (pos == kListChunk - 1) mbar_arrive(&empty[b]);
     return true;
   }
   // Same for a whole warp: lane 0 waits and releases, every lane reads.
-  __device__ __forceinline__ bool next_warp(int* e, volatile int* abort) {
-    const int pos = n & (kListChunk - 1);
+  __device__ __forceinline__ bool next_warp_raw(int* e, volatile int* abort) {
+    const int pos = n % kListChunk;
     const int c = n / kListChunk;
-    if (pos == 0 && !warp_wait(&full[c & 1], (c >> 1) & 1, abort)) return false;
-    *e = list[(c & 1) * kListChunk + pos];
+    const int b = c % kListBufs;
+    if (pos == 0 && !warp_wait(&full[b], (c / kListBufs) & 1, abort)) return false;
+    *e = list[b * kListChunk + pos];
     ++n;
-    if (pos == kListChunk - 1 || *e < 0) {
+    if (pos == kListChunk - 1) {
       __syncwarp();
-      if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[c & 1]);
+      if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[b]);
     }
     return true;
   }
@@ -224,8 +256,10 @@ struct ListReader {
 
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    fwd_tc_kernel(const FwdParams p, const __grid_constant__ TcMaps maps) {
+    fwd_tc_kernel(const FwdParams p, const __grid_constant__ TcMaps maps, int n_items,
+                  int claim_limit) {
   using C = TcCfg<D>;
+  constexpr int kRows = kTcBM * kTcQT;  // query rows per work item
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -235,17 +269,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const SeqWork it = find_work(p, kTcBM * kTcQT);
-  if (!it.live) return;  // uniform across the CTA
-  const int base = it.base, L = it.L;
-  const int q0 = it.qr * (kTcBM * kTcQT);
-  const int qm = min(q0 + kTcBM, L);
-  const int q1 = min(q0 + kTcBM * kTcQT, L);
-
   // ------------------------------------------------------------ set-up
   int* list = reinterpret_cast<int*>(smem + C::kListOff);
   if (threadIdx.x == 0) {
     mbar_init(&ctrl->q_full, 1);
+    mbar_init(&ctrl->q_free, 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&ctrl->kv_full[s], 1);
       mbar_init(&ctrl->kv_empty[s], 1);
@@ -254,8 +282,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&ctrl->s_full[i], 1);
       mbar_init(&ctrl->p_full[i], kTcBM);
       mbar_init(&ctrl->o_full[i], 1);
+      mbar_init(&ctrl->o_free[i], kTcBM);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kListBufs; ++b) {
       mbar_init(&ctrl->list_full[b], 1);
       mbar_init(&ctrl->list_empty[b], kListConsumers);
     }
@@ -281,34 +310,70 @@ __global__ void __launch_bounds__(kTcThreads, 1)
    regs_dec<kRegsControl>();
    if (warp == kTcListWarp) {
     // ---------------------------------------------------------- schedule
-    if (lane == 0) {
-      const RingGeom g = make_geom(L, p.n_ring, p.layout, p.causal, p.passes);
-      TileWalk walk;
-      walk.init(g, q0, qm, q1, kTcBN);
-      bool done = false, ok = true;
-      for (int c = 0; !done; ++c) {
-        const int b = c & 1;
-        if (c >= 2 && !mbar_wait(&ctrl->list_empty[b], ((c >> 1) - 1) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        int* dst = list + b * kListChunk;
-        for (int pos = 0; pos < kListChunk; ++pos) {
-          int kt, c0, c1;
-          if (walk.next(&kt, &c0, &c1)) {
-            dst[pos] = (kt << 4) | (c1 << 2) | c0;
-          } else {
-            dst[pos] = -1;
-            done = true;
-            break;
-          }
-        }
+    // Claims work items from the launch's counter (dynamic balance; heavy
+    // items come first in the item order), at most one item ahead of the
+    // producer, and streams each item's header, ring-order visit list and
+    // end marker, in chunks of kListChunk entries.
+    int c = 0, pos = 0;
+    bool ok = true;
+    auto put = [&](int v) -> bool {
+      const int b = c % kListBufs;
+      if (pos == 0 && c >= kListBufs &&
+          !mbar_wait(&ctrl->list_empty[b], ((c / kListBufs) - 1) & 1, abort_flag))
+        return false;
+      list[b * kListChunk + pos] = v;
+      if (++pos == kListChunk) {
         mbar_arrive(&ctrl->list_full[b]);
+        ++c;
+        pos = 0;
       }
-      if (!ok) {
-        *abort_flag = 1;
-        latch_status(p.status, ST_TIMEOUT);
+      return true;
+    };
+    // publish the current chunk now (padded), so a waiting consumer sees it
+    auto flush = [&]() -> bool {
+      bool f = true;
+      while (f && pos != 0) f = put(kPad);
+      return f;
+    };
+    int j = 0;  // items emitted
+    while (ok) {
+      if (claim_limit > 0 && j >= claim_limit) {
+        if (lane == 0) ok = put(kAllDone) && flush();
+        break;
       }
+      if (lane == 0 && j > 0) {
+        ok = flush();
+        // item j-1 has started (its Q landed) before another item is claimed
+        if (ok) ok = mbar_wait(&ctrl->q_full, (j - 1) & 1, abort_flag);
+      }
+      int item = 0;
+      if (lane == 0 && ok) item = atomicAdd(p.work_counter, 1);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      item = __shfl_sync(0xffffffffu, item, 0);
+      if (!ok) break;
+      if (item >= n_items) {
+        if (lane == 0) ok = put(kAllDone) && flush();
+        break;
+      }
+      const SeqWork it = find_work_item(p, kRows, item);
+      if (!it.live) continue;
+      if (lane == 0) {
+        const int q0 = it.qr * kRows;
+        const int qm = min(q0 + kTcBM, it.L), q1 = min(q0 + kRows, it.L);
+        const RingGeom g = make_geom(it.L, p.n_ring, p.layout, p.causal, p.passes);
+        TileWalk walk;
+        walk.init(g, q0, qm, q1, kTcBN);
+        int kt, c0, c1;
+        ok = put(item_header(item));
+        while (ok && walk.next(&kt, &c0, &c1)) ok = put((kt << 4) | (c1 << 2) | c0);
+        if (ok) ok = put(kItemEnd);
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      ++j;
+    }
+    if (lane == 0 && !ok) {
+      *abort_flag = 1;
+      latch_status(p.status, ST_TIMEOUT);
     }
     __syncwarp();
    } else if (warp == kTcProducerWarp) {
@@ -317,134 +382,178 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tma_prefetch_desc(&maps.q);
       tma_prefetch_desc(&maps.k);
       tma_prefetch_desc(&maps.v);
-      uint8_t* qs = smem + C::kQOff;
-      mbar_arrive_expect_tx(&ctrl->q_full, kTcQT * C::kTileBytes);
-      for (int i = 0; i < kTcQT; ++i)
-        for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_3d(qs + i * C::kTileBytes + pn * C::kPanelBytes, &maps.q, &ctrl->q_full,
-                      pn * 64, it.h, base + q0 + i * kTcBM);
-      int n = 0;
-      bool ok = true;
-      int e;
-      while (true) {
-        ok = rd.next(&e, abort_flag);
-        if (!ok || e < 0) break;
-        const int kt = entry_tile(e);
-        for (int which = 0; which < 2 && ok; ++which) {
-          const int slot = n % C::kStages;
-          if (n >= C::kStages) {
-            ok = mbar_wait(&ctrl->kv_empty[slot], ((n / C::kStages) - 1) & 1, abort_flag);
-            if (!ok) break;
-          }
-          uint8_t* dst = smem + C::kKVOff + slot * C::kTileBytes;
-          mbar_arrive_expect_tx(&ctrl->kv_full[slot], C::kTileBytes);
-          const CUtensorMap* map = which == 0 ? &maps.k : &maps.v;
-          for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_3d(dst + pn * C::kPanelBytes, map, &ctrl->kv_full[slot], pn * 64, it.h,
-                        base + kt * kTcBN);
-          ++n;
+    }
+    int n = 0, k = 0;
+    bool ok = true;
+    while (ok) {
+      int h = 0;
+      if (lane == 0) ok = rd.next(&h, abort_flag);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      h = __shfl_sync(0xffffffffu, h, 0);
+      if (!ok || h == kAllDone) break;
+      const SeqWork it = find_work_item(p, kRows, header_item(h));
+      if (lane == 0) {
+        // Q of this item once the previous item's last S MMA is done
+        if (k > 0) ok = mbar_wait(&ctrl->q_free, (k - 1) & 1, abort_flag);
+        if (ok) {
+          uint8_t* qs = smem + C::kQOff;
+          const int q0 = it.qr * kRows;
+          mbar_arrive_expect_tx(&ctrl->q_full, kTcQT * C::kTileBytes);
+          for (int i = 0; i < kTcQT; ++i)
+            for (int pn = 0; pn < C::kPanels; ++pn)
+              tma_load_3d(qs + i * C::kTileBytes + pn * C::kPanelBytes, &maps.q,
+                          &ctrl->q_full, pn * 64, it.h, it.base + q0 + i * kTcBM);
         }
-        if (!ok) break;
+        int e;
+        while (ok) {
+          ok = rd.next(&e, abort_flag);
+          if (!ok || e < 0) break;
+          const int kt = entry_tile(e);
+          for (int which = 0; which < 2 && ok; ++which) {
+            const int slot = n % C::kStages;
+            if (n >= C::kStages) {
+              ok = mbar_wait(&ctrl->kv_empty[slot], ((n / C::kStages) - 1) & 1, abort_flag);
+              if (!ok) break;
+            }
+            uint8_t* dst = smem + C::kKVOff + slot * C::kTileBytes;
+            mbar_arrive_expect_tx(&ctrl->kv_full[slot], C::kTileBytes);
+            const CUtensorMap* map = which == 0 ? &maps.k : &maps.v;
+            for (int pn = 0; pn < C::kPanels; ++pn)
+              tma_load_3d(dst + pn * C::kPanelBytes, map, &ctrl->kv_full[slot], pn * 64, it.h,
+                          it.base + kt * kTcBN);
+            ++n;
+          }
+        }
       }
-      if (!ok) {
-        *abort_flag = 1;
-        latch_status(p.status, ST_TIMEOUT);
-        // let the copies already issued land before the CTA can exit
-        for (int u = (n > C::kStages ? n - C::kStages : 0); u < n; ++u)
-          mbar_wait(&ctrl->kv_full[u % C::kStages], (u / C::kStages) & 1, nullptr);
-        mbar_wait(&ctrl->q_full, 0, nullptr);
-      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      ++k;
+    }
+    if (lane == 0 && !ok) {
+      *abort_flag = 1;
+      latch_status(p.status, ST_TIMEOUT);
+      // let the copies already issued land before the CTA can exit
+      for (int u = (n > C::kStages ? n - C::kStages : 0); u < n; ++u)
+        mbar_wait(&ctrl->kv_full[u % C::kStages], (u / C::kStages) & 1, nullptr);
+      if (k > 0) mbar_wait(&ctrl->q_full, (k - 1) & 1, nullptr);
     }
     __syncwarp();
    } else if (warp == kTcMmaWarp) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      // a negative softmax scale is applied as S = (-Q) K^T times |scale|
-      const uint32_t idesc_s =
-          idesc_bf16_f32(kTcBM, kTcBN, 0) | (p.scale_log2 < 0.f ? (1u << 13) : 0u);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(kTcBM, D, 1);
-      // base descriptors: K-major tiles (Q, K) and MN-major tiles (V)
-      const uint32_t qs = smem_u32(smem + C::kQOff);
-      const uint32_t kvs = smem_u32(smem + C::kKVOff);
-      uint64_t qdesc[kTcQT];
+    // a negative softmax scale is applied as S = (-Q) K^T times |scale|
+    const uint32_t idesc_s =
+        idesc_bf16_f32(kTcBM, kTcBN, 0) | (p.scale_log2 < 0.f ? (1u << 13) : 0u);
+    constexpr uint32_t idesc_o = idesc_bf16_f32(kTcBM, D, 1);
+    // base descriptors: K-major tiles (Q, K) and MN-major tiles (V)
+    const uint32_t qs = smem_u32(smem + C::kQOff);
+    const uint32_t kvs = smem_u32(smem + C::kKVOff);
+    uint64_t qdesc[kTcQT];
 #pragma unroll
-      for (int i = 0; i < kTcQT; ++i) qdesc[i] = smem_desc_sw128(qs + i * C::kTileBytes, 16, 1024);
-      const uint64_t kdesc0 = smem_desc_sw128(kvs, 16, 1024);
-      const uint64_t vdesc0 = smem_desc_sw128(kvs, C::kPanelBytes, 1024);
-      constexpr uint64_t kSlotStep = (uint64_t)(C::kTileBytes >> 4);
-      bool ok = mbar_wait(&ctrl->q_full, 0, abort_flag);
-      tc_fence_after();
-      uint32_t pphase[kTcQT] = {0, 0};
-      bool started[kTcQT] = {false, false};
-      int n = 0;
-      bool issued_any = false;
-      int e = -1, ep = -1;
-      if (ok) ok = rd.next(&e, abort_flag);
-      if (ok && e >= 0) {
-        const int slot = n % C::kStages;
-        ok = mbar_wait(&ctrl->kv_full[slot], (n / C::kStages) & 1, abort_flag);
-        ++n;
-        if (ok) {
-          tc_fence_after();
-          for (int i = 0; i < kTcQT; ++i)
-            if (entry_cls(e, i) != CLS_EMPTY) {
-              issue_qk<D>(tmem + C::kColS + i * kTcBN, qdesc[i], kdesc0 + slot * kSlotStep,
-                          idesc_s);
-              umma_commit(&ctrl->s_full[i]);
-            }
-          umma_commit(&ctrl->kv_empty[slot]);
-          issued_any = true;
-        }
-        ep = e;
-        while (ok) {
-          const int slot_v = n % C::kStages;
-          ok = mbar_wait(&ctrl->kv_full[slot_v], (n / C::kStages) & 1, abort_flag);
+    for (int i = 0; i < kTcQT; ++i) qdesc[i] = smem_desc_sw128(qs + i * C::kTileBytes, 16, 1024);
+    const uint64_t kdesc0 = smem_desc_sw128(kvs, 16, 1024);
+    const uint64_t vdesc0 = smem_desc_sw128(kvs, C::kPanelBytes, 1024);
+    constexpr uint64_t kSlotStep = (uint64_t)(C::kTileBytes >> 4);
+    uint32_t pphase[kTcQT] = {0, 0};
+    int n = 0, k = 0;
+    bool ok = true, issued_any = false;
+    while (ok) {
+      int h = 0;
+      if (lane == 0) ok = rd.next(&h, abort_flag);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      h = __shfl_sync(0xffffffffu, h, 0);
+      if (!ok || h == kAllDone) break;
+      if (lane == 0) {
+        ok = mbar_wait(&ctrl->q_full, k & 1, abort_flag);
+        tc_fence_after();
+        bool started[kTcQT] = {false, false};
+        // the previous item's O_i must have been read out before it is overwritten
+        bool ofree_pending[kTcQT] = {k > 0, k > 0};
+        auto wait_ofree = [&](int i) {
+          if (ok && ofree_pending[i]) {
+            ok = mbar_wait(&ctrl->o_free[i], (k - 1) & 1, abort_flag);
+            ofree_pending[i] = false;
+            tc_fence_after();
+          }
+        };
+        int e = -1, ep = -1;
+        if (ok) ok = rd.next(&e, abort_flag);
+        if (ok && e >= 0) {
+          const int slot = n % C::kStages;
+          ok = mbar_wait(&ctrl->kv_full[slot], (n / C::kStages) & 1, abort_flag);
           ++n;
-          if (!ok) break;
-          ok = rd.next(&e, abort_flag);
-          if (!ok) break;
-          const bool has = e >= 0;
-          int slot_k = 0;
-          if (has) {
-            slot_k = n % C::kStages;
-            ok = mbar_wait(&ctrl->kv_full[slot_k], (n / C::kStages) & 1, abort_flag);
+          if (ok) {
+            tc_fence_after();
+            for (int i = 0; i < kTcQT; ++i)
+              if (entry_cls(e, i) != CLS_EMPTY) {
+                issue_qk<D>(tmem + C::kColS + i * kTcBN, qdesc[i], kdesc0 + slot * kSlotStep,
+                            idesc_s);
+                umma_commit(&ctrl->s_full[i]);
+              }
+            umma_commit(&ctrl->kv_empty[slot]);
+            issued_any = true;
+          }
+          ep = e;
+          while (ok) {
+            const int slot_v = n % C::kStages;
+            ok = mbar_wait(&ctrl->kv_full[slot_v], (n / C::kStages) & 1, abort_flag);
             ++n;
             if (!ok) break;
-          }
-          tc_fence_after();
-          for (int i = 0; i < kTcQT && ok; ++i) {
-            if (entry_cls(ep, i) != CLS_EMPTY) {
-              ok = mbar_wait(&ctrl->p_full[i], pphase[i], abort_flag);
-              pphase[i] ^= 1;
+            ok = rd.next(&e, abort_flag);
+            if (!ok) break;
+            const bool has = e >= 0;
+            int slot_k = 0;
+            if (has) {
+              slot_k = n % C::kStages;
+              ok = mbar_wait(&ctrl->kv_full[slot_k], (n / C::kStages) & 1, abort_flag);
+              ++n;
               if (!ok) break;
-              tc_fence_after();
-              issue_pv<D>(tmem + C::kColO + i * D, tmem + C::kColS + i * kTcBN,
-                          vdesc0 + slot_v * kSlotStep, idesc_o, started[i]);
-              started[i] = true;
+            } else {
+              // every S of this item is issued: Q may be replaced once they finish
+              umma_commit(&ctrl->q_free);
             }
-            if (has && entry_cls(e, i) != CLS_EMPTY) {
-              issue_qk<D>(tmem + C::kColS + i * kTcBN, qdesc[i], kdesc0 + slot_k * kSlotStep,
-                          idesc_s);
-              umma_commit(&ctrl->s_full[i]);
+            tc_fence_after();
+            for (int i = 0; i < kTcQT && ok; ++i) {
+              if (entry_cls(ep, i) != CLS_EMPTY) {
+                ok = mbar_wait(&ctrl->p_full[i], pphase[i], abort_flag);
+                pphase[i] ^= 1;
+                if (!ok) break;
+                tc_fence_after();
+                if (!started[i]) wait_ofree(i);
+                if (!ok) break;
+                issue_pv<D>(tmem + C::kColO + i * D, tmem + C::kColS + i * kTcBN,
+                            vdesc0 + slot_v * kSlotStep, idesc_o, started[i]);
+                started[i] = true;
+              }
+              if (has && entry_cls(e, i) != CLS_EMPTY) {
+                issue_qk<D>(tmem + C::kColS + i * kTcBN, qdesc[i], kdesc0 + slot_k * kSlotStep,
+                            idesc_s);
+                umma_commit(&ctrl->s_full[i]);
+              }
             }
+            if (!ok) break;
+            umma_commit(&ctrl->kv_empty[slot_v]);
+            if (!has) break;
+            umma_commit(&ctrl->kv_empty[slot_k]);
+            ep = e;
           }
-          if (!ok) break;
-          umma_commit(&ctrl->kv_empty[slot_v]);
-          if (!has) break;
-          umma_commit(&ctrl->kv_empty[slot_k]);
-          ep = e;
+        } else if (ok) {
+          umma_commit(&ctrl->q_free);  // an item without tiles
+        }
+        if (ok) {
+          for (int i = 0; i < kTcQT; ++i) wait_ofree(i);
+          if (ok)
+            for (int i = 0; i < kTcQT; ++i) umma_commit(&ctrl->o_full[i]);
         }
       }
-      if (ok) {
-        for (int i = 0; i < kTcQT; ++i) umma_commit(&ctrl->o_full[i]);
-      } else {
-        *abort_flag = 1;
-        latch_status(p.status, ST_TIMEOUT);
-        if (issued_any) {
-          // wait (bounded) for the MMAs already issued before TMEM is freed
-          umma_commit(&ctrl->drain);
-          mbar_wait(&ctrl->drain, 0, nullptr);
-        }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      ++k;
+    }
+    if (lane == 0 && !ok) {
+      *abort_flag = 1;
+      latch_status(p.status, ST_TIMEOUT);
+      if (issued_any) {
+        // wait (bounded) for the MMAs already issued before TMEM is freed
+        umma_commit(&ctrl->drain);
+        mbar_wait(&ctrl->drain, 0, nullptr);
       }
     }
     __syncwarp();
@@ -455,103 +564,112 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int tile = warp >> 2;          // query tile handled by this warp
     const int quad = warp & 3;           // TMEM lane quadrant
     const int r = quad * 32 + lane;      // row within the query tile
-    const int sq = q0 + tile * kTcBM + r;
-    const bool valid = sq < L;
-    int rq = 0, tq = 0;
-    if (valid) {
-      const RingGeom g = make_geom(L, p.n_ring, p.layout, p.causal, p.passes);
-      rq = block_of(g, sq);
-      tq = token_of(g, sq, rq);
-    }
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::kColS + tile * kTcBN;
     const uint32_t tO = tmem + lane_off + C::kColO + tile * D;
     const float sl2 = fabsf(p.scale_log2);  // > 0; the sign is folded into the MMA
-
-    float m_ref = -INFINITY;  // reference max, log2 domain
-    float l = 0.f;
     uint32_t sphase = 0;
-    bool first = true;
+    int k = 0;
     bool ok = true;
 
     while (true) {
-      int e;
-      ok = rd.next_warp(&e, abort_flag);
-      if (!ok || e < 0) break;
-      const int cls = entry_cls(e, tile);
-      if (cls == CLS_EMPTY) continue;
-      ok = warp_wait(&ctrl->s_full[tile], sphase, abort_flag);
-      sphase ^= 1;
+      int h;
+      ok = rd.next_warp(&h, abort_flag);
+      if (!ok || h == kAllDone) break;
+      const SeqWork it = find_work_item(p, kRows, header_item(h));
+      const int L = it.L;
+      const int sq = it.qr * kRows + tile * kTcBM + r;
+      const bool valid = sq < L;
+      int rq = 0, tq = 0;
+      if (valid) {
+        const RingGeom g = make_geom(L, p.n_ring, p.layout, p.causal, p.passes);
+        rq = block_of(g, sq);
+        tq = token_of(g, sq, rq);
+      }
+      float m_ref = -INFINITY;  // reference max, log2 domain
+      float l = 0.f;
+      bool first = true;
+
+      while (true) {
+        int e;
+        ok = rd.next_warp(&e, abort_flag);
+        if (!ok || e < 0) break;
+        const int cls = entry_cls(e, tile);
+        if (cls == CLS_EMPTY) continue;
+        ok = warp_wait(&ctrl->s_full[tile], sphase, abort_flag);
+        sphase ^= 1;
+        if (!ok) break;
+        tc_fence_after();
+
+        float x[kTcBN];
+        {
+          uint32_t* xr = reinterpret_cast<uint32_t*>(x);
+#pragma unroll
+          for (int c = 0; c < kTcBN; c += 32) RA_TMEM_LD32(tS + c, (xr + c));
+          tmem_wait_ld();
+        }
+        const int k0 = entry_tile(e) * kTcBN;
+        const int nk = min(kTcBN, L - k0);
+        if (cls == CLS_PARTIAL || nk < kTcBN) {
+          apply_mask(x, p, L, valid, cls, sq, rq, tq, k0, nk);
+        }
+        // row max as a tree of independent maxima (short dependency chains)
+        float mx8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) mx8[j] = x[j];
+#pragma unroll
+        for (int c = 8; c < kTcBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        const float m_tile = mx * sl2;  // -inf stays -inf (sl2 > 0)
+        const bool need = m_tile > m_ref + kRescaleLog2;
+        float alpha = 1.f;
+        if (need) {
+          alpha = ex2_approx(m_ref - m_tile);  // 0 when m_ref == -inf
+          m_ref = m_tile;
+        }
+        const float msub = m_ref == -INFINITY ? 0.f : m_ref;
+        float rs4[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial row sums
+#pragma unroll
+        for (int q = 0; q < kTcBN / 32; ++q) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float a = ex2_approx(fmaf(x[q * 32 + 2 * j], sl2, -msub));
+            const float b = ex2_approx(fmaf(x[q * 32 + 2 * j + 1], sl2, -msub));
+            rs4[j & 3] += a + b;
+            pk[j] = pack_bf16x2(a, b);
+          }
+          RA_TMEM_ST16(tS + q * 16, pk);
+        }
+        l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
+        if (!first && __any_sync(0xffffffffu, need)) {
+          // O_row *= alpha (exactly 1.0 for rows that keep their reference)
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            uint32_t o[32];
+            RA_TMEM_LD32(tO + c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+            RA_TMEM_ST32(tO + c, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&ctrl->p_full[tile]);
+        first = false;
+      }
+      if (!ok) break;
+
+      // epilogue: O is read out of tensor memory, handed back, then stored
+      ok = warp_wait(&ctrl->o_full[tile], k & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
-
-      float x[kTcBN];
-      {
-        uint32_t* xr = reinterpret_cast<uint32_t*>(x);
-#pragma unroll
-        for (int c = 0; c < kTcBN; c += 32) RA_TMEM_LD32(tS + c, (xr + c));
-        tmem_wait_ld();
-      }
-      const int k0 = entry_tile(e) * kTcBN;
-      const int nk = min(kTcBN, L - k0);
-      if (cls == CLS_PARTIAL || nk < kTcBN) {
-        apply_mask(x, p, L, valid, cls, sq, rq, tq, k0, nk);
-      }
-      // row max as a tree of independent maxima (short dependency chains)
-      float mx8[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) mx8[j] = x[j];
-#pragma unroll
-      for (int c = 8; c < kTcBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      const float m_tile = mx * sl2;  // -inf stays -inf (sl2 > 0)
-      const bool need = m_tile > m_ref + kRescaleLog2;
-      float alpha = 1.f;
-      if (need) {
-        alpha = ex2_approx(m_ref - m_tile);  // 0 when m_ref == -inf
-        m_ref = m_tile;
-      }
-      const float msub = m_ref == -INFINITY ? 0.f : m_ref;
-      float rs4[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial row sums
-#pragma unroll
-      for (int q = 0; q < kTcBN / 32; ++q) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float a = ex2_approx(fmaf(x[q * 32 + 2 * j], sl2, -msub));
-          const float b = ex2_approx(fmaf(x[q * 32 + 2 * j + 1], sl2, -msub));
-          rs4[j & 3] += a + b;
-          pk[j] = pack_bf16x2(a, b);
-        }
-        RA_TMEM_ST16(tS + q * 16, pk);
-      }
-      l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
-      if (!first && __any_sync(0xffffffffu, need)) {
-        // O_row *= alpha (exactly 1.0 for rows that keep their reference)
-#pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t o[32];
-          RA_TMEM_LD32(tO + c, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-          RA_TMEM_ST32(tO + c, o);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&ctrl->p_full[tile]);
-      first = false;
-    }
-
-    if (ok && !first) {
-      ok = warp_wait(&ctrl->o_full[tile], 0, abort_flag);
-      if (ok) {
-        tc_fence_after();
+      if (!first) {
         const float inv_l = valid ? 1.f / l : 0.f;
         __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) +
-                              ((int64_t)(base + sq) * p.heads + it.h) * D;
+                              ((int64_t)(it.base + sq) * p.heads + it.h) * D;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
           uint32_t o[32];
@@ -569,12 +687,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
           }
         }
-        if (valid) {
-          const int64_t li = (int64_t)it.b * p.lse_seq_stride +
-                             (int64_t)it.h * p.lse_head_stride + (p.cu_seqlens ? base : 0) + sq;
-          p.lse[li] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
-        }
       }
+      tc_fence_before();
+      mbar_arrive(&ctrl->o_free[tile]);
+      if (!first && valid) {
+        const int64_t li = (int64_t)it.b * p.lse_seq_stride + (int64_t)it.h * p.lse_head_stride +
+                           (p.cu_seqlens ? it.base : 0) + sq;
+        p.lse[li] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
+      }
+      ++k;
     }
     if (!ok) {
       *abort_flag = 1;
@@ -633,9 +754,23 @@ static cudaError_t launch_tc_t(const FwdParams& p, cudaStream_t stream) {
   using C = TcCfg<D>;
   FwdParams pp = p;
   pp.n_qranges = (p.seqlen + kTcBM * kTcQT - 1) / (kTcBM * kTcQT);
-  const int64_t grid = work_grid(pp, kTcBM * kTcQT);
-  if (grid == 0) return cudaSuccess;
-  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  set_striped_order(pp, kTcBM * kTcQT);
+  const int64_t items = work_grid(pp, kTcBM * kTcQT);
+  if (items == 0) return cudaSuccess;
+  if (items > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  // persistent: one CTA per SM (shared memory and tensor memory allow one)
+  static int sms[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!sms[dev] && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) !=
+                       cudaSuccess)
+    return cudaErrorInvalidDevice;
+  // Dense causal work varies per item: one CTA per item, balanced by the
+  // hardware block scheduler, measured faster than persistent CTAs there.
+  // Otherwise persistent CTAs (one per SM) claim items until none is left.
+  const bool per_item = p.causal && !p.cu_seqlens;
+  const int64_t grid = per_item ? items : (items < sms[dev] ? items : sms[dev]);
+  const int claim_limit = per_item ? 1 : 0;
   TcMaps maps;
   if (!make_map(&maps.q, p.q, p.total_rows, p.heads, D, p.tok_stride) ||
       !make_map(&maps.k, p.k, p.total_rows, p.heads, D, p.tok_stride) ||
@@ -645,7 +780,8 @@ static cudaError_t launch_tc_t(const FwdParams& p, cudaStream_t stream) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  fwd_tc_kernel<D><<<(unsigned)grid, kTcThreads, C::kSmemBytes, stream>>>(pp, maps);
+  fwd_tc_kernel<D><<<(unsigned)grid, kTcThreads, C::kSmemBytes, stream>>>(pp, maps, (int)items,
+                                                                        claim_limit);
   return cudaGetLastError();
 }
 

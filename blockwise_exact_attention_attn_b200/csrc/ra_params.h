@@ -23,16 +23,22 @@ struct FwdParams {
   int n_ring, layout, causal, passes;
   int total_rows;           // rows of q/k/v/out (dense: batch*seqlen)
   int n_qranges;            // query ranges per sequence (ceil(seqlen / rows per CTA))
-  int longest_first;        // visit query ranges from the last to the first
+  int order;                // query-range order inside a (sequence, head): 0 natural,
+                            // 1 last to first, 2 striped (local position descending)
+  int qr_per_block;         // order 2: query ranges per ring block
   float scale;              // softmax scale
   float scale_log2;         // scale * log2(e)
   int* status;              // device status word (never NULL at launch)
+  int* work_counter;        // persistent kernels: next work item (zeroed per launch)
 };
 
-// Map a linear CTA index to (query range, batch, head).  The (batch, head)
-// pair is the slowest index, so the CTAs resident at one time share the K/V
-// of a few heads in L2; inside a head the query ranges run from the last to
-// the first with longest_first (heaviest causal ranges first).
+// Map a linear work index to (query range, batch, head).  The (batch, head)
+// pair is the slowest index, so the work running at one time shares the K/V
+// of a few heads in L2.  Inside a head the causal query ranges come heaviest
+// first: from the last to the first (contiguous layout), or, striped, by
+// local position inside the ring blocks from the last to the first (a
+// striped query range at local position j of its block sees keys up to j of
+// every block).
 struct WorkItem {
   int qr, b, h;
 };
@@ -48,7 +54,14 @@ WorkItem decode_work(const FwdParams& p, int64_t w) {
   const int qr = (int)(w - bh * p.n_qranges);
   it.b = (int)(bh / p.heads);
   it.h = (int)(bh - (int64_t)it.b * p.heads);
-  it.qr = p.longest_first ? (p.n_qranges - 1 - qr) : qr;
+  if (p.order == 1) {
+    it.qr = p.n_qranges - 1 - qr;
+  } else if (p.order == 2) {
+    const int jj = qr / p.n_ring, r = qr - jj * p.n_ring;
+    it.qr = r * p.qr_per_block + (p.qr_per_block - 1 - jj);
+  } else {
+    it.qr = qr;
+  }
   return it;
 }
 

@@ -2,13 +2,13 @@
 //
 // Dense inputs: CTA index w -> (batch, head, query range) with the query
 // range fastest, so the CTAs running together share a few heads' K/V in L2;
-// with longest_first a head's heaviest causal ranges start first.
+// causal ranges are ordered heaviest first (see decode_work).
 // Varlen inputs (cu_seqlens, "Tensorflow flash attention" page: cumulative
 // sequence lengths of shape (batch_size + 1,) index ragged, unpadded
 // tensors): CTA index w -> (flat range, head) with the head fastest; the flat
 // range is located among the sequences by a warp-wide scan of their range
 // counts ceil(L_b / rows_per_cta), and inside a sequence the ranges run from
-// the last to the first when longest_first.
+// the last to the first for causal contiguous inputs.
 #pragma once
 
 #include <stdint.h>
@@ -25,15 +25,17 @@ struct SeqWork {
   bool live;      // false: nothing to do for this CTA
 };
 
-// Must be called by all 32 lanes of a warp (any warp; every warp of a CTA
-// computes the same answer).  Latches ST_INVALID for malformed cu_seqlens.
-__device__ __forceinline__ SeqWork find_work(const FwdParams& p, int rows_per_cta) {
+// Work item `item` (a CTA index of the non-persistent grid).  Must be called
+// by all 32 lanes of a warp (any warp; every warp computes the same answer).
+// Latches ST_INVALID for malformed cu_seqlens.
+__device__ __forceinline__ SeqWork find_work_item(const FwdParams& p, int rows_per_cta,
+                                                  int item) {
   SeqWork w;
   w.live = false;
   w.b = w.qr = w.h = w.base = w.L = 0;
   const int lane = threadIdx.x & 31;
   if (!p.cu_seqlens) {
-    const WorkItem it = decode_work(p, blockIdx.x);
+    const WorkItem it = decode_work(p, item);
     w.b = it.b;
     w.qr = it.qr;
     w.h = it.h;
@@ -42,9 +44,9 @@ __device__ __forceinline__ SeqWork find_work(const FwdParams& p, int rows_per_ct
     w.live = (int64_t)it.qr * rows_per_cta < p.seqlen;
     return w;
   }
-  const int flat = blockIdx.x / p.heads;
-  w.h = blockIdx.x - flat * p.heads;
-  if (lane == 0 && threadIdx.x == 0 && blockIdx.x == 0 &&
+  const int flat = item / p.heads;
+  w.h = item - flat * p.heads;
+  if (lane == 0 && threadIdx.x == 0 && item == 0 &&
       (p.cu_seqlens[0] != 0 || p.cu_seqlens[p.batch] != p.total_rows))
     latch_status(p.status, ST_INVALID);
   int acc = 0;
@@ -77,13 +79,27 @@ __device__ __forceinline__ SeqWork find_work(const FwdParams& p, int rows_per_ct
       w.L = __shfl_sync(0xffffffffu, len, src);
       const int nq = __shfl_sync(0xffffffffu, n, src);
       const int qi = flat - acc - __shfl_sync(0xffffffffu, excl, src);
-      w.qr = p.longest_first ? nq - 1 - qi : qi;
+      w.qr = p.order == 1 ? nq - 1 - qi : qi;
       w.live = true;
       return w;
     }
     acc += __shfl_sync(0xffffffffu, incl, 31);
   }
   return w;
+}
+
+__device__ __forceinline__ SeqWork find_work(const FwdParams& p, int rows_per_cta) {
+  return find_work_item(p, rows_per_cta, (int)blockIdx.x);
+}
+
+// Causal striped dense inputs whose ring blocks hold a whole number of work
+// items: order the items by local position (heaviest first).
+inline void set_striped_order(FwdParams& p, int rows_per_cta) {
+  if (p.cu_seqlens || !p.causal || p.layout != 1) return;
+  const int blk = p.seqlen / p.n_ring;
+  if (blk % rows_per_cta != 0 || blk == 0) return;
+  p.order = 2;
+  p.qr_per_block = blk / rows_per_cta;
 }
 
 // Launch size: dense n_qranges * batch * heads; varlen (ceil(total /

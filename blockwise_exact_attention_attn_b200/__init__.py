@@ -20,6 +20,7 @@ from ._binding import (  # noqa: F401
     load_library,
     ring_attn_func,
     ring_attn_fwd,
+    ring_attn_fwd_noalloc,
     ring_attn_fwd_simt,
     ring_attn_merge,
     ring_attn_qkvpacked_fwd,

@@ -27,6 +27,7 @@ EXPORTS = (
     "ring_attn_fwd",
     "ring_attn_qkvpacked_fwd",
     "ring_attn_fwd_simt",
+    "ring_attn_fwd_noalloc",
     "ring_attn_merge",
     "ring_attn_status",
     "ring_attn_status_string",
@@ -67,6 +68,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.ring_attn_fwd.restype = _c_int
         lib.ring_attn_fwd_simt.argtypes = _FWD_ARGS
         lib.ring_attn_fwd_simt.restype = _c_int
+        lib.ring_attn_fwd_noalloc.argtypes = _FWD_ARGS
+        lib.ring_attn_fwd_noalloc.restype = _c_int
         lib.ring_attn_qkvpacked_fwd.argtypes = [_c_vp, _c_vp, _c_vp] + _FWD_ARGS[5:]
         lib.ring_attn_qkvpacked_fwd.restype = _c_int
         lib.ring_attn_merge.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
@@ -174,6 +177,26 @@ def ring_attn_fwd_simt(q, k, v, out, lse, batch: int, heads: int, seqlen: int, d
         _ptr(cu_seqlens, "cu_seqlens"), _dtype_code(q) if dtype is None else int(dtype),
         _stream(stream))
     _check("ring_attn_fwd_simt", st)
+
+
+def ring_attn_fwd_noalloc(q, k, v, out, lse, batch: int, heads: int, seqlen: int,
+                          d_head: int, n_ring_blocks: int, layout=CONTIGUOUS,
+                          causal: bool = False, softmax_scale: Optional[float] = None,
+                          max_ring_passes: Optional[int] = None, cu_seqlens=None,
+                          dtype: Optional[int] = None, stream=None) -> None:
+    """ring_attn_fwd without any device allocation (see ring_attn.h)."""
+    lib = load_library()
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d_head)
+    if max_ring_passes is None:
+        max_ring_passes = n_ring_blocks
+    st = lib.ring_attn_fwd_noalloc(
+        _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _ptr(out, "out"), _ptr(lse, "lse"),
+        int(batch), int(heads), int(seqlen), int(d_head), int(n_ring_blocks),
+        _layout_code(layout), int(bool(causal)), float(softmax_scale), int(max_ring_passes),
+        _ptr(cu_seqlens, "cu_seqlens"), _dtype_code(q) if dtype is None else int(dtype),
+        _stream(stream))
+    _check("ring_attn_fwd_noalloc", st)
 
 
 def ring_attn_qkvpacked_fwd(qkv, out, lse, batch: int, heads: int, seqlen: int, d_head: int,

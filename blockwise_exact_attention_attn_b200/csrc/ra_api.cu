@@ -275,3 +275,118 @@ int64_t ring_attn_schedule(int seqlen, int n_ring_blocks, int layout, int causal
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of ring_attn_fwd.
+//
+// The tensor-core forward needs a little device scratch: the word that
+// latches device-side errors and the counter its persistent CTAs claim work
+// items from.  ring_attn_fwd takes both from memory the library allocates
+// with cudaMalloc on the first call on a device.  ring_attn_fwd_noalloc takes
+// them from the fixed array below instead, so it never allocates.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+constexpr int kNoAllocWords = 64;       // 256 bytes per device
+constexpr int kNoAllocStatus = 0;       // device status word of these calls
+constexpr int kNoAllocCounter = 32;     // work counter (own 128-byte line)
+
+}  // namespace
+
+// Lives in every device context that loads the library, until it exits.
+static __device__ __align__(256) int g_noalloc_scratch[kNoAllocWords];
+
+namespace {
+
+int* g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_noalloc_scratch on the current device (looked up once
+// per device, with that device current).
+ra_status noalloc_scratch(int** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr)
+      return RA_ERR_CUDA;
+    g_noalloc_ptr[dev] = static_cast<int*>(ptr);
+  }
+  *out = g_noalloc_ptr[dev];
+  return RA_OK;
+}
+
+}  // namespace
+
+extern "C" ra_status ring_attn_fwd_noalloc(const void* q, const void* k, const void* v,
+                                           void* out, float* lse, int batch, int heads,
+                                           int seqlen, int d_head, int n_ring_blocks,
+                                           int layout, int causal, float softmax_scale,
+                                           int max_ring_passes, const int32_t* cu_seqlens,
+                                           int dtype, void* stream) {
+  if (!q || !k || !v || !out || !lse) return RA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return RA_ERR_INVALID;
+  ra_status st = validate_fwd(batch, heads, seqlen, d_head, n_ring_blocks, layout, causal,
+                              softmax_scale, max_ring_passes, cu_seqlens, dtype);
+  if (st != RA_OK) return st;
+  // Scratch this call needs: the status word and one work counter.  Both
+  // sit at fixed offsets, so no problem size can outgrow the array; the check
+  // keeps that true if a kernel ever needs more.
+  constexpr size_t need = sizeof(int) * (kNoAllocCounter + 1);
+  static_assert(need <= sizeof(int) * kNoAllocWords, "no-alloc scratch too small");
+  if (need > sizeof(int) * kNoAllocWords) return RA_ERR_UNSUPPORTED;
+
+  int* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != RA_OK) return st;
+
+  ra::FwdParams p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.tok_stride = (int64_t)heads * d_head;
+  p.out = out;
+  p.lse = lse;
+  p.cu_seqlens = cu_seqlens;
+  p.batch = batch;
+  p.heads = heads;
+  p.seqlen = seqlen;
+  p.d_head = d_head;
+  p.n_ring = n_ring_blocks;
+  p.layout = layout;
+  p.causal = causal;
+  p.passes = max_ring_passes < n_ring_blocks ? max_ring_passes : n_ring_blocks;
+  p.scale = softmax_scale;
+  p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634074);
+  p.n_qranges = 0;
+  p.order = (causal && layout == RA_LAYOUT_CONTIGUOUS) ? 1 : 0;
+  p.qr_per_block = 0;
+  if (cu_seqlens) {
+    p.total_rows = seqlen;
+    p.lse_seq_stride = 0;
+    p.lse_head_stride = seqlen;
+  } else {
+    p.total_rows = batch * seqlen;
+    p.lse_seq_stride = (int64_t)heads * seqlen;
+    p.lse_head_stride = seqlen;
+  }
+  p.status = scratch + kNoAllocStatus;
+  p.work_counter = scratch + kNoAllocCounter;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the array keeps the previous call's contents: start from zero
+  if (cudaMemsetAsync(scratch + kNoAllocStatus, 0, sizeof(int), s) != cudaSuccess ||
+      cudaMemsetAsync(scratch + kNoAllocCounter, 0, sizeof(int), s) != cudaSuccess)
+    return RA_ERR_CUDA;
+  cudaError_t e;
+  if (dtype == RA_BF16 && softmax_scale != 0.f) {
+    if (d_head != 64 && d_head != 128) return RA_ERR_UNSUPPORTED;
+    e = ra::launch_fwd_tc(p, s);
+  } else {
+    e = ra::launch_fwd_simt(p, dtype == RA_F32 ? 0 : 1, s);
+  }
+  if (e == cudaErrorInvalidValue) return RA_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}

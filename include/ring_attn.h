@@ -184,6 +184,43 @@ ra_status ring_attn_merge(void* out_a, float* lse_a, const void* out_b,
                           int d_head, int dtype, void* stream);
 
 /*
+ * ring_attn_fwd_noalloc -- ring_attn_fwd that allocates nothing.  (No
+ * counterpart in the pages: this is a deployment variant of the same call.)
+ *
+ * For callers that cannot allocate device memory: code being captured into a
+ * CUDA graph in a mode that forbids allocation, processes whose device memory
+ * is owned by a fixed pool or budget, and runtimes that must not touch the
+ * allocator after start-up.  ring_attn_fwd allocates a small device scratch
+ * (error status word, work counters) with cudaMalloc on its first call on a
+ * device; this entry point uses a 256-byte array that is part of the
+ * library's device image instead (every device that loads the library holds
+ * it until the process exits), and calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *
+ *  - Arguments, layouts, ownership and host-side errors are those of
+ *    ring_attn_fwd; results are identical to it.
+ *  - Scratch limit: 256 bytes, of which each call uses the status word and
+ *    one work counter.  No problem size changes that; a call that would need
+ *    more than the array holds returns RA_ERR_UNSUPPORTED.
+ *  - The first call on each device looks the array up (cudaGetSymbolAddress)
+ *    with that device current; make that first call before any stream
+ *    capture.
+ *  - All calls share the array, which keeps the last call's contents: each
+ *    call clears the status word and the counter at its start (in-stream
+ *    memsets).  Calls that overlap on the GPU (e.g. on different streams)
+ *    race on the array and may compute wrong results; issue them on one
+ *    stream or order them.
+ *  - Device-side errors (malformed cu_seqlens, an expired wait) are latched in
+ *    the array's status word, which ring_attn_status does not read.
+ */
+ra_status ring_attn_fwd_noalloc(const void* q, const void* k, const void* v,
+                                void* out, float* lse, int batch, int heads,
+                                int seqlen, int d_head, int n_ring_blocks,
+                                int layout, int causal, float softmax_scale,
+                                int max_ring_passes, const int32_t* cu_seqlens,
+                                int dtype, void* stream);
+
+/*
  * ring_attn_status -- synchronize `stream`, then return and clear the current
  * device's status word (RA_OK when no device-side error was latched since the
  * last call).  Returns RA_ERR_CUDA when the synchronization itself fails.

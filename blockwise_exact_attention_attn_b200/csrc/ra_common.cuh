@@ -125,6 +125,19 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy reads (tensor-core operands, TMA).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
 // D[tmem] (+)= A[smem desc] * B[smem desc]; kind::f16 (bf16 inputs, fp32 acc).
 __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                         uint32_t idesc, uint32_t accumulate) {
@@ -238,6 +251,22 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA and integer pipes, for x <= 126: x = j + f with j =
+// round(x) (the 1.5 * 2^23 addition leaves j in the low mantissa bits) and
+// |f| <= 1/2; 2^f from a cubic with constant term exactly 1, fitted to the
+// relative error of 2^f on [-1/2, 1/2] (Lawson-weighted least squares; max
+// relative error 1.02e-4 in fp32 Horner form); j is added to the exponent
+// field.  x <= -127 (and -inf) gives exactly +0; x = 0 gives exactly 1.
+__device__ __forceinline__ float exp2_poly3(float x) {
+  x = fmaxf(x, -127.0f);
+  const float t = __fadd_rn(x, 12582912.0f);
+  const float f = __fsub_rn(x, __fsub_rn(t, 12582912.0f));
+  const float p = fmaf(fmaf(fmaf(0.05500892922282219f, f, 0.2422109693288803f), f,
+                            0.6932829022407532f),
+                       f, 1.0f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

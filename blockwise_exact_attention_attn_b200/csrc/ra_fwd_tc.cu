@@ -15,30 +15,33 @@
 // Persistent CTAs (one per SM, 384 threads) claim work items (two query
 // tiles of one (sequence, head)) from a per-launch counter, in item order
 // (heaviest causal ranges first); the pipelines run across item boundaries:
-// the next item's Q is loaded
-// as soon as the last S MMA of the current one is done (q_free), and its
-// first PV MMA waits only until the softmax warps have read O out (o_free).
+// the next item's Q is loaded as soon as the last S MMA of the current one is
+// done (q_free), and its first PV MMA waits only until the softmax warps have
+// read O out (o_free).
 // Warp roles:
 //   warps 0-3  softmax for query tile 0 (one TMEM lane = one query row each)
 //   warps 4-7  softmax for query tile 1
-//   warp  8    TMA producer: Q tiles once, then K and V tiles through an
-//              NS-slot shared-memory ring guarded by mbarriers
-//   warp  9    MMA issuer: S_i = Q_i K^T and O_i += P_i V as tcgen05.mma,
-//              completion signalled with tcgen05.commit
+//   warp  8    TMA producer: Q once per item; K and V tiles into one ring of
+//              shared-memory slots in the order K(0), K(1), V(0), K(2), V(1),
+//              ... (the order in which the MMA issuers consume them)
+//   warps 9,11 MMA issuers, one per query tile i: S_i = Q_i K^T into tensor
+//              memory and O_i += P_i V with P_i from shared memory, as
+//              tcgen05.mma; completion signalled with tcgen05.commit.  Two
+//              issuers keep the tensor pipe fed while one of them waits on a
+//              barrier (a tcgen05.mma group issues at about the rate it runs).
 //   warp  10   schedule builder: runs the ring-order tile walk (ra_sched.h)
 //              and publishes the visited kv tiles with their per-query-tile
-//              class into a shared-memory ring of small list chunks (the
-//              first chunk is ready after a few entries)
-//   warp  11   idle (completes the control warpgroup, whose register budget
-//              is handed to the softmax warpgroups with setmaxnreg)
-// Tensor memory (512 columns): S_0 | S_1 | O_0 | O_1; P_i (bf16) is written
-// over the first BN/2 columns of S_i once its scores are in registers.
+//              class into a shared-memory ring of small list chunks
+// The control warpgroup (warps 8-11) hands registers to the softmax
+// warpgroups with setmaxnreg.
+// Tensor memory (512 columns): S_0 | S_1 | O_0 | O_1.  Shared memory: Q_0,
+// Q_1, the K/V ring, P_0, P_1 (bf16, 128-byte swizzle), the list.
 //
-// Issue order of the MMA warp for consecutive kv tiles t-1, t:
-//   PV_0(t-1), S_0(t), PV_1(t-1), S_1(t)
-// so the tensor core computes S of one query tile while the softmax warps of
-// the other tile work, and a finished S_i(t) implies PV_i(t-1) finished
-// (commits track all earlier MMAs), which makes the O rescale safe.
+// Per kv tile t issuer i issues S_i(t+1) as soon as softmax i has loaded
+// S_i(t) into registers (s_free), then PV_i(t) once P_i(t) is in shared
+// memory (p_full).  The tensor core so computes the next scores while the
+// softmax warps still work on the current ones.  pv_done tells softmax i that
+// PV_i(t) finished: P_i may be overwritten and O_i is stable for a rescale.
 //
 // The running max is only moved when it grows by more than kRescaleLog2
 // (in log2 units); until then exponentials are taken against the stale max
@@ -60,11 +63,12 @@ constexpr int kTcQT = 2;            // query tiles per CTA
 constexpr int kTcBN = 128;          // keys per kv tile
 constexpr int kTcThreads = 384;     // 2 softmax warpgroups + 1 control warpgroup
 constexpr int kTcProducerWarp = 8;
-constexpr int kTcMmaWarp = 9;
+constexpr int kTcMmaWarp = 9;      // issuer of query tile 0 (allocates TMEM)
+constexpr int kTcMmaWarp1 = 11;    // issuer of query tile 1
 constexpr int kTcListWarp = 10;
 constexpr int kListChunk = 16;      // entries per schedule-list chunk (published at once)
-constexpr int kListBufs = 32;       // chunks in the shared-memory ring
-constexpr int kListConsumers = 10;  // producer, MMA, 8 softmax warps
+constexpr int kListBufs = 16;       // chunks in the shared-memory ring
+constexpr int kListConsumers = 11;  // producer, 2 MMA issuers, 8 softmax warps
 // Register split.  Launch: 384 threads x 168 = 64512 registers.  After the
 // split: 256 softmax threads x 176 + 128 control threads x 152 = 64512.
 constexpr int kRegsSoftmax = 176;
@@ -77,31 +81,38 @@ struct TcCfg {
   static constexpr int kPanels = D / 64;                    // 128-byte swizzle panels
   static constexpr int kPanelBytes = kTcBM * 128;           // 128 rows x 128 B
   static constexpr int kTileBytes = kPanels * kPanelBytes;  // one Q/K/V tile
-  static constexpr int kStages = D == 128 ? 4 : 8;          // K/V slots
+  static constexpr int kStages = D == 128 ? 3 : 6;          // K/V ring slots
+  static constexpr int kPBytes = kTcBM * kTcBN * 2;         // one P tile (2 panels)
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = kTcQT * kTileBytes;
-  static constexpr int kListOff = kKVOff + kStages * kTileBytes;
+  static constexpr int kPOff = kKVOff + kStages * kTileBytes;
+  static constexpr int kListOff = kPOff + kTcQT * kPBytes;
   static constexpr int kCtrlOff = kListOff + kListBufs * kListChunk * 4;
-  static constexpr int kSmemBytes = kCtrlOff + 1024 + 1024;  // + ctrl + align slack
+  static constexpr int kCtrlBytes = 512;
+  static constexpr int kSmemBytes = kCtrlOff + kCtrlBytes + 1024;  // + align slack
   static constexpr uint32_t kColS = 0;                      // S_i at i * 128
   static constexpr uint32_t kColO = 256;                    // O_i at 256 + i * D
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
 struct TcCtrl {
   uint64_t q_full;
   uint64_t q_free;
-  uint64_t kv_full[8];
-  uint64_t kv_empty[8];
+  uint64_t kv_full[6];
+  uint64_t kv_empty[6];
   uint64_t s_full[kTcQT];
+  uint64_t s_free[kTcQT];
   uint64_t p_full[kTcQT];
+  uint64_t pv_done[kTcQT];
   uint64_t o_full[kTcQT];
   uint64_t o_free[kTcQT];
   uint64_t list_full[kListBufs];
   uint64_t list_empty[kListBufs];
-  uint64_t drain;
+  uint64_t drain[kTcQT];
   uint32_t tmem_base;
   int abort;
 };
+static_assert(sizeof(TcCtrl) <= 512, "control block");
 
 struct TcMaps {
   CUtensorMap q, k, v;
@@ -149,16 +160,17 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t qdesc, uint64
   }
 }
 
-// O (+)= P V for one query tile: A = P from tensor memory (128 x 128 bf16,
-// 8 columns per 16 keys), B = V tile MN-major (N = D split in 64-element
-// panels, LBO = panel stride; 8-key groups 1024 bytes apart); step kk starts
-// 16 keys (2048 bytes, 128 units) further.
+// O (+)= P V for one query tile: A = P from shared memory (128 x 128 bf16,
+// K-major in two 64-key panels, like Q), B = V tile MN-major (N = D split in
+// 64-element panels, LBO = panel stride; 8-key groups 1024 bytes apart).
+// Step kk covers 16 keys.
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t vdesc,
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint64_t pdesc, uint64_t vdesc,
                                          uint32_t idesc, bool accumulate) {
 #pragma unroll
   for (int kk = 0; kk < kTcBN / 16; ++kk) {
-    umma_ts(d_tmem, p_tmem + kk * 8, vdesc + (uint64_t)(kk * 128), idesc,
+    const uint64_t aoff = (uint64_t)((kk >> 2) * ((kTcBM * 128) >> 4) + (kk & 3) * 2);
+    umma_ss(d_tmem, pdesc + aoff, vdesc + (uint64_t)(kk * 128), idesc,
             (accumulate || kk > 0) ? 1u : 0u);
   }
 }
@@ -260,6 +272,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                   int claim_limit) {
   using C = TcCfg<D>;
   constexpr int kRows = kTcBM * kTcQT;  // query rows per work item
+  constexpr int KVS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -273,22 +286,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   int* list = reinterpret_cast<int*>(smem + C::kListOff);
   if (threadIdx.x == 0) {
     mbar_init(&ctrl->q_full, 1);
-    mbar_init(&ctrl->q_free, 1);
-    for (int s = 0; s < C::kStages; ++s) {
+    mbar_init(&ctrl->q_free, kTcQT);  // one commit per issuer
+    for (int s = 0; s < KVS; ++s) {
       mbar_init(&ctrl->kv_full[s], 1);
-      mbar_init(&ctrl->kv_empty[s], 1);
+      mbar_init(&ctrl->kv_empty[s], kTcQT);
     }
     for (int i = 0; i < kTcQT; ++i) {
       mbar_init(&ctrl->s_full[i], 1);
+      mbar_init(&ctrl->s_free[i], kTcBM);
       mbar_init(&ctrl->p_full[i], kTcBM);
+      mbar_init(&ctrl->pv_done[i], 1);
       mbar_init(&ctrl->o_full[i], 1);
       mbar_init(&ctrl->o_free[i], kTcBM);
+      mbar_init(&ctrl->drain[i], 1);
     }
     for (int b = 0; b < kListBufs; ++b) {
       mbar_init(&ctrl->list_full[b], 1);
       mbar_init(&ctrl->list_empty[b], kListConsumers);
     }
-    mbar_init(&ctrl->drain, 1);
     ctrl->abort = 0;
     mbar_fence_init();
   }
@@ -378,6 +393,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
    } else if (warp == kTcProducerWarp) {
     // ---------------------------------------------------------- producer
+    // Ring order K(0), K(1), V(0), K(2), V(1), ...: a K tile is needed one
+    // kv tile before the V tile of the same position.
     if (lane == 0) {
       tma_prefetch_desc(&maps.q);
       tma_prefetch_desc(&maps.k);
@@ -385,6 +402,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     int n = 0, k = 0;
     bool ok = true;
+    auto load = [&](const CUtensorMap* map, int h, int row) -> bool {
+      const int slot = n % KVS;
+      if (n >= KVS && !mbar_wait(&ctrl->kv_empty[slot], ((n / KVS) - 1) & 1, abort_flag))
+        return false;
+      uint8_t* dst = smem + C::kKVOff + slot * C::kTileBytes;
+      mbar_arrive_expect_tx(&ctrl->kv_full[slot], C::kTileBytes);
+      for (int pn = 0; pn < C::kPanels; ++pn)
+        tma_load_3d(dst + pn * C::kPanelBytes, map, &ctrl->kv_full[slot], pn * 64, h, row);
+      ++n;
+      return true;
+    };
     while (ok) {
       int h = 0;
       if (lane == 0) ok = rd.next(&h, abort_flag);
@@ -393,7 +421,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!ok || h == kAllDone) break;
       const SeqWork it = find_work_item(p, kRows, header_item(h));
       if (lane == 0) {
-        // Q of this item once the previous item's last S MMA is done
+        // Q of this item once the previous item's last S MMAs are done
         if (k > 0) ok = mbar_wait(&ctrl->q_free, (k - 1) & 1, abort_flag);
         if (ok) {
           uint8_t* qs = smem + C::kQOff;
@@ -404,25 +432,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               tma_load_3d(qs + i * C::kTileBytes + pn * C::kPanelBytes, &maps.q,
                           &ctrl->q_full, pn * 64, it.h, it.base + q0 + i * kTcBM);
         }
-        int e;
+        int e, prev = -1;
         while (ok) {
           ok = rd.next(&e, abort_flag);
-          if (!ok || e < 0) break;
-          const int kt = entry_tile(e);
-          for (int which = 0; which < 2 && ok; ++which) {
-            const int slot = n % C::kStages;
-            if (n >= C::kStages) {
-              ok = mbar_wait(&ctrl->kv_empty[slot], ((n / C::kStages) - 1) & 1, abort_flag);
-              if (!ok) break;
-            }
-            uint8_t* dst = smem + C::kKVOff + slot * C::kTileBytes;
-            mbar_arrive_expect_tx(&ctrl->kv_full[slot], C::kTileBytes);
-            const CUtensorMap* map = which == 0 ? &maps.k : &maps.v;
-            for (int pn = 0; pn < C::kPanels; ++pn)
-              tma_load_3d(dst + pn * C::kPanelBytes, map, &ctrl->kv_full[slot], pn * 64, it.h,
-                          it.base + kt * kTcBN);
-            ++n;
-          }
+          if (!ok) break;
+          if (e >= 0) ok = load(&maps.k, it.h, it.base + entry_tile(e) * kTcBN);
+          if (ok && prev >= 0) ok = load(&maps.v, it.h, it.base + entry_tile(prev) * kTcBN);
+          if (e < 0) break;
+          prev = e;
         }
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -432,29 +449,60 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       *abort_flag = 1;
       latch_status(p.status, ST_TIMEOUT);
       // let the copies already issued land before the CTA can exit
-      for (int u = (n > C::kStages ? n - C::kStages : 0); u < n; ++u)
-        mbar_wait(&ctrl->kv_full[u % C::kStages], (u / C::kStages) & 1, nullptr);
+      for (int u = (n > KVS ? n - KVS : 0); u < n; ++u)
+        mbar_wait(&ctrl->kv_full[u % KVS], (u / KVS) & 1, nullptr);
       if (k > 0) mbar_wait(&ctrl->q_full, (k - 1) & 1, nullptr);
     }
     __syncwarp();
-   } else if (warp == kTcMmaWarp) {
-    // ---------------------------------------------------------- MMA issuer
+   } else {
+    // ---------------------------------------------------------- MMA issuers
+    // Issuer qi, per kv tile t: S_qi(t+1) as soon as softmax qi has read
+    // S_qi(t) (s_free), then PV_qi(t) once P_qi(t) is written (p_full).  Both
+    // issuers walk the K/V ring in load order; a slot is released by a commit
+    // of each of them (its count is 2).
+    const int qi = warp == kTcMmaWarp ? 0 : 1;
     // a negative softmax scale is applied as S = (-Q) K^T times |scale|
     const uint32_t idesc_s =
         idesc_bf16_f32(kTcBM, kTcBN, 0) | (p.scale_log2 < 0.f ? (1u << 13) : 0u);
     constexpr uint32_t idesc_o = idesc_bf16_f32(kTcBM, D, 1);
-    // base descriptors: K-major tiles (Q, K) and MN-major tiles (V)
-    const uint32_t qs = smem_u32(smem + C::kQOff);
-    const uint32_t kvs = smem_u32(smem + C::kKVOff);
-    uint64_t qdesc[kTcQT];
-#pragma unroll
-    for (int i = 0; i < kTcQT; ++i) qdesc[i] = smem_desc_sw128(qs + i * C::kTileBytes, 16, 1024);
-    const uint64_t kdesc0 = smem_desc_sw128(kvs, 16, 1024);
-    const uint64_t vdesc0 = smem_desc_sw128(kvs, C::kPanelBytes, 1024);
+    // base descriptors: K-major tiles (Q, K, P) and MN-major tiles (V)
+    const uint64_t qdesc =
+        smem_desc_sw128(smem_u32(smem + C::kQOff + qi * C::kTileBytes), 16, 1024);
+    const uint64_t pdesc = smem_desc_sw128(smem_u32(smem + C::kPOff + qi * C::kPBytes), 16, 1024);
+    const uint64_t kdesc0 = smem_desc_sw128(smem_u32(smem + C::kKVOff), 16, 1024);
+    const uint64_t vdesc0 = smem_desc_sw128(smem_u32(smem + C::kKVOff), C::kPanelBytes, 1024);
     constexpr uint64_t kSlotStep = (uint64_t)(C::kTileBytes >> 4);
-    uint32_t pphase[kTcQT] = {0, 0};
+    const uint32_t tSq = tmem + C::kColS + qi * kTcBN;
+    const uint32_t tOq = tmem + C::kColO + qi * D;
+    uint32_t ns = 0;  // S_qi issued so far
+    uint32_t pphase = 0;
     int n = 0, k = 0;
     bool ok = true, issued_any = false;
+    // next ring slot, once its tile has landed
+    auto take = [&]() -> int {
+      const int slot = n % KVS;
+      ok = mbar_wait(&ctrl->kv_full[slot], (n / KVS) & 1, abort_flag);
+      ++n;
+      if (ok) tc_fence_after();
+      return slot;
+    };
+    // S_qi = Q_qi K^T if query tile qi visits kv tile entry e
+    auto issue_s = [&](int e) {
+      const int slot = take();
+      if (!ok) return;
+      if (entry_cls(e, qi) != CLS_EMPTY) {
+        if (ns > 0) {
+          ok = mbar_wait(&ctrl->s_free[qi], (ns - 1) & 1, abort_flag);
+          if (!ok) return;
+          tc_fence_after();
+        }
+        issue_qk<D>(tSq, qdesc, kdesc0 + slot * kSlotStep, idesc_s);
+        umma_commit(&ctrl->s_full[qi]);
+        ++ns;
+        issued_any = true;
+      }
+      umma_commit(&ctrl->kv_empty[slot]);
+    };
     while (ok) {
       int h = 0;
       if (lane == 0) ok = rd.next(&h, abort_flag);
@@ -464,84 +512,55 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0) {
         ok = mbar_wait(&ctrl->q_full, k & 1, abort_flag);
         tc_fence_after();
-        bool started[kTcQT] = {false, false};
-        // the previous item's O_i must have been read out before it is overwritten
-        bool ofree_pending[kTcQT] = {k > 0, k > 0};
-        auto wait_ofree = [&](int i) {
-          if (ok && ofree_pending[i]) {
-            ok = mbar_wait(&ctrl->o_free[i], (k - 1) & 1, abort_flag);
-            ofree_pending[i] = false;
+        bool started = false;
+        // the previous item's O_qi must have been read out before it is overwritten
+        bool ofree_pending = k > 0;
+        auto wait_ofree = [&]() {
+          if (ok && ofree_pending) {
+            ok = mbar_wait(&ctrl->o_free[qi], (k - 1) & 1, abort_flag);
+            ofree_pending = false;
             tc_fence_after();
           }
         };
-        int e = -1, ep = -1;
+        int e = -1;
         if (ok) ok = rd.next(&e, abort_flag);
         if (ok && e >= 0) {
-          const int slot = n % C::kStages;
-          ok = mbar_wait(&ctrl->kv_full[slot], (n / C::kStages) & 1, abort_flag);
-          ++n;
-          if (ok) {
-            tc_fence_after();
-            for (int i = 0; i < kTcQT; ++i)
-              if (entry_cls(e, i) != CLS_EMPTY) {
-                issue_qk<D>(tmem + C::kColS + i * kTcBN, qdesc[i], kdesc0 + slot * kSlotStep,
-                            idesc_s);
-                umma_commit(&ctrl->s_full[i]);
-              }
-            umma_commit(&ctrl->kv_empty[slot]);
-            issued_any = true;
-          }
-          ep = e;
+          issue_s(e);
+          int ep = e;
           while (ok) {
-            const int slot_v = n % C::kStages;
-            ok = mbar_wait(&ctrl->kv_full[slot_v], (n / C::kStages) & 1, abort_flag);
-            ++n;
-            if (!ok) break;
             ok = rd.next(&e, abort_flag);
             if (!ok) break;
             const bool has = e >= 0;
-            int slot_k = 0;
             if (has) {
-              slot_k = n % C::kStages;
-              ok = mbar_wait(&ctrl->kv_full[slot_k], (n / C::kStages) & 1, abort_flag);
-              ++n;
+              issue_s(e);
               if (!ok) break;
             } else {
-              // every S of this item is issued: Q may be replaced once they finish
+              // every S_qi of this item is issued: Q may be replaced once they finish
               umma_commit(&ctrl->q_free);
             }
-            tc_fence_after();
-            for (int i = 0; i < kTcQT && ok; ++i) {
-              if (entry_cls(ep, i) != CLS_EMPTY) {
-                ok = mbar_wait(&ctrl->p_full[i], pphase[i], abort_flag);
-                pphase[i] ^= 1;
-                if (!ok) break;
-                tc_fence_after();
-                if (!started[i]) wait_ofree(i);
-                if (!ok) break;
-                issue_pv<D>(tmem + C::kColO + i * D, tmem + C::kColS + i * kTcBN,
-                            vdesc0 + slot_v * kSlotStep, idesc_o, started[i]);
-                started[i] = true;
-              }
-              if (has && entry_cls(e, i) != CLS_EMPTY) {
-                issue_qk<D>(tmem + C::kColS + i * kTcBN, qdesc[i], kdesc0 + slot_k * kSlotStep,
-                            idesc_s);
-                umma_commit(&ctrl->s_full[i]);
-              }
-            }
+            const int slot_v = take();
             if (!ok) break;
+            if (entry_cls(ep, qi) != CLS_EMPTY) {
+              ok = mbar_wait(&ctrl->p_full[qi], pphase, abort_flag);
+              pphase ^= 1;
+              if (!ok) break;
+              tc_fence_after();
+              if (!started) wait_ofree();
+              if (!ok) break;
+              issue_pv<D>(tOq, pdesc, vdesc0 + slot_v * kSlotStep, idesc_o, started);
+              umma_commit(&ctrl->pv_done[qi]);
+              started = true;
+            }
             umma_commit(&ctrl->kv_empty[slot_v]);
             if (!has) break;
-            umma_commit(&ctrl->kv_empty[slot_k]);
             ep = e;
           }
         } else if (ok) {
           umma_commit(&ctrl->q_free);  // an item without tiles
         }
         if (ok) {
-          for (int i = 0; i < kTcQT; ++i) wait_ofree(i);
-          if (ok)
-            for (int i = 0; i < kTcQT; ++i) umma_commit(&ctrl->o_full[i]);
+          wait_ofree();
+          if (ok) umma_commit(&ctrl->o_full[qi]);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -552,8 +571,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       latch_status(p.status, ST_TIMEOUT);
       if (issued_any) {
         // wait (bounded) for the MMAs already issued before TMEM is freed
-        umma_commit(&ctrl->drain);
-        mbar_wait(&ctrl->drain, 0, nullptr);
+        umma_commit(&ctrl->drain[qi]);
+        mbar_wait(&ctrl->drain[qi], 0, nullptr);
       }
     }
     __syncwarp();
@@ -567,8 +586,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::kColS + tile * kTcBN;
     const uint32_t tO = tmem + lane_off + C::kColO + tile * D;
+    // this row of P_tile: 128-byte rows, 16-byte chunks XOR-swizzled by row % 8,
+    // keys 0-63 in the first 16 KB panel and keys 64-127 in the second
+    const uint32_t prow = smem_u32(smem + C::kPOff + tile * C::kPBytes) + (uint32_t)r * 128u;
+    const uint32_t pswz = (uint32_t)(r & 7);
     const float sl2 = fabsf(p.scale_log2);  // > 0; the sign is folded into the MMA
     uint32_t sphase = 0;
+    uint32_t np = 0;  // P tiles written so far
     int k = 0;
     bool ok = true;
 
@@ -608,6 +632,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int c = 0; c < kTcBN; c += 32) RA_TMEM_LD32(tS + c, (xr + c));
           tmem_wait_ld();
         }
+        // S_tile is in registers: the next S may be computed into its columns
+        tc_fence_before();
+        mbar_arrive(&ctrl->s_free[tile]);
         const int k0 = entry_tile(e) * kTcBN;
         const int nk = min(kTcBN, L - k0);
         if (cls == CLS_PARTIAL || nk < kTcBN) {
@@ -629,18 +656,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           m_ref = m_tile;
         }
         const float msub = m_ref == -INFINITY ? 0.f : m_ref;
+        // P row in registers (bf16 pairs) while the previous PV still runs
         float rs4[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial row sums
+        uint32_t pk[kTcBN / 2];
 #pragma unroll
-        for (int q = 0; q < kTcBN / 32; ++q) {
-          uint32_t pk[16];
+        for (int j = 0; j < kTcBN / 2; ++j) {
+          const float a = ex2_approx(fmaf(x[2 * j], sl2, -msub));
+          const float b = ex2_approx(fmaf(x[2 * j + 1], sl2, -msub));
+          rs4[j & 3] += a + b;
+          pk[j] = pack_bf16x2(a, b);
+        }
+        // the previous PV of this query tile has finished reading P and
+        // writing O
+        if (np > 0) {
+          ok = warp_wait(&ctrl->pv_done[tile], (np - 1) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+        }
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float a = ex2_approx(fmaf(x[q * 32 + 2 * j], sl2, -msub));
-            const float b = ex2_approx(fmaf(x[q * 32 + 2 * j + 1], sl2, -msub));
-            rs4[j & 3] += a + b;
-            pk[j] = pack_bf16x2(a, b);
-          }
-          RA_TMEM_ST16(tS + q * 16, pk);
+        for (int g8 = 0; g8 < kTcBN / 8; ++g8) {
+          const uint32_t addr =
+              prow + (uint32_t)(g8 >> 3) * (kTcBM * 128u) + ((((uint32_t)g8 & 7u) ^ pswz) << 4);
+          st_shared_v4(addr, pk[4 * g8], pk[4 * g8 + 1], pk[4 * g8 + 2], pk[4 * g8 + 3]);
         }
         l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
         if (!first && __any_sync(0xffffffffu, need)) {
@@ -654,10 +691,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
             RA_TMEM_ST32(tO + c, o);
           }
+          tmem_wait_st();
         }
-        tmem_wait_st();
+        fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&ctrl->p_full[tile]);
+        ++np;
         first = false;
       }
       if (!ok) break;

@@ -253,6 +253,44 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Paired fp32 arithmetic (sm_100 f32x2 instructions): half the issue slots of
+// two scalar operations.  A pair travels as one 64-bit register, low = first.
+__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float f32x2_lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f32x2_hi(uint64_t v) {
+  return __uint_as_float((uint32_t)(v >> 32));
+}
+// (d0, d1) = (a0, a1) * b2 + c2, round to nearest
+__device__ __forceinline__ void ffma2(float a0, float a1, uint64_t b2, uint64_t c2, float& d0,
+                                      float& d1) {
+  asm("{\n\t.reg .b64 ra, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "fma.rn.f32x2 rd, ra, %4, %5;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "l"(b2), "l"(c2));
+}
+// acc + (a0, a1), round to nearest
+__device__ __forceinline__ uint64_t fadd2(uint64_t acc, float a0, float a1) {
+  uint64_t r;
+  asm("{\n\t.reg .b64 ra;\n\t"
+      "mov.b64 ra, {%1, %2};\n\t"
+      "add.rn.f32x2 %0, %3, ra;\n\t}"
+      : "=l"(r)
+      : "f"(a0), "f"(a1), "l"(acc));
+  return r;
+}
+// max of three (one instruction on sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // 2^x on the FMA and integer pipes, for x <= 126: x = j + f with j =
 // round(x) (the 1.5 * 2^23 addition leaves j in the low mantissa bits) and
 // |f| <= 1/2; 2^f from a cubic with constant term exactly 1, fitted to the

@@ -63,12 +63,14 @@ constexpr int kTcQT = 2;            // query tiles per CTA
 constexpr int kTcBN = 128;          // keys per kv tile
 constexpr int kTcThreads = 384;     // 2 softmax warpgroups + 1 control warpgroup
 constexpr int kTcProducerWarp = 8;
-constexpr int kTcMmaWarp = 9;      // issuer of query tile 0 (allocates TMEM)
-constexpr int kTcMmaWarp1 = 11;    // issuer of query tile 1
+constexpr int kTcMmaWarp = 9;      // MMA issuer (allocates TMEM)
+constexpr int kTcMmaWarp1 = 11;    // second MMA issuer when kTcIssuers == 2
 constexpr int kTcListWarp = 10;
+// MMA issuer warps: 2 = one per query tile, 1 = warp 9 issues for both tiles
+constexpr int kTcIssuers = 2;
 constexpr int kListChunk = 16;      // entries per schedule-list chunk (published at once)
 constexpr int kListBufs = 16;       // chunks in the shared-memory ring
-constexpr int kListConsumers = 11;  // producer, 2 MMA issuers, 8 softmax warps
+constexpr int kListConsumers = 9 + kTcIssuers;  // producer, issuers, 8 softmax warps
 // Register split.  Launch: 384 threads x 168 = 64512 registers.  After the
 // split: 256 softmax threads x 176 + 128 control threads x 152 = 64512.
 constexpr int kRegsSoftmax = 176;
@@ -286,10 +288,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   int* list = reinterpret_cast<int*>(smem + C::kListOff);
   if (threadIdx.x == 0) {
     mbar_init(&ctrl->q_full, 1);
-    mbar_init(&ctrl->q_free, kTcQT);  // one commit per issuer
+    mbar_init(&ctrl->q_free, kTcIssuers);  // one commit per issuer
     for (int s = 0; s < KVS; ++s) {
       mbar_init(&ctrl->kv_full[s], 1);
-      mbar_init(&ctrl->kv_empty[s], kTcQT);
+      mbar_init(&ctrl->kv_empty[s], kTcIssuers);
     }
     for (int i = 0; i < kTcQT; ++i) {
       mbar_init(&ctrl->s_full[i], 1);
@@ -454,28 +456,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (k > 0) mbar_wait(&ctrl->q_full, (k - 1) & 1, nullptr);
     }
     __syncwarp();
-   } else {
+   } else if (warp == kTcMmaWarp || kTcIssuers == 2) {
     // ---------------------------------------------------------- MMA issuers
-    // Issuer qi, per kv tile t: S_qi(t+1) as soon as softmax qi has read
-    // S_qi(t) (s_free), then PV_qi(t) once P_qi(t) is written (p_full).  Both
-    // issuers walk the K/V ring in load order; a slot is released by a commit
-    // of each of them (its count is 2).
-    const int qi = warp == kTcMmaWarp ? 0 : 1;
+    // Issuer of query tiles [i0, i1), per kv tile t: S_i(t+1) as soon as
+    // softmax i has read S_i(t) (s_free), then PV_i(t) once P_i(t) is
+    // written (p_full).  Every issuer walks the K/V ring in load order; a
+    // slot is released by one commit of each issuer.
+    const int i0 = (kTcIssuers == 2 && warp == kTcMmaWarp1) ? 1 : 0;
+    const int i1 = kTcIssuers == 2 ? i0 + 1 : kTcQT;
     // a negative softmax scale is applied as S = (-Q) K^T times |scale|
     const uint32_t idesc_s =
         idesc_bf16_f32(kTcBM, kTcBN, 0) | (p.scale_log2 < 0.f ? (1u << 13) : 0u);
     constexpr uint32_t idesc_o = idesc_bf16_f32(kTcBM, D, 1);
     // base descriptors: K-major tiles (Q, K, P) and MN-major tiles (V)
-    const uint64_t qdesc =
-        smem_desc_sw128(smem_u32(smem + C::kQOff + qi * C::kTileBytes), 16, 1024);
-    const uint64_t pdesc = smem_desc_sw128(smem_u32(smem + C::kPOff + qi * C::kPBytes), 16, 1024);
+    const uint64_t qdesc0 = smem_desc_sw128(smem_u32(smem + C::kQOff), 16, 1024);
+    const uint64_t pdesc0 = smem_desc_sw128(smem_u32(smem + C::kPOff), 16, 1024);
     const uint64_t kdesc0 = smem_desc_sw128(smem_u32(smem + C::kKVOff), 16, 1024);
     const uint64_t vdesc0 = smem_desc_sw128(smem_u32(smem + C::kKVOff), C::kPanelBytes, 1024);
     constexpr uint64_t kSlotStep = (uint64_t)(C::kTileBytes >> 4);
-    const uint32_t tSq = tmem + C::kColS + qi * kTcBN;
-    const uint32_t tOq = tmem + C::kColO + qi * D;
-    uint32_t ns = 0;  // S_qi issued so far
-    uint32_t pphase = 0;
+    constexpr uint64_t kQStep = (uint64_t)(C::kTileBytes >> 4);
+    constexpr uint64_t kPStep = (uint64_t)(C::kPBytes >> 4);
+    uint32_t ns[kTcQT] = {0, 0};  // S_i issued so far
+    uint32_t pphase[kTcQT] = {0, 0};
     int n = 0, k = 0;
     bool ok = true, issued_any = false;
     // next ring slot, once its tile has landed
@@ -486,19 +488,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (ok) tc_fence_after();
       return slot;
     };
-    // S_qi = Q_qi K^T if query tile qi visits kv tile entry e
+    // S_i = Q_i K^T for this issuer's query tiles that visit kv tile entry e
     auto issue_s = [&](int e) {
       const int slot = take();
       if (!ok) return;
-      if (entry_cls(e, qi) != CLS_EMPTY) {
-        if (ns > 0) {
-          ok = mbar_wait(&ctrl->s_free[qi], (ns - 1) & 1, abort_flag);
+      for (int i = i0; i < i1; ++i) {
+        if (entry_cls(e, i) == CLS_EMPTY) continue;
+        if (ns[i] > 0) {
+          ok = mbar_wait(&ctrl->s_free[i], (ns[i] - 1) & 1, abort_flag);
           if (!ok) return;
           tc_fence_after();
         }
-        issue_qk<D>(tSq, qdesc, kdesc0 + slot * kSlotStep, idesc_s);
-        umma_commit(&ctrl->s_full[qi]);
-        ++ns;
+        issue_qk<D>(tmem + C::kColS + i * kTcBN, qdesc0 + i * kQStep,
+                    kdesc0 + slot * kSlotStep, idesc_s);
+        umma_commit(&ctrl->s_full[i]);
+        ++ns[i];
         issued_any = true;
       }
       umma_commit(&ctrl->kv_empty[slot]);
@@ -512,13 +516,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0) {
         ok = mbar_wait(&ctrl->q_full, k & 1, abort_flag);
         tc_fence_after();
-        bool started = false;
-        // the previous item's O_qi must have been read out before it is overwritten
-        bool ofree_pending = k > 0;
-        auto wait_ofree = [&]() {
-          if (ok && ofree_pending) {
-            ok = mbar_wait(&ctrl->o_free[qi], (k - 1) & 1, abort_flag);
-            ofree_pending = false;
+        bool started[kTcQT] = {false, false};
+        // the previous item's O_i must have been read out before it is overwritten
+        bool ofree_pending[kTcQT] = {k > 0, k > 0};
+        auto wait_ofree = [&](int i) {
+          if (ok && ofree_pending[i]) {
+            ok = mbar_wait(&ctrl->o_free[i], (k - 1) & 1, abort_flag);
+            ofree_pending[i] = false;
             tc_fence_after();
           }
         };
@@ -535,22 +539,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               issue_s(e);
               if (!ok) break;
             } else {
-              // every S_qi of this item is issued: Q may be replaced once they finish
+              // every S of this item is issued: Q may be replaced once they finish
               umma_commit(&ctrl->q_free);
             }
             const int slot_v = take();
             if (!ok) break;
-            if (entry_cls(ep, qi) != CLS_EMPTY) {
-              ok = mbar_wait(&ctrl->p_full[qi], pphase, abort_flag);
-              pphase ^= 1;
+            for (int i = i0; i < i1 && ok; ++i) {
+              if (entry_cls(ep, i) == CLS_EMPTY) continue;
+              ok = mbar_wait(&ctrl->p_full[i], pphase[i], abort_flag);
+              pphase[i] ^= 1;
               if (!ok) break;
               tc_fence_after();
-              if (!started) wait_ofree();
+              if (!started[i]) wait_ofree(i);
               if (!ok) break;
-              issue_pv<D>(tOq, pdesc, vdesc0 + slot_v * kSlotStep, idesc_o, started);
-              umma_commit(&ctrl->pv_done[qi]);
-              started = true;
+              issue_pv<D>(tmem + C::kColO + i * D, pdesc0 + i * kPStep,
+                          vdesc0 + slot_v * kSlotStep, idesc_o, started[i]);
+              umma_commit(&ctrl->pv_done[i]);
+              started[i] = true;
             }
+            if (!ok) break;
             umma_commit(&ctrl->kv_empty[slot_v]);
             if (!has) break;
             ep = e;
@@ -559,8 +566,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           umma_commit(&ctrl->q_free);  // an item without tiles
         }
         if (ok) {
-          wait_ofree();
-          if (ok) umma_commit(&ctrl->o_full[qi]);
+          for (int i = i0; i < i1; ++i) wait_ofree(i);
+          if (ok)
+            for (int i = i0; i < i1; ++i) umma_commit(&ctrl->o_full[i]);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -571,8 +579,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       latch_status(p.status, ST_TIMEOUT);
       if (issued_any) {
         // wait (bounded) for the MMAs already issued before TMEM is freed
-        umma_commit(&ctrl->drain[qi]);
-        mbar_wait(&ctrl->drain[qi], 0, nullptr);
+        umma_commit(&ctrl->drain[i0]);
+        mbar_wait(&ctrl->drain[i0], 0, nullptr);
       }
     }
     __syncwarp();
@@ -645,7 +653,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int j = 0; j < 8; ++j) mx8[j] = x[j];
 #pragma unroll
-        for (int c = 8; c < kTcBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
+        for (int c = 8; c < kTcBN; c += 2)
+          mx8[(c >> 1) & 7] = fmax3(mx8[(c >> 1) & 7], x[c], x[c + 1]);
         const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float m_tile = mx * sl2;  // -inf stays -inf (sl2 > 0)
@@ -656,14 +665,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           m_ref = m_tile;
         }
         const float msub = m_ref == -INFINITY ? 0.f : m_ref;
-        // P row in registers (bf16 pairs) while the previous PV still runs
-        float rs4[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial row sums
+        // P row in registers (bf16 pairs) while the previous PV still runs;
+        // scale-and-subtract and the row sums in paired fp32 instructions
+        const uint64_t sc2 = f32x2_pack(sl2, sl2), ms2 = f32x2_pack(-msub, -msub);
+        uint64_t sum2[2] = {0ull, 0ull};  // two independent (even, odd) partial sums
         uint32_t pk[kTcBN / 2];
 #pragma unroll
         for (int j = 0; j < kTcBN / 2; ++j) {
-          const float a = ex2_approx(fmaf(x[2 * j], sl2, -msub));
-          const float b = ex2_approx(fmaf(x[2 * j + 1], sl2, -msub));
-          rs4[j & 3] += a + b;
+          float ya, yb;
+          ffma2(x[2 * j], x[2 * j + 1], sc2, ms2, ya, yb);
+          const float a = ex2_approx(ya);
+          const float b = ex2_approx(yb);
+          sum2[j & 1] = fadd2(sum2[j & 1], a, b);
           pk[j] = pack_bf16x2(a, b);
         }
         // the previous PV of this query tile has finished reading P and
@@ -679,7 +692,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               prow + (uint32_t)(g8 >> 3) * (kTcBM * 128u) + ((((uint32_t)g8 & 7u) ^ pswz) << 4);
           st_shared_v4(addr, pk[4 * g8], pk[4 * g8 + 1], pk[4 * g8 + 2], pk[4 * g8 + 3]);
         }
-        l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
+        l = l * alpha + ((f32x2_lo(sum2[0]) + f32x2_hi(sum2[0])) +
+                         (f32x2_lo(sum2[1]) + f32x2_hi(sum2[1])));
         if (!first && __any_sync(0xffffffffu, need)) {
           // O_row *= alpha (exactly 1.0 for rows that keep their reference)
 #pragma unroll

@@ -177,33 +177,44 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint64_t pdesc, uint64
   }
 }
 
+// Bits [lo, hi) of a 32-bit word, 0 <= lo < hi <= 32.
+__device__ __forceinline__ uint32_t bit_range(int lo, int hi) {
+  const uint32_t upto = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
+  return upto & ~((1u << lo) - 1u);
+}
+
 // Replace the scores of disallowed keys by -inf.  Keys at or beyond L (the
 // next sequence, or rows past the tensor) are always disallowed; on PARTIAL
-// tiles the ring mask is applied too.
+// tiles the ring mask is applied too.  In stored order the keys of one ring
+// block are consecutive and a query's allowed keys among them form a prefix
+// (single_block_limit), so the allowed columns of a tile are the union of one
+// interval per ring block the tile meets.
 __device__ __forceinline__ void apply_mask(float* x, const FwdParams& p, int L, bool valid,
-                                           int cls, int sq, int rq, int tq, int k0, int nk) {
-  int lim;
-  const RingGeom g = make_geom(L, p.n_ring, p.layout, p.causal, p.passes);
+                                           int cls, int rq, int tq, int k0, int nk) {
+  uint32_t mw[kTcBN / 32];  // allowed columns as 4 x 32-bit masks (indices stay compile-time)
   if (!valid || cls == CLS_FULL) {
-    lim = nk;
-  } else {
-    const int rk0 = block_of(g, k0), rk1 = block_of(g, k0 + nk - 1);
-    lim = rk0 == rk1 ? single_block_limit(g, rq, tq, rk0, k0, nk) : -1;
-  }
-  // allowed columns as 4 x 32-bit masks (indices stay compile-time)
-  uint32_t mw[kTcBN / 32];
 #pragma unroll
-  for (int w = 0; w < kTcBN / 32; ++w) {
-    if (lim >= 0) {
-      const int n = min(max(lim - 32 * w, 0), 32);
+    for (int w = 0; w < kTcBN / 32; ++w) {
+      const int n = min(max(nk - 32 * w, 0), 32);
       mw[w] = n >= 32 ? 0xffffffffu : ((1u << n) - 1u);
-    } else {
-      uint32_t bits = 0;
-      for (int bit = 0; bit < 32; ++bit) {
-        const int c = 32 * w + bit;
-        if (c < nk && allowed(g, sq, rq, tq, k0 + c)) bits |= 1u << bit;
+    }
+  } else {
+    const RingGeom g = make_geom(L, p.n_ring, p.layout, p.causal, p.passes);
+#pragma unroll
+    for (int w = 0; w < kTcBN / 32; ++w) mw[w] = 0u;
+    const int kend = k0 + nk;
+    int c = k0;
+    // at most one pass per ring block (empty blocks advance rk only)
+    for (int rk = block_of(g, k0); c < kend && rk < g.N; ++rk) {
+      const int be = min(block_start(g, rk + 1), kend);
+      if (be <= c) continue;
+      const int a = c - k0, bnd = a + single_block_limit(g, rq, tq, rk, c, be - c);
+#pragma unroll
+      for (int w = 0; w < kTcBN / 32; ++w) {
+        const int lo = max(a - 32 * w, 0), hi = min(bnd - 32 * w, 32);
+        if (hi > lo) mw[w] |= bit_range(lo, hi);
       }
-      mw[w] = bits;
+      c = be;
     }
   }
 #pragma unroll
@@ -213,13 +224,15 @@ __device__ __forceinline__ void apply_mask(float* x, const FwdParams& p, int L, 
 // Schedule-list entries: (kt << 4) | (class of query tile 1 << 2) | class of
 // query tile 0 for a visited kv tile; kItemEnd ends a work item, kAllDone ends
 // the stream, kPad fills a chunk published early, and -(item + 8) starts work
-// item `item`.  Chunks are released by every consumer after it read their
-// last entry.
+// item `item`.  A header is followed by kItemInfo entries describing the item
+// (sequence, query range, head, first row, length), decoded once by the
+// builder.  Chunks are released by every consumer after it read their last
+// entry.
 constexpr int kItemEnd = -1;
 constexpr int kAllDone = -2;
 constexpr int kPad = -3;
+constexpr int kItemInfo = 5;
 __device__ __forceinline__ int item_header(int item) { return -(item + 8); }
-__device__ __forceinline__ int header_item(int e) { return -e - 8; }
 __device__ __forceinline__ int entry_tile(int e) { return e >> 4; }
 __device__ __forceinline__ int entry_cls(int e, int i) { return (e >> (2 * i)) & 3; }
 
@@ -267,6 +280,25 @@ struct ListReader {
     return true;
   }
 };
+
+// The kItemInfo entries after a header, for one thread (kWarp false) or a
+// whole warp.
+template <bool kWarp>
+__device__ __forceinline__ bool read_item(ListReader& rd, SeqWork* it, volatile int* abort) {
+  int v[kItemInfo];
+#pragma unroll
+  for (int i = 0; i < kItemInfo; ++i) {
+    if (!(kWarp ? rd.next_warp_raw(&v[i], abort) : rd.next_raw(&v[i], abort)))
+      return false;
+  }
+  it->b = v[0];
+  it->qr = v[1];
+  it->h = v[2];
+  it->base = v[3];
+  it->L = v[4];
+  it->live = true;
+  return true;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -381,7 +413,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         TileWalk walk;
         walk.init(g, q0, qm, q1, kTcBN);
         int kt, c0, c1;
-        ok = put(item_header(item));
+        ok = put(item_header(item)) && put(it.b) && put(it.qr) && put(it.h) && put(it.base) &&
+             put(it.L);
         while (ok && walk.next(&kt, &c0, &c1)) ok = put((kt << 4) | (c1 << 2) | c0);
         if (ok) ok = put(kItemEnd);
       }
@@ -421,10 +454,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       h = __shfl_sync(0xffffffffu, h, 0);
       if (!ok || h == kAllDone) break;
-      const SeqWork it = find_work_item(p, kRows, header_item(h));
       if (lane == 0) {
-        // Q of this item once the previous item's last S MMAs are done
-        if (k > 0) ok = mbar_wait(&ctrl->q_free, (k - 1) & 1, abort_flag);
+        SeqWork it;
+        ok = read_item<false>(rd, &it, abort_flag);
+        // the item's first K enters the ring before Q waits for the previous
+        // item's last S MMAs (q_free)
+        int e = -1;
+        if (ok) ok = rd.next(&e, abort_flag);
+        if (ok && e >= 0) ok = load(&maps.k, it.h, it.base + entry_tile(e) * kTcBN);
+        if (ok && k > 0) ok = mbar_wait(&ctrl->q_free, (k - 1) & 1, abort_flag);
         if (ok) {
           uint8_t* qs = smem + C::kQOff;
           const int q0 = it.qr * kRows;
@@ -434,13 +472,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               tma_load_3d(qs + i * C::kTileBytes + pn * C::kPanelBytes, &maps.q,
                           &ctrl->q_full, pn * 64, it.h, it.base + q0 + i * kTcBM);
         }
-        int e, prev = -1;
-        while (ok) {
+        int prev = e;
+        while (ok && prev >= 0) {
           ok = rd.next(&e, abort_flag);
           if (!ok) break;
           if (e >= 0) ok = load(&maps.k, it.h, it.base + entry_tile(e) * kTcBN);
-          if (ok && prev >= 0) ok = load(&maps.v, it.h, it.base + entry_tile(prev) * kTcBN);
-          if (e < 0) break;
+          if (ok) ok = load(&maps.v, it.h, it.base + entry_tile(prev) * kTcBN);
           prev = e;
         }
       }
@@ -514,7 +551,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       h = __shfl_sync(0xffffffffu, h, 0);
       if (!ok || h == kAllDone) break;
       if (lane == 0) {
-        ok = mbar_wait(&ctrl->q_full, k & 1, abort_flag);
+        SeqWork skip;  // the item's description is not needed here
+        ok = read_item<false>(rd, &skip, abort_flag);
+        if (ok) ok = mbar_wait(&ctrl->q_full, k & 1, abort_flag);
         tc_fence_after();
         bool started[kTcQT] = {false, false};
         // the previous item's O_i must have been read out before it is overwritten
@@ -608,7 +647,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       int h;
       ok = rd.next_warp(&h, abort_flag);
       if (!ok || h == kAllDone) break;
-      const SeqWork it = find_work_item(p, kRows, header_item(h));
+      SeqWork it;
+      ok = read_item<true>(rd, &it, abort_flag);
+      if (!ok) break;
       const int L = it.L;
       const int sq = it.qr * kRows + tile * kTcBM + r;
       const bool valid = sq < L;
@@ -646,7 +687,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int k0 = entry_tile(e) * kTcBN;
         const int nk = min(kTcBN, L - k0);
         if (cls == CLS_PARTIAL || nk < kTcBN) {
-          apply_mask(x, p, L, valid, cls, sq, rq, tq, k0, nk);
+          apply_mask(x, p, L, valid, cls, rq, tq, k0, nk);
         }
         // row max as a tree of independent maxima (short dependency chains)
         float mx8[8];

@@ -5,7 +5,8 @@ none of the attention arithmetic.  Both the CUDA path and the oracle receive
 the very arrays produced here (bf16 values reach the oracle upcast exactly).
 
 Every workload draws q, k, v i.i.d. N(0, 1) from ``torch.Generator('cpu')``
-seeded per workload (fp32 draws, cast to bf16 where the workload is bf16).
+seeded per workload (fp32 draws, cast to bf16 where the workload is bf16);
+grouped-query workloads draw k and v with their own (smaller) head count.
 The varlen workload first draws its sequence lengths from the same generator
 (uniform in [1024, 7168] in fp64, rescaled to sum to the total with
 largest-remainder rounding, ties to the lower index), then the packed qkv.
@@ -40,6 +41,11 @@ class Workload:
     packed: bool = False
     n_seqs: int = 0                   # varlen only
     len_range: tuple = field(default=(1024, 7168))
+    heads_kv: int = 0                 # key/value heads (0: same as heads)
+
+    @property
+    def kv_heads(self) -> int:
+        return self.heads_kv if self.heads_kv else self.heads
 
     @property
     def softmax_scale(self) -> float:
@@ -51,7 +57,8 @@ class Workload:
 
 
 # The five workloads of the benchmark description (sizes, seeds) plus small
-# variants used by the tests.
+# variants used by the tests, and one grouped-query workload (8 query heads
+# per key/value head).
 WORKLOADS = {
     "fp32_b1_h1_s1024_d16_noncausal_n16": Workload(
         "fp32_b1_h1_s1024_d16_noncausal_n16", "f32", 1, 1, 1024, 16, False, 16,
@@ -74,6 +81,9 @@ WORKLOADS = {
     "bf16_b1_h8_s262144_d128_causal_striped_n16_p4": Workload(
         "bf16_b1_h8_s262144_d128_causal_striped_n16_p4", "bf16", 1, 8, 262144, 128, True,
         16, STRIPED, 4, 5),
+    "bf16_b1_h32_kv4_s32768_d128_causal_n8_contiguous": Workload(
+        "bf16_b1_h32_kv4_s32768_d128_causal_n8_contiguous", "bf16", 1, 32, 32768, 128, True,
+        8, CONTIGUOUS, 8, 6, heads_kv=4),
 }
 
 
@@ -110,9 +120,10 @@ def make_inputs(w: Workload):
                    q=qkv[:, 0], k=qkv[:, 1], v=qkv[:, 2])
         return out
     shape = (w.batch, w.seqlen, w.heads, w.d_head)
+    kv_shape = (w.batch, w.seqlen, w.kv_heads, w.d_head)
     q = torch.randn(*shape, generator=g).to(w.torch_dtype)
-    k = torch.randn(*shape, generator=g).to(w.torch_dtype)
-    v = torch.randn(*shape, generator=g).to(w.torch_dtype)
+    k = torch.randn(*kv_shape, generator=g).to(w.torch_dtype)
+    v = torch.randn(*kv_shape, generator=g).to(w.torch_dtype)
     out.update(q=q, k=k, v=v)
     return out
 
@@ -129,8 +140,10 @@ def make_device_inputs(w: Workload, device="cuda", seed: Optional[int] = None):
         qkv = torch.randn(w.seqlen, 3, w.heads, w.d_head, generator=g, device=device,
                           dtype=torch.float32).to(w.torch_dtype)
         return dict(qkv=qkv, cu_seqlens=cu.to(device), lengths=lens)
-    shape = (w.batch, w.seqlen, w.heads, w.d_head)
-    return {n: torch.randn(*shape, generator=g, device=device,
+    shapes = {"q": (w.batch, w.seqlen, w.heads, w.d_head),
+              "k": (w.batch, w.seqlen, w.kv_heads, w.d_head),
+              "v": (w.batch, w.seqlen, w.kv_heads, w.d_head)}
+    return {n: torch.randn(*shapes[n], generator=g, device=device,
                            dtype=torch.float32).to(w.torch_dtype) for n in ("q", "k", "v")}
 
 

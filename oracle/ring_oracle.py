@@ -141,10 +141,24 @@ def masked_attention(q, k, v, mask, scale: float):
     return o, lse
 
 
+def kv_head(h, heads: int, heads_kv: int):
+    """Key/value head read by query head h.
+
+    Grouped-query and multi-query attention ("Tensorflow flash attention"
+    page: several query heads attend to one key/value head) -- the page does
+    not say which query heads share; the reading taken is consecutive groups
+    of heads / heads_kv query heads per key/value head (heads_kv == heads is
+    ordinary multi-head attention, heads_kv == 1 multi-query)."""
+    if heads_kv < 1 or heads % heads_kv != 0:
+        raise ValueError("heads must be a multiple of heads_kv")
+    return h // (heads // heads_kv)
+
+
 @dataclass
 class Problem:
-    """One forward call: tensors are float arrays [T, H, D] over all tokens
-    of all sequences (bf16 inputs are passed upcast, exactly)."""
+    """One forward call: q is a float array [T, H, D] over all tokens of all
+    sequences, k and v are [T, H_kv, D] with H a multiple of H_kv (bf16 inputs
+    are passed upcast, exactly)."""
     q: np.ndarray
     k: np.ndarray
     v: np.ndarray
@@ -179,8 +193,9 @@ def attention_rows(p: Problem, seq, head, row, chunk: int = 64):
             continue
         b, h = int(seq[grp[0]]), int(head[grp[0]])
         s0, L = int(p.seq_start[b]), int(p.seq_len[b])
-        K = p.k[s0:s0 + L, h, :].astype(np.float64)
-        V = p.v[s0:s0 + L, h, :].astype(np.float64)
+        hk = kv_head(h, p.q.shape[1], p.k.shape[1])
+        K = p.k[s0:s0 + L, hk, :].astype(np.float64)
+        V = p.v[s0:s0 + L, hk, :].astype(np.float64)
         tk = np.arange(L, dtype=np.int64)
         for c in range(0, grp.size, chunk):
             idx = grp[c:c + chunk]
@@ -295,5 +310,5 @@ __all__ = [
     "CONTIGUOUS", "STRIPED", "Problem", "allowed", "allowed_matrix",
     "attention_full", "attention_rows", "blas_threads", "masked_attention",
     "merge", "ring_block", "row_flops", "striped_block_sizes", "timed_rows",
-    "token_pos", "unmasked_pairs",
+    "kv_head", "token_pos", "unmasked_pairs",
 ]

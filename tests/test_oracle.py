@@ -195,6 +195,47 @@ def test_core_definition_vs_torch_sdpa(layout, causal, P):
         assert np.abs(lse[h] - ref_lse.numpy()).max() < TIGHT
 
 
+@pytest.mark.parametrize("H,Hkv", [(4, 2), (4, 1), (6, 3), (3, 3)])
+@pytest.mark.parametrize("layout,causal,P", [(0, True, 4), (1, True, 2), (0, False, 3)])
+def test_grouped_query_heads_vs_torch_sdpa(H, Hkv, layout, causal, P):
+    """Grouped-query / multi-query attention: query head h reads key/value
+    head h // (H / Hkv).  Pinned against torch's own grouped-query SDPA
+    (enable_gqa), fp64."""
+    L, N, D = 20, 4, 6
+    g = torch.Generator().manual_seed(17)
+    q = torch.randn(L, H, D, generator=g, dtype=torch.float64)
+    k = torch.randn(L, Hkv, D, generator=g, dtype=torch.float64)
+    v = torch.randn(L, Hkv, D, generator=g, dtype=torch.float64)
+    scale = 0.41
+    p = problem(q.numpy(), k.numpy(), v.numpy(), N, layout, causal, P, scale)
+    o, _ = oracle.attention_full(p)
+    mask = torch.from_numpy(explicit_mask(L, N, layout, causal, P))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.permute(1, 0, 2)[None], k.permute(1, 0, 2)[None], v.permute(1, 0, 2)[None],
+        attn_mask=mask[None, None], scale=scale, enable_gqa=True)[0].permute(1, 0, 2)
+    assert np.abs(o - ref.numpy()).max() < TIGHT
+
+
+def test_grouped_query_zero_queries_give_group_means():
+    # q = 0 with 2 key/value heads for 4 query heads: lse = ln|A(i)| and O is
+    # the mean of the allowed values of the shared head
+    rng = np.random.default_rng(9)
+    L, N, D, H, Hkv = 30, 5, 3, 4, 2
+    q = np.zeros((L, H, D))
+    k = rng.standard_normal((L, Hkv, D))
+    v = rng.standard_normal((L, Hkv, D))
+    p = problem(q, k, v, N, 1, True, 3, 0.5)
+    o, lse = oracle.attention_full(p)
+    mask = explicit_mask(L, N, 1, True, 3)
+    cnt = mask.sum(axis=1)
+    for h in range(H):
+        assert np.allclose(lse[h], np.log(cnt), atol=TIGHT, rtol=0)
+        mean = (mask.astype(np.float64) @ v[:, h // 2, :]) / cnt[:, None]
+        assert np.allclose(o[:, h, :], mean, atol=TIGHT, rtol=0)
+    with pytest.raises(ValueError):
+        oracle.kv_head(0, 4, 3)
+
+
 # ----------------------------------------------------------------------------
 # Brute force on tiny inputs (pure Python exp / normalise)
 # ----------------------------------------------------------------------------

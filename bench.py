@@ -39,6 +39,7 @@ EXTRAS = [
     "bf16_varlen_t65536_s16_h16_d128_causal_n4_packed",
     "bf16_b1_h8_s262144_d128_causal_striped_n16_p16",
     "bf16_b1_h8_s262144_d128_causal_striped_n16_p4",
+    "bf16_b1_h32_kv4_s32768_d128_causal_n8_contiguous",
     "fp32_b1_h1_s1024_d16_noncausal_n16",
 ]
 METRIC = "attention fwd TFLOP/s (unmasked FLOPs) and % of B200 bf16 tensor peak"
@@ -210,11 +211,16 @@ def make_step(w, dev, rank=0):
         out = torch.empty_like(q)
         lse = torch.empty(B, H, S, dtype=torch.float32, device=dev)
         lens = [S] * B
-        in_bytes = 3 * q.numel() * q.element_size()
+        in_bytes = (q.numel() + k.numel() + v.numel()) * q.element_size()
 
-        def step():
-            ra.ring_attn_fwd(q, k, v, out, lse, B, H, S, D, w.n_ring, w.layout, w.causal,
-                             w.softmax_scale, w.passes)
+        if w.kv_heads != H:
+            def step():
+                ra.ring_attn_gqa_fwd(q, k, v, out, lse, B, H, w.kv_heads, S, D, w.n_ring,
+                                     w.layout, w.causal, w.softmax_scale, w.passes)
+        else:
+            def step():
+                ra.ring_attn_fwd(q, k, v, out, lse, B, H, S, D, w.n_ring, w.layout, w.causal,
+                                 w.softmax_scale, w.passes)
     out_bytes = out.numel() * out.element_size() + lse.numel() * 4
     return step, lens, in_bytes, out_bytes, (inp, out, lse)
 

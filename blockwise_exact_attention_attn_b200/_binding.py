@@ -25,6 +25,7 @@ F32, BF16 = 0, 1
 
 EXPORTS = (
     "ring_attn_fwd",
+    "ring_attn_gqa_fwd",
     "ring_attn_qkvpacked_fwd",
     "ring_attn_fwd_simt",
     "ring_attn_fwd_noalloc",
@@ -51,6 +52,8 @@ _c_i64 = ctypes.c_int64
 
 _FWD_ARGS = [_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int, _c_int,
              _c_int, _c_int, _c_float, _c_int, _c_vp, _c_int, _c_vp]
+# ring_attn_gqa_fwd: heads_kv follows heads
+_GQA_ARGS = _FWD_ARGS[:7] + [_c_int] + _FWD_ARGS[7:]
 
 
 def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
@@ -66,6 +69,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib = ctypes.CDLL(path)
         lib.ring_attn_fwd.argtypes = _FWD_ARGS
         lib.ring_attn_fwd.restype = _c_int
+        lib.ring_attn_gqa_fwd.argtypes = _GQA_ARGS
+        lib.ring_attn_gqa_fwd.restype = _c_int
         lib.ring_attn_fwd_simt.argtypes = _FWD_ARGS
         lib.ring_attn_fwd_simt.restype = _c_int
         lib.ring_attn_fwd_noalloc.argtypes = _FWD_ARGS
@@ -157,6 +162,27 @@ def ring_attn_fwd(q, k, v, out, lse, batch: int, heads: int, seqlen: int, d_head
         _ptr(cu_seqlens, "cu_seqlens"), _dtype_code(q) if dtype is None else int(dtype),
         _stream(stream))
     _check("ring_attn_fwd", st)
+
+
+def ring_attn_gqa_fwd(q, k, v, out, lse, batch: int, heads: int, heads_kv: int, seqlen: int,
+                      d_head: int, n_ring_blocks: int, layout=CONTIGUOUS, causal: bool = False,
+                      softmax_scale: Optional[float] = None,
+                      max_ring_passes: Optional[int] = None, cu_seqlens=None,
+                      dtype: Optional[int] = None, stream=None) -> None:
+    """ring_attn_fwd with heads_kv key/value heads shared by consecutive
+    groups of heads / heads_kv query heads (see ring_attn.h)."""
+    lib = load_library()
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d_head)
+    if max_ring_passes is None:
+        max_ring_passes = n_ring_blocks
+    st = lib.ring_attn_gqa_fwd(
+        _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _ptr(out, "out"), _ptr(lse, "lse"),
+        int(batch), int(heads), int(heads_kv), int(seqlen), int(d_head), int(n_ring_blocks),
+        _layout_code(layout), int(bool(causal)), float(softmax_scale), int(max_ring_passes),
+        _ptr(cu_seqlens, "cu_seqlens"), _dtype_code(q) if dtype is None else int(dtype),
+        _stream(stream))
+    _check("ring_attn_gqa_fwd", st)
 
 
 def ring_attn_fwd_simt(q, k, v, out, lse, batch: int, heads: int, seqlen: int, d_head: int,
@@ -268,12 +294,18 @@ def _alloc_out(q_like, rows_shape, heads, d_head, lse_shape):
 def ring_attn_func(q, k, v, n_ring_blocks: int, causal: bool = False, layout=CONTIGUOUS,
                    softmax_scale: Optional[float] = None, max_ring_passes: Optional[int] = None,
                    stream=None):
-    """q, k, v: [batch, seqlen, heads, d_head] CUDA tensors -> (out, lse[batch, heads,
-    seqlen])."""
+    """q: [batch, seqlen, heads, d_head], k, v: [batch, seqlen, heads_kv, d_head]
+    CUDA tensors (heads_kv a divisor of heads; fewer key/value heads is
+    grouped-query attention) -> (out, lse[batch, heads, seqlen])."""
     B, S, H, D = q.shape
+    Hkv = k.shape[2]
     out, lse = _alloc_out(q, (B, S), H, D, (B, H, S))
-    ring_attn_fwd(q, k, v, out, lse, B, H, S, D, n_ring_blocks, layout, causal, softmax_scale,
-                  max_ring_passes, None, None, stream)
+    if Hkv == H:
+        ring_attn_fwd(q, k, v, out, lse, B, H, S, D, n_ring_blocks, layout, causal,
+                      softmax_scale, max_ring_passes, None, None, stream)
+    else:
+        ring_attn_gqa_fwd(q, k, v, out, lse, B, H, Hkv, S, D, n_ring_blocks, layout, causal,
+                          softmax_scale, max_ring_passes, None, None, stream)
     return out, lse
 
 

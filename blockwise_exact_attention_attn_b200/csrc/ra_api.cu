@@ -72,10 +72,11 @@ int* next_counter(int* status) {
 
 // Shared validation of the forward calls; fills everything but the tensor
 // pointers' derived fields.
-ra_status validate_fwd(int batch, int heads, int seqlen, int d_head, int n_ring, int layout,
-                       int causal, float scale, int passes, const int32_t* cu_seqlens,
-                       int dtype) {
+ra_status validate_fwd(int batch, int heads, int heads_kv, int seqlen, int d_head, int n_ring,
+                       int layout, int causal, float scale, int passes,
+                       const int32_t* cu_seqlens, int dtype) {
   if (batch < 1 || heads < 1 || seqlen < 1 || n_ring < 1) return RA_ERR_INVALID;
+  if (heads_kv < 1 || heads % heads_kv != 0) return RA_ERR_INVALID;
   if (layout != RA_LAYOUT_CONTIGUOUS && layout != RA_LAYOUT_STRIPED) return RA_ERR_INVALID;
   if (causal != 0 && causal != 1) return RA_ERR_INVALID;
   if (!std::isfinite(scale)) return RA_ERR_INVALID;
@@ -90,20 +91,26 @@ ra_status validate_fwd(int batch, int heads, int seqlen, int d_head, int n_ring,
   return RA_OK;
 }
 
-ra_status run_fwd(const void* q, const void* k, const void* v, int64_t tok_stride, void* out,
-                  float* lse, int batch, int heads, int seqlen, int d_head, int n_ring,
-                  int layout, int causal, float scale, int passes, const int32_t* cu_seqlens,
-                  int dtype, void* stream, bool force_simt) {
+// The parameters every forward kernel consumes.  q/out rows are tok_stride
+// elements apart, k/v rows kv_tok_stride; query head h reads key/value head
+// h / (heads / heads_kv).
+ra::FwdParams make_params(const void* q, const void* k, const void* v, int64_t tok_stride,
+                          int heads_kv, int64_t kv_tok_stride, void* out, float* lse,
+                          int batch, int heads, int seqlen, int d_head, int n_ring, int layout,
+                          int causal, float scale, int passes, const int32_t* cu_seqlens) {
   ra::FwdParams p;
   p.q = q;
   p.k = k;
   p.v = v;
   p.tok_stride = tok_stride;
+  p.kv_tok_stride = kv_tok_stride;
   p.out = out;
   p.lse = lse;
   p.cu_seqlens = cu_seqlens;
   p.batch = batch;
   p.heads = heads;
+  p.heads_kv = heads_kv;
+  p.kv_group = heads / heads_kv;
   p.seqlen = seqlen;
   p.d_head = d_head;
   p.n_ring = n_ring;
@@ -126,26 +133,47 @@ ra_status run_fwd(const void* q, const void* k, const void* v, int64_t tok_strid
     p.lse_seq_stride = (int64_t)heads * seqlen;
     p.lse_head_stride = seqlen;
   }
-  int* status = nullptr;
-  ra_status st = device_state(&status, nullptr);
-  if (st != RA_OK) return st;
-  p.status = status;
+  p.status = nullptr;
   p.work_counter = nullptr;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return p;
+}
+
+// bf16 with a nonzero scale runs on the tensor cores.  A zero scale (a plain
+// average over the allowed keys) has no log2-domain reference there; the
+// CUDA-core kernel handles it, and fp32.
+bool uses_tc(const ra::FwdParams& p, int dtype, bool force_simt) {
+  return dtype == RA_BF16 && !force_simt && p.scale != 0.f;
+}
+
+// Launch the kernel for p (status and, on the tensor-core path, a zeroed work
+// counter already in p).
+ra_status dispatch(const ra::FwdParams& p, int dtype, bool force_simt, cudaStream_t s) {
   cudaError_t e;
-  // scale 0 (a plain average over the allowed keys) has no log2-domain
-  // reference on the tensor-core path; the CUDA-core kernel handles it
-  if (dtype == RA_BF16 && !force_simt && scale != 0.f) {
-    if (d_head != 64 && d_head != 128) return RA_ERR_UNSUPPORTED;
-    if (((tok_stride * 2) & 15) != 0) return RA_ERR_INVALID;
-    p.work_counter = next_counter(status);
-    if (cudaMemsetAsync(p.work_counter, 0, sizeof(int), s) != cudaSuccess) return RA_ERR_CUDA;
+  if (uses_tc(p, dtype, force_simt)) {
+    if (p.d_head != 64 && p.d_head != 128) return RA_ERR_UNSUPPORTED;
+    // TMA row strides are multiples of 16 bytes
+    if (((p.tok_stride * 2) & 15) != 0 || ((p.kv_tok_stride * 2) & 15) != 0)
+      return RA_ERR_INVALID;
     e = ra::launch_fwd_tc(p, s);
   } else {
     e = ra::launch_fwd_simt(p, dtype == RA_F32 ? 0 : 1, s);
   }
   if (e == cudaErrorInvalidValue) return RA_ERR_UNSUPPORTED;
   return e == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+ra_status run_fwd(const ra::FwdParams& params, int dtype, void* stream, bool force_simt) {
+  ra::FwdParams p = params;
+  int* status = nullptr;
+  ra_status st = device_state(&status, nullptr);
+  if (st != RA_OK) return st;
+  p.status = status;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (uses_tc(p, dtype, force_simt)) {
+    p.work_counter = next_counter(status);
+    if (cudaMemsetAsync(p.work_counter, 0, sizeof(int), s) != cudaSuccess) return RA_ERR_CUDA;
+  }
+  return dispatch(p, dtype, force_simt, s);
 }
 
 }  // namespace
@@ -159,11 +187,31 @@ ra_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out, 
   if (!q || !k || !v || !out || !lse) return RA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
     return RA_ERR_INVALID;
-  ra_status st = validate_fwd(batch, heads, seqlen, d_head, n_ring_blocks, layout, causal,
-                              softmax_scale, max_ring_passes, cu_seqlens, dtype);
+  ra_status st = validate_fwd(batch, heads, heads, seqlen, d_head, n_ring_blocks, layout,
+                              causal, softmax_scale, max_ring_passes, cu_seqlens, dtype);
   if (st != RA_OK) return st;
-  return run_fwd(q, k, v, (int64_t)heads * d_head, out, lse, batch, heads, seqlen, d_head,
-                 n_ring_blocks, layout, causal, softmax_scale, max_ring_passes, cu_seqlens,
+  const int64_t hd = (int64_t)heads * d_head;
+  return run_fwd(make_params(q, k, v, hd, heads, hd, out, lse, batch, heads, seqlen, d_head,
+                             n_ring_blocks, layout, causal, softmax_scale, max_ring_passes,
+                             cu_seqlens),
+                 dtype, stream, false);
+}
+
+ra_status ring_attn_gqa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                            int batch, int heads, int heads_kv, int seqlen, int d_head,
+                            int n_ring_blocks, int layout, int causal, float softmax_scale,
+                            int max_ring_passes, const int32_t* cu_seqlens, int dtype,
+                            void* stream) {
+  if (!q || !k || !v || !out || !lse) return RA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return RA_ERR_INVALID;
+  ra_status st = validate_fwd(batch, heads, heads_kv, seqlen, d_head, n_ring_blocks, layout,
+                              causal, softmax_scale, max_ring_passes, cu_seqlens, dtype);
+  if (st != RA_OK) return st;
+  return run_fwd(make_params(q, k, v, (int64_t)heads * d_head, heads_kv,
+                             (int64_t)heads_kv * d_head, out, lse, batch, heads, seqlen, d_head,
+                             n_ring_blocks, layout, causal, softmax_scale, max_ring_passes,
+                             cu_seqlens),
                  dtype, stream, false);
 }
 
@@ -175,11 +223,13 @@ ra_status ring_attn_fwd_simt(const void* q, const void* k, const void* v, void* 
   if (!q || !k || !v || !out || !lse) return RA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
     return RA_ERR_INVALID;
-  ra_status st = validate_fwd(batch, heads, seqlen, d_head, n_ring_blocks, layout, causal,
-                              softmax_scale, max_ring_passes, cu_seqlens, dtype);
+  ra_status st = validate_fwd(batch, heads, heads, seqlen, d_head, n_ring_blocks, layout,
+                              causal, softmax_scale, max_ring_passes, cu_seqlens, dtype);
   if (st != RA_OK) return st;
-  return run_fwd(q, k, v, (int64_t)heads * d_head, out, lse, batch, heads, seqlen, d_head,
-                 n_ring_blocks, layout, causal, softmax_scale, max_ring_passes, cu_seqlens,
+  const int64_t hd = (int64_t)heads * d_head;
+  return run_fwd(make_params(q, k, v, hd, heads, hd, out, lse, batch, heads, seqlen, d_head,
+                             n_ring_blocks, layout, causal, softmax_scale, max_ring_passes,
+                             cu_seqlens),
                  dtype, stream, true);
 }
 
@@ -189,15 +239,16 @@ ra_status ring_attn_qkvpacked_fwd(const void* qkv, void* out, float* lse, int ba
                                   const int32_t* cu_seqlens, int dtype, void* stream) {
   if (!qkv || !out || !lse) return RA_ERR_INVALID;
   if (!aligned16(qkv) || !aligned16(out) || !aligned16(lse)) return RA_ERR_INVALID;
-  ra_status st = validate_fwd(batch, heads, seqlen, d_head, n_ring_blocks, layout, causal,
-                              softmax_scale, max_ring_passes, cu_seqlens, dtype);
+  ra_status st = validate_fwd(batch, heads, heads, seqlen, d_head, n_ring_blocks, layout,
+                              causal, softmax_scale, max_ring_passes, cu_seqlens, dtype);
   if (st != RA_OK) return st;
   const int esize = dtype == RA_F32 ? 4 : 2;
   const int64_t hd = (int64_t)heads * d_head;
   const char* base = static_cast<const char*>(qkv);
-  return run_fwd(base, base + hd * esize, base + 2 * hd * esize, 3 * hd, out, lse, batch,
-                 heads, seqlen, d_head, n_ring_blocks, layout, causal, softmax_scale,
-                 max_ring_passes, cu_seqlens, dtype, stream, false);
+  return run_fwd(make_params(base, base + hd * esize, base + 2 * hd * esize, 3 * hd, heads,
+                             3 * hd, out, lse, batch, heads, seqlen, d_head, n_ring_blocks,
+                             layout, causal, softmax_scale, max_ring_passes, cu_seqlens),
+                 dtype, stream, false);
 }
 
 ra_status ring_attn_merge(void* out_a, float* lse_a, const void* out_b, const float* lse_b,
@@ -328,8 +379,8 @@ extern "C" ra_status ring_attn_fwd_noalloc(const void* q, const void* k, const v
   if (!q || !k || !v || !out || !lse) return RA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
     return RA_ERR_INVALID;
-  ra_status st = validate_fwd(batch, heads, seqlen, d_head, n_ring_blocks, layout, causal,
-                              softmax_scale, max_ring_passes, cu_seqlens, dtype);
+  ra_status st = validate_fwd(batch, heads, heads, seqlen, d_head, n_ring_blocks, layout,
+                              causal, softmax_scale, max_ring_passes, cu_seqlens, dtype);
   if (st != RA_OK) return st;
   // Scratch this call needs: the status word and one work counter.  Both
   // sit at fixed offsets, so no problem size can outgrow the array; the check
@@ -342,36 +393,10 @@ extern "C" ra_status ring_attn_fwd_noalloc(const void* q, const void* k, const v
   st = noalloc_scratch(&scratch);
   if (st != RA_OK) return st;
 
-  ra::FwdParams p;
-  p.q = q;
-  p.k = k;
-  p.v = v;
-  p.tok_stride = (int64_t)heads * d_head;
-  p.out = out;
-  p.lse = lse;
-  p.cu_seqlens = cu_seqlens;
-  p.batch = batch;
-  p.heads = heads;
-  p.seqlen = seqlen;
-  p.d_head = d_head;
-  p.n_ring = n_ring_blocks;
-  p.layout = layout;
-  p.causal = causal;
-  p.passes = max_ring_passes < n_ring_blocks ? max_ring_passes : n_ring_blocks;
-  p.scale = softmax_scale;
-  p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634074);
-  p.n_qranges = 0;
-  p.order = (causal && layout == RA_LAYOUT_CONTIGUOUS) ? 1 : 0;
-  p.qr_per_block = 0;
-  if (cu_seqlens) {
-    p.total_rows = seqlen;
-    p.lse_seq_stride = 0;
-    p.lse_head_stride = seqlen;
-  } else {
-    p.total_rows = batch * seqlen;
-    p.lse_seq_stride = (int64_t)heads * seqlen;
-    p.lse_head_stride = seqlen;
-  }
+  const int64_t hd = (int64_t)heads * d_head;
+  ra::FwdParams p = make_params(q, k, v, hd, heads, hd, out, lse, batch, heads, seqlen, d_head,
+                                n_ring_blocks, layout, causal, softmax_scale, max_ring_passes,
+                                cu_seqlens);
   p.status = scratch + kNoAllocStatus;
   p.work_counter = scratch + kNoAllocCounter;
 
@@ -380,13 +405,5 @@ extern "C" ra_status ring_attn_fwd_noalloc(const void* q, const void* k, const v
   if (cudaMemsetAsync(scratch + kNoAllocStatus, 0, sizeof(int), s) != cudaSuccess ||
       cudaMemsetAsync(scratch + kNoAllocCounter, 0, sizeof(int), s) != cudaSuccess)
     return RA_ERR_CUDA;
-  cudaError_t e;
-  if (dtype == RA_BF16 && softmax_scale != 0.f) {
-    if (d_head != 64 && d_head != 128) return RA_ERR_UNSUPPORTED;
-    e = ra::launch_fwd_tc(p, s);
-  } else {
-    e = ra::launch_fwd_simt(p, dtype == RA_F32 ? 0 : 1, s);
-  }
-  if (e == cudaErrorInvalidValue) return RA_ERR_UNSUPPORTED;
-  return e == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+  return dispatch(p, dtype, false, s);
 }

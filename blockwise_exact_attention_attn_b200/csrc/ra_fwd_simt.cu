@@ -92,6 +92,7 @@ __global__ void __launch_bounds__(kSimtThreads)
     tq = token_of(g, sq, rq);
   }
 
+  const int hk = it.h / p.kv_group;  // key/value head read by this query head
   const T* qg = static_cast<const T*>(p.q);
   const T* kg = static_cast<const T*>(p.k);
   const T* vg = static_cast<const T*>(p.v);
@@ -119,7 +120,7 @@ __global__ void __launch_bounds__(kSimtThreads)
       float kv = 0.f, vv = 0.f;
       if (c < nk) {
         const int64_t off =
-            (int64_t)(base + k0 + c) * p.tok_stride + (int64_t)it.h * D + d;
+            (int64_t)(base + k0 + c) * p.kv_tok_stride + (int64_t)hk * D + d;
         kv = to_f32(kg[off]);
         vv = to_f32(vg[off]);
       }

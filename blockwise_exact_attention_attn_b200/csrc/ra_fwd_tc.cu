@@ -461,7 +461,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // item's last S MMAs (q_free)
         int e = -1;
         if (ok) ok = rd.next(&e, abort_flag);
-        if (ok && e >= 0) ok = load(&maps.k, it.h, it.base + entry_tile(e) * kTcBN);
+        const int hk = it.h / p.kv_group;  // key/value head of this query head
+        if (ok && e >= 0) ok = load(&maps.k, hk, it.base + entry_tile(e) * kTcBN);
         if (ok && k > 0) ok = mbar_wait(&ctrl->q_free, (k - 1) & 1, abort_flag);
         if (ok) {
           uint8_t* qs = smem + C::kQOff;
@@ -476,8 +477,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         while (ok && prev >= 0) {
           ok = rd.next(&e, abort_flag);
           if (!ok) break;
-          if (e >= 0) ok = load(&maps.k, it.h, it.base + entry_tile(e) * kTcBN);
-          if (ok) ok = load(&maps.v, it.h, it.base + entry_tile(prev) * kTcBN);
+          if (e >= 0) ok = load(&maps.k, hk, it.base + entry_tile(e) * kTcBN);
+          if (ok) ok = load(&maps.v, hk, it.base + entry_tile(prev) * kTcBN);
           prev = e;
         }
       }
@@ -867,8 +868,8 @@ static cudaError_t launch_tc_t(const FwdParams& p, cudaStream_t stream) {
   const int claim_limit = per_item ? 1 : 0;
   TcMaps maps;
   if (!make_map(&maps.q, p.q, p.total_rows, p.heads, D, p.tok_stride) ||
-      !make_map(&maps.k, p.k, p.total_rows, p.heads, D, p.tok_stride) ||
-      !make_map(&maps.v, p.v, p.total_rows, p.heads, D, p.tok_stride))
+      !make_map(&maps.k, p.k, p.total_rows, p.heads_kv, D, p.kv_tok_stride) ||
+      !make_map(&maps.v, p.v, p.total_rows, p.heads_kv, D, p.kv_tok_stride))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -11,15 +11,18 @@ namespace ra {
 // cu_seqlens[b] (varlen).
 struct FwdParams {
   const void* q;            // element (row, h, d) at q + row*tok_stride + h*d_head + d
-  const void* k;
-  const void* v;
-  int64_t tok_stride;       // elements between consecutive rows of q/k/v
+  const void* k;            // element (row, hk, d) at k + row*kv_tok_stride + hk*d_head + d
+  const void* v;            // (same layout as k)
+  int64_t tok_stride;       // elements between consecutive rows of q
+  int64_t kv_tok_stride;    // elements between consecutive rows of k/v
   void* out;                // [rows, heads, d_head], same dtype as q
   float* lse;               // see lse_seq_stride / lse_head_stride
   int64_t lse_seq_stride;   // dense: heads*seqlen; varlen: 0
   int64_t lse_head_stride;  // dense: seqlen;       varlen: total rows
   const int32_t* cu_seqlens;  // NULL for dense
   int batch, heads, seqlen, d_head;
+  int heads_kv;             // key/value heads; query head h reads hk = h / kv_group
+  int kv_group;             // heads / heads_kv
   int n_ring, layout, causal, passes;
   int total_rows;           // rows of q/k/v/out (dense: batch*seqlen)
   int n_qranges;            // query ranges per sequence (ceil(seqlen / rows per CTA))

@@ -124,6 +124,32 @@ ra_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out,
                         const int32_t* cu_seqlens, int dtype, void* stream);
 
 /*
+ * ring_attn_gqa_fwd -- ring_attn_fwd with fewer key/value heads than query
+ * heads (grouped-query attention; heads_kv = 1 is multi-query attention).
+ *
+ * Source: "Tensorflow flash attention" page: multi-query and grouped-query
+ * attention, in which several query heads attend to one key/value head.  The
+ * page does not say which heads share; here query head h reads key/value
+ * head h / (heads / heads_kv), i.e. consecutive groups of query heads share.
+ *
+ *  q, out    dense: [batch, seqlen, heads, d_head]; varlen: [seqlen, heads,
+ *            d_head].
+ *  k, v      dense: [batch, seqlen, heads_kv, d_head]; varlen: [seqlen,
+ *            heads_kv, d_head].
+ *  heads_kv  >= 1 and a divisor of heads; heads_kv == heads is ring_attn_fwd.
+ *  lse       as ring_attn_fwd (one row per query head).
+ * All other arguments as ring_attn_fwd.  Errors as ring_attn_fwd, plus
+ * RA_ERR_INVALID when heads_kv < 1 or heads % heads_kv != 0.
+ */
+ra_status ring_attn_gqa_fwd(const void* q, const void* k, const void* v,
+                            void* out, float* lse, int batch, int heads,
+                            int heads_kv, int seqlen, int d_head,
+                            int n_ring_blocks, int layout, int causal,
+                            float softmax_scale, int max_ring_passes,
+                            const int32_t* cu_seqlens, int dtype,
+                            void* stream);
+
+/*
  * ring_attn_qkvpacked_fwd -- same computation, q/k/v packed in one tensor.
  *
  * Source: issue thread "A ring attention with flash attention kernel

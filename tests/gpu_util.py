@@ -36,7 +36,13 @@ def run_gpu(w, inp, impl="tc", stream=None):
     B, S, H, D = q.shape
     out = torch.empty_like(q)
     lse = torch.empty(B, H, S, dtype=torch.float32, device=dev)
-    fn(q, k, v, out, lse, B, H, S, D, w.n_ring, w.layout, w.causal, w.softmax_scale, w.passes)
+    if w.kv_heads != w.heads:
+        # one entry point for both kernels: fp32 runs on the CUDA cores
+        ra.ring_attn_gqa_fwd(q, k, v, out, lse, B, H, w.kv_heads, S, D, w.n_ring, w.layout,
+                             w.causal, w.softmax_scale, w.passes)
+    else:
+        fn(q, k, v, out, lse, B, H, S, D, w.n_ring, w.layout, w.causal, w.softmax_scale,
+           w.passes)
     torch.cuda.synchronize()
     assert ra.ring_attn_status() == ra.RA_OK
     # to token-major [T, H, D] / [H, T]
@@ -49,9 +55,12 @@ def problem_for(w, inp, heads=None):
     if w.varlen:
         q, k, v = inp["q"], inp["k"], inp["v"]
     else:
-        q, k, v = (inp[n].reshape(-1, w.heads, w.d_head) for n in ("q", "k", "v"))
+        q = inp["q"].reshape(-1, w.heads, w.d_head)
+        k, v = (inp[n].reshape(-1, w.kv_heads, w.d_head) for n in ("k", "v"))
     if heads is not None:
-        q, k, v = q[:, heads], k[:, heads], v[:, heads]
+        # the listed query heads with the key/value head each of them reads
+        kvh = [oracle.kv_head(h, w.heads, w.kv_heads) for h in heads]
+        q, k, v = q[:, heads], k[:, kvh], v[:, kvh]
     starts, lens = gen.seq_offsets(w, inp)
     return oracle.Problem(q=q.float().numpy(), k=k.float().numpy(), v=v.float().numpy(),
                           seq_start=np.array(starts), seq_len=np.array(lens), n_ring=w.n_ring,

@@ -71,6 +71,21 @@ def test_qkvpacked_and_simt_reject_invalid_arguments(lib):
     assert st == ra.RA_ERR_INVALID
 
 
+@pytest.mark.parametrize("heads,heads_kv", [(4, 3), (4, 0), (4, -2), (2, 4)])
+def test_gqa_rejects_heads_that_do_not_group(lib, heads, heads_kv):
+    st = lib.ring_attn_gqa_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1, heads, heads_kv, 256, 128, 4, 0,
+                               1, 0.1, 4, None, 1, None)
+    assert st == ra.RA_ERR_INVALID
+
+
+def test_gqa_shares_the_forward_validation(lib):
+    # the same checks as ring_attn_fwd run first (null pointer, bad seqlen)
+    assert lib.ring_attn_gqa_fwd(None, FAKE, FAKE, FAKE, FAKE, 1, 4, 2, 256, 128, 4, 0, 1, 0.1,
+                                 4, None, 1, None) == ra.RA_ERR_INVALID
+    assert lib.ring_attn_gqa_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, 2, 250, 128, 4, 0, 1, 0.1,
+                                 4, None, 1, None) == ra.RA_ERR_INVALID
+
+
 @pytest.mark.parametrize("args", [
     (None, FAKE, FAKE, FAKE, 1, 1, 8, 128, 0),         # null
     (FAKE, FAKE + 4, FAKE, FAKE, 1, 1, 8, 128, 0),     # misaligned lse

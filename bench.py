@@ -40,6 +40,7 @@ EXTRAS = [
     "bf16_b1_h8_s262144_d128_causal_striped_n16_p16",
     "bf16_b1_h8_s262144_d128_causal_striped_n16_p4",
     "bf16_b1_h32_kv4_s32768_d128_causal_n8_contiguous",
+    "f16_b2_h16_s8192_d128_noncausal_n8",
     "fp32_b1_h1_s1024_d16_noncausal_n16",
 ]
 METRIC = "attention fwd TFLOP/s (unmasked FLOPs) and % of B200 bf16 tensor peak"
@@ -279,11 +280,12 @@ def measure_workload(name, steps, warmup, dist, dev, peaks):
     tflops = flops / (per * 1e-3) / 1e12
     res = {"workload": name, "ms_per_step": per, "tflops_per_gpu": tflops,
            "tflops": tflops * dist.world, "flops_per_step": flops,
-           "frac_of_measured_bf16_peak": tflops / peaks["bf16_tflops"] if w.dtype == "bf16"
+           # fp16 and bf16 have the same dense tensor peak (nominal ratio 1)
+           "frac_of_measured_bf16_peak": tflops / peaks["bf16_tflops"] if w.dtype != "f32"
            else None,
-           "frac_of_datasheet_bf16_peak": tflops / DATASHEET_BF16_TFLOPS if w.dtype == "bf16"
+           "frac_of_datasheet_bf16_peak": tflops / DATASHEET_BF16_TFLOPS if w.dtype != "f32"
            else None,
-           "kernel": "fwd_tc (tcgen05)" if w.dtype == "bf16" else "fwd_simt (fp32)"}
+           "kernel": "fwd_tc (tcgen05)" if w.dtype != "f32" else "fwd_simt (fp32)"}
     return res, w, in_bytes, out_bytes, flops
 
 

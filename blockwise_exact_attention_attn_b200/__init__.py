@@ -8,6 +8,7 @@ from ._binding import (  # noqa: F401
     BF16,
     CONTIGUOUS,
     EXPORTS,
+    F16,
     F32,
     RA_ERR_CUDA,
     RA_ERR_INVALID,

@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(HERE, "libringattn.so")
 
 RA_OK, RA_ERR_INVALID, RA_ERR_UNSUPPORTED, RA_ERR_CUDA, RA_ERR_TIMEOUT = range(5)
 CONTIGUOUS, STRIPED = 0, 1
-F32, BF16 = 0, 1
+F32, BF16, F16 = 0, 1, 2
 
 EXPORTS = (
     "ring_attn_fwd",
@@ -129,6 +129,8 @@ def _dtype_code(t) -> int:
         return F32
     if t.dtype == torch.bfloat16:
         return BF16
+    if t.dtype == torch.float16:
+        return F16
     raise ValueError(f"unsupported dtype {t.dtype}")
 
 

@@ -12,7 +12,7 @@
 #include "ring_attn.h"
 
 namespace ra {
-cudaError_t launch_fwd_tc(const FwdParams& p, cudaStream_t stream);
+cudaError_t launch_fwd_tc(const FwdParams& p, int fmt, cudaStream_t stream);
 cudaError_t launch_fwd_simt(const FwdParams& p, int dtype, cudaStream_t stream);
 cudaError_t launch_merge(void* out_a, float* lse_a, const void* out_b, const float* lse_b,
                          int batch, int heads, int seqlen, int d_head, int dtype, int num_sms,
@@ -81,7 +81,7 @@ ra_status validate_fwd(int batch, int heads, int heads_kv, int seqlen, int d_hea
   if (causal != 0 && causal != 1) return RA_ERR_INVALID;
   if (!std::isfinite(scale)) return RA_ERR_INVALID;
   if (passes < 1) return RA_ERR_INVALID;
-  if (dtype != RA_F32 && dtype != RA_BF16) return RA_ERR_INVALID;
+  if (dtype != RA_F32 && dtype != RA_BF16 && dtype != RA_F16) return RA_ERR_INVALID;
   if (d_head != 16 && d_head != 32 && d_head != 64 && d_head != 128) return RA_ERR_INVALID;
   if (!cu_seqlens && seqlen % n_ring != 0) return RA_ERR_INVALID;
   if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return RA_ERR_INVALID;
@@ -138,11 +138,11 @@ ra::FwdParams make_params(const void* q, const void* k, const void* v, int64_t t
   return p;
 }
 
-// bf16 with a nonzero scale runs on the tensor cores.  A zero scale (a plain
-// average over the allowed keys) has no log2-domain reference there; the
-// CUDA-core kernel handles it, and fp32.
+// bf16 and fp16 with a nonzero scale run on the tensor cores.  A zero scale
+// (a plain average over the allowed keys) has no log2-domain reference there;
+// the CUDA-core kernel handles it, and fp32.
 bool uses_tc(const ra::FwdParams& p, int dtype, bool force_simt) {
-  return dtype == RA_BF16 && !force_simt && p.scale != 0.f;
+  return (dtype == RA_BF16 || dtype == RA_F16) && !force_simt && p.scale != 0.f;
 }
 
 // Launch the kernel for p (status and, on the tensor-core path, a zeroed work
@@ -154,9 +154,9 @@ ra_status dispatch(const ra::FwdParams& p, int dtype, bool force_simt, cudaStrea
     // TMA row strides are multiples of 16 bytes
     if (((p.tok_stride * 2) & 15) != 0 || ((p.kv_tok_stride * 2) & 15) != 0)
       return RA_ERR_INVALID;
-    e = ra::launch_fwd_tc(p, s);
+    e = ra::launch_fwd_tc(p, dtype == RA_BF16 ? ra::kFmtBF16 : ra::kFmtF16, s);
   } else {
-    e = ra::launch_fwd_simt(p, dtype == RA_F32 ? 0 : 1, s);
+    e = ra::launch_fwd_simt(p, dtype == RA_F32 ? 0 : (dtype == RA_BF16 ? 1 : 2), s);
   }
   if (e == cudaErrorInvalidValue) return RA_ERR_UNSUPPORTED;
   return e == cudaSuccess ? RA_OK : RA_ERR_CUDA;
@@ -258,7 +258,7 @@ ra_status ring_attn_merge(void* out_a, float* lse_a, const void* out_b, const fl
   if (!aligned16(out_a) || !aligned16(out_b) || !aligned16(lse_a) || !aligned16(lse_b))
     return RA_ERR_INVALID;
   if (batch < 1 || heads < 1 || seqlen < 1 || d_head < 1) return RA_ERR_INVALID;
-  if (dtype != RA_F32 && dtype != RA_BF16) return RA_ERR_INVALID;
+  if (dtype != RA_F32 && dtype != RA_BF16 && dtype != RA_F16) return RA_ERR_INVALID;
   const int esize = dtype == RA_F32 ? 4 : 2;
   if ((d_head * esize) % 16 != 0) return RA_ERR_INVALID;
   const int chunks = d_head * esize / 16;
@@ -269,7 +269,7 @@ ra_status ring_attn_merge(void* out_a, float* lse_a, const void* out_b, const fl
   ra_status st = device_state(&status, &sms);
   if (st != RA_OK) return st;
   cudaError_t e = ra::launch_merge(out_a, lse_a, out_b, lse_b, batch, heads, seqlen, d_head,
-                                   dtype == RA_F32 ? 0 : 1, sms,
+                                   dtype == RA_F32 ? 0 : (dtype == RA_BF16 ? 1 : 2), sms,
                                    reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }

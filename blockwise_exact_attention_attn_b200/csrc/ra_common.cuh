@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "ra_params.h"
+
 namespace ra {
 
 // Device status word values (mirror ra_status in include/ring_attn.h).
@@ -183,13 +185,16 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
-// Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulator:
-//   [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format,
-//   [13] negate A, [15] A major (0 = K), [16] B major (0 = K, 1 = MN),
+// Instruction descriptor for kind::f16 with fp16 or bf16 A/B (fmt) and fp32
+// accumulator:
+//   [4,6) D format (1 = f32), [7,10) A format (0 = f16, 1 = bf16), [10,13) B
+//   format, [13] negate A, [15] A major (0 = K), [16] B major (0 = K, 1 = MN),
 //   [17,23) N >> 3, [24,29) M >> 4.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn_major << 16) |
-         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+__host__ __device__ constexpr uint32_t idesc_f16kind_f32(int M, int N, int b_mn_major,
+                                                         int fmt) {
+  return (1u << 4) | ((uint32_t)fmt << 7) | ((uint32_t)fmt << 10) |
+         ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
 }
 
 // 32 lanes x 32 bit x 32 columns: thread t of the warp gets lane (base + t),
@@ -311,6 +316,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two floats rounded to the 16-bit element format fmt, low half first.
+template <int kFmt>
+__device__ __forceinline__ uint32_t pack_x2(float lo, float hi) {
+  return kFmt == kFmtBF16 ? pack_bf16x2(lo, hi) : pack_f16x2(lo, hi);
 }
 
 }  // namespace ra

@@ -16,6 +16,7 @@
 // d_head / min(d_head, 32) of them (dot products completed with warp
 // shuffles) and its keys over the rest (key lanes merged at the end).
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "ra_common.cuh"
@@ -36,6 +37,10 @@ template <>
 __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
   return __bfloat162float(x);
 }
+template <>
+__device__ __forceinline__ float to_f32<__half>(__half x) {
+  return __half2float(x);
+}
 
 template <typename T>
 __device__ __forceinline__ T from_f32(float x);
@@ -44,6 +49,10 @@ __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
+}
+template <>
+__device__ __forceinline__ __half from_f32<__half>(float x) {
+  return __float2half_rn(x);
 }
 
 // Thread layout: 8 threads serve one query row, 16 rows per CTA.  The row's
@@ -211,23 +220,24 @@ static cudaError_t launch_simt_t(const FwdParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-// dtype: 0 = fp32, 1 = bf16.  Returns cudaErrorInvalidValue for an
-// unsupported head dimension.
+template <typename T>
+static cudaError_t launch_simt_d(const FwdParams& p, cudaStream_t stream) {
+  switch (p.d_head) {
+    case 16: return launch_simt_t<T, 16>(p, stream);
+    case 32: return launch_simt_t<T, 32>(p, stream);
+    case 64: return launch_simt_t<T, 64>(p, stream);
+    case 128: return launch_simt_t<T, 128>(p, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+// dtype: 0 = fp32, 1 = bf16, 2 = fp16.  Returns cudaErrorInvalidValue for an
+// unsupported head dimension or dtype.
 cudaError_t launch_fwd_simt(const FwdParams& p, int dtype, cudaStream_t stream) {
-  if (dtype == 0) {
-    switch (p.d_head) {
-      case 16: return launch_simt_t<float, 16>(p, stream);
-      case 32: return launch_simt_t<float, 32>(p, stream);
-      case 64: return launch_simt_t<float, 64>(p, stream);
-      case 128: return launch_simt_t<float, 128>(p, stream);
-    }
-  } else {
-    switch (p.d_head) {
-      case 16: return launch_simt_t<__nv_bfloat16, 16>(p, stream);
-      case 32: return launch_simt_t<__nv_bfloat16, 32>(p, stream);
-      case 64: return launch_simt_t<__nv_bfloat16, 64>(p, stream);
-      case 128: return launch_simt_t<__nv_bfloat16, 128>(p, stream);
-    }
+  switch (dtype) {
+    case 0: return launch_simt_d<float>(p, stream);
+    case 1: return launch_simt_d<__nv_bfloat16>(p, stream);
+    case 2: return launch_simt_d<__half>(p, stream);
   }
   return cudaErrorInvalidValue;
 }

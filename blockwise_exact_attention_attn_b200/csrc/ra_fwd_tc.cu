@@ -1,5 +1,5 @@
 // ra_fwd_tc.cu -- ring-ordered blockwise attention forward on the sm_100a
-// tensor cores (tcgen05 + TMEM), bf16 inputs, fp32 accumulation.
+// tensor cores (tcgen05 + TMEM), bf16 or fp16 inputs, fp32 accumulation.
 //
 // The method: the sequence is split into N ring blocks; a query block keeps
 // its queries in place and meets the key/value blocks in ring order, folding
@@ -35,7 +35,7 @@
 // The control warpgroup (warps 8-11) hands registers to the softmax
 // warpgroups with setmaxnreg.
 // Tensor memory (512 columns): S_0 | S_1 | O_0 | O_1.  Shared memory: Q_0,
-// Q_1, the K/V ring, P_0, P_1 (bf16, 128-byte swizzle), the list.
+// Q_1, the K/V ring, P_0, P_1 (input format, 128-byte swizzle), the list.
 //
 // Per kv tile t issuer i issues S_i(t+1) as soon as softmax i has loaded
 // S_i(t) into registers (s_free), then PV_i(t) once P_i(t) is in shared
@@ -300,7 +300,7 @@ __device__ __forceinline__ bool read_item(ListReader& rd, SeqWork* it, volatile 
   return true;
 }
 
-template <int D>
+template <int D, int kFmt>
 __global__ void __launch_bounds__(kTcThreads, 1)
     fwd_tc_kernel(const FwdParams p, const __grid_constant__ TcMaps maps, int n_items,
                   int claim_limit) {
@@ -504,8 +504,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int i1 = kTcIssuers == 2 ? i0 + 1 : kTcQT;
     // a negative softmax scale is applied as S = (-Q) K^T times |scale|
     const uint32_t idesc_s =
-        idesc_bf16_f32(kTcBM, kTcBN, 0) | (p.scale_log2 < 0.f ? (1u << 13) : 0u);
-    constexpr uint32_t idesc_o = idesc_bf16_f32(kTcBM, D, 1);
+        idesc_f16kind_f32(kTcBM, kTcBN, 0, kFmt) | (p.scale_log2 < 0.f ? (1u << 13) : 0u);
+    constexpr uint32_t idesc_o = idesc_f16kind_f32(kTcBM, D, 1, kFmt);
     // base descriptors: K-major tiles (Q, K, P) and MN-major tiles (V)
     const uint64_t qdesc0 = smem_desc_sw128(smem_u32(smem + C::kQOff), 16, 1024);
     const uint64_t pdesc0 = smem_desc_sw128(smem_u32(smem + C::kPOff), 16, 1024);
@@ -707,7 +707,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           m_ref = m_tile;
         }
         const float msub = m_ref == -INFINITY ? 0.f : m_ref;
-        // P row in registers (bf16 pairs) while the previous PV still runs;
+        // P row in registers (16-bit pairs) while the previous PV still runs;
         // scale-and-subtract and the row sums in paired fp32 instructions
         const uint64_t sc2 = f32x2_pack(sl2, sl2), ms2 = f32x2_pack(-msub, -msub);
         uint64_t sum2[2] = {0ull, 0ull};  // two independent (even, odd) partial sums
@@ -719,7 +719,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const float a = ex2_approx(ya);
           const float b = ex2_approx(yb);
           sum2[j & 1] = fadd2(sum2[j & 1], a, b);
-          pk[j] = pack_bf16x2(a, b);
+          pk[j] = pack_x2<kFmt>(a, b);
         }
         // the previous PV of this query tile has finished reading P and
         // writing O
@@ -763,7 +763,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_after();
       if (!first) {
         const float inv_l = valid ? 1.f / l : 0.f;
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) +
+        uint16_t* orow = static_cast<uint16_t*>(p.out) +
                               ((int64_t)(it.base + sq) * p.heads + it.h) * D;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
@@ -773,7 +773,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            pk[j] = pack_bf16x2(__uint_as_float(o[2 * j]) * inv_l,
+            pk[j] = pack_x2<kFmt>(__uint_as_float(o[2 * j]) * inv_l,
                                 __uint_as_float(o[2 * j + 1]) * inv_l);
           if (valid) {
             uint4* dst = reinterpret_cast<uint4*>(orow + c);
@@ -828,23 +828,26 @@ static EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// [rows, heads, D] bf16 view with the given row stride; box 64 x 1 x 128.
+// [rows, heads, D] view of 16-bit elements (bf16 or fp16) with the given row
+// stride; box 64 x 1 x 128.
 static bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int heads, int D,
-                     int64_t tok_stride) {
+                     int64_t tok_stride, int fmt) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)tok_stride * 2};
   cuuint32_t box[3] = {64, 1, (cuuint32_t)kTcBM};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+  const CUtensorMapDataType dt =
+      fmt == kFmtBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUresult r = enc(map, dt, 3, const_cast<void*>(ptr), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, int kFmt>
 static cudaError_t launch_tc_t(const FwdParams& p, cudaStream_t stream) {
   using C = TcCfg<D>;
   FwdParams pp = p;
@@ -867,24 +870,31 @@ static cudaError_t launch_tc_t(const FwdParams& p, cudaStream_t stream) {
   const int64_t grid = per_item ? items : (items < sms[dev] ? items : sms[dev]);
   const int claim_limit = per_item ? 1 : 0;
   TcMaps maps;
-  if (!make_map(&maps.q, p.q, p.total_rows, p.heads, D, p.tok_stride) ||
-      !make_map(&maps.k, p.k, p.total_rows, p.heads_kv, D, p.kv_tok_stride) ||
-      !make_map(&maps.v, p.v, p.total_rows, p.heads_kv, D, p.kv_tok_stride))
+  if (!make_map(&maps.q, p.q, p.total_rows, p.heads, D, p.tok_stride, kFmt) ||
+      !make_map(&maps.k, p.k, p.total_rows, p.heads_kv, D, p.kv_tok_stride, kFmt) ||
+      !make_map(&maps.v, p.v, p.total_rows, p.heads_kv, D, p.kv_tok_stride, kFmt))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D>,
+  cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D, kFmt>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  fwd_tc_kernel<D><<<(unsigned)grid, kTcThreads, C::kSmemBytes, stream>>>(pp, maps, (int)items,
-                                                                        claim_limit);
+  fwd_tc_kernel<D, kFmt><<<(unsigned)grid, kTcThreads, C::kSmemBytes, stream>>>(
+      pp, maps, (int)items, claim_limit);
   return cudaGetLastError();
 }
 
-// bf16 inputs, d_head 64 or 128.
-cudaError_t launch_fwd_tc(const FwdParams& p, cudaStream_t stream) {
-  switch (p.d_head) {
-    case 64: return launch_tc_t<64>(p, stream);
-    case 128: return launch_tc_t<128>(p, stream);
+// 16-bit inputs (fmt kFmtBF16 or kFmtF16), d_head 64 or 128.
+cudaError_t launch_fwd_tc(const FwdParams& p, int fmt, cudaStream_t stream) {
+  if (fmt == kFmtBF16) {
+    switch (p.d_head) {
+      case 64: return launch_tc_t<64, kFmtBF16>(p, stream);
+      case 128: return launch_tc_t<128, kFmtBF16>(p, stream);
+    }
+  } else if (fmt == kFmtF16) {
+    switch (p.d_head) {
+      case 64: return launch_tc_t<64, kFmtF16>(p, stream);
+      case 128: return launch_tc_t<128, kFmtF16>(p, stream);
+    }
   }
   return cudaErrorInvalidValue;
 }

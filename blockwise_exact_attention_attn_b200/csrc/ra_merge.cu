@@ -16,6 +16,7 @@
 // row divides 32), so the row's lse is read by its lanes before lane 0 of the
 // row overwrites it (separated by __syncwarp).
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "ra_common.cuh"
@@ -86,9 +87,25 @@ __device__ __forceinline__ void combine_chunk(float4* a, const float4* b, float 
   __stcs(a, r);
 }
 
-// bf16: a chunk is 8 values held in a uint4
-__device__ __forceinline__ void combine_chunk_bf16(uint4* a, const uint4* b, float wa, float wb,
-                                                   bool b_only, bool a_only) {
+// Pairs of 16-bit values to and from float2.
+__device__ __forceinline__ float2 to_float2(__nv_bfloat162 v) { return __bfloat1622float2(v); }
+__device__ __forceinline__ float2 to_float2(__half2 v) { return __half22float2(v); }
+template <typename T2>
+__device__ __forceinline__ T2 from_float2(float x, float y);
+template <>
+__device__ __forceinline__ __nv_bfloat162 from_float2<__nv_bfloat162>(float x, float y) {
+  return __floats2bfloat162_rn(x, y);
+}
+template <>
+__device__ __forceinline__ __half2 from_float2<__half2>(float x, float y) {
+  return __floats2half2_rn(x, y);
+}
+
+// 16-bit elements (T2 = __nv_bfloat162 or __half2): a chunk is 8 values in a
+// uint4
+template <typename T2>
+__device__ __forceinline__ void combine_chunk_16(uint4* a, const uint4* b, float wa, float wb,
+                                                 bool b_only, bool a_only) {
   uint4 x = *a;
   const uint4 y = __ldcs(b);
   uint4 r;
@@ -97,20 +114,21 @@ __device__ __forceinline__ void combine_chunk_bf16(uint4* a, const uint4* b, flo
   } else if (a_only) {
     r = x;
   } else {
-    const __nv_bfloat162* xa = reinterpret_cast<const __nv_bfloat162*>(&x);
-    const __nv_bfloat162* yb = reinterpret_cast<const __nv_bfloat162*>(&y);
-    __nv_bfloat162* rr = reinterpret_cast<__nv_bfloat162*>(&r);
+    const T2* xa = reinterpret_cast<const T2*>(&x);
+    const T2* yb = reinterpret_cast<const T2*>(&y);
+    T2* rr = reinterpret_cast<T2*>(&r);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float2 fa = __bfloat1622float2(xa[i]);
-      const float2 fb = __bfloat1622float2(yb[i]);
-      rr[i] = __floats2bfloat162_rn(wa * fa.x + wb * fb.x, wa * fa.y + wb * fb.y);
+      const float2 fa = to_float2(xa[i]);
+      const float2 fb = to_float2(yb[i]);
+      rr[i] = from_float2<T2>(wa * fa.x + wb * fb.x, wa * fa.y + wb * fb.y);
     }
   }
   __stcs(a, r);
 }
 
-template <bool kBf16>
+// kType: 0 = fp32, 1 = bf16, 2 = fp16
+template <int kType>
 __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
   const int64_t total = p.rows << p.log2_chunks;
   const int lane = threadIdx.x & 31;
@@ -140,13 +158,15 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
       merge_weights(la, lb, &wa, &wb, &lse);
       const bool b_only = la == -INFINITY && lb != -INFINITY;
       const bool a_only = lb == -INFINITY;
-      if (kBf16) {
+      if (kType != 0) {
         uint4* a = reinterpret_cast<uint4*>(p.out_a) + chunk;
         const uint4* b = reinterpret_cast<const uint4*>(p.out_b) + chunk;
         if (la == -INFINITY && lb == -INFINITY) {
           __stcs(a, make_uint4(0u, 0u, 0u, 0u));
+        } else if (kType == 1) {
+          combine_chunk_16<__nv_bfloat162>(a, b, wa, wb, b_only, a_only);
         } else {
-          combine_chunk_bf16(a, b, wa, wb, b_only, a_only);
+          combine_chunk_16<__half2>(a, b, wa, wb, b_only, a_only);
         }
       } else {
         float4* a = reinterpret_cast<float4*>(p.out_a) + chunk;
@@ -162,7 +182,7 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
   }
 }
 
-// dtype: 0 = fp32, 1 = bf16.  The host checks that the chunks per row are a
+// dtype: 0 = fp32, 1 = bf16, 2 = fp16.  The host checks that the chunks per row are a
 // power of two dividing 32 and that rows < 2^31.
 cudaError_t launch_merge(void* out_a, float* lse_a, const void* out_b, const float* lse_b,
                          int batch, int heads, int seqlen, int d_head, int dtype,
@@ -190,9 +210,11 @@ cudaError_t launch_merge(void* out_a, float* lse_a, const void* out_b, const flo
   const int64_t need = (total + threads - 1) / threads;
   if (need < blocks) blocks = need;
   if (dtype == 0)
-    merge_kernel<false><<<(unsigned)blocks, threads, 0, stream>>>(p);
+    merge_kernel<0><<<(unsigned)blocks, threads, 0, stream>>>(p);
+  else if (dtype == 1)
+    merge_kernel<1><<<(unsigned)blocks, threads, 0, stream>>>(p);
   else
-    merge_kernel<true><<<(unsigned)blocks, threads, 0, stream>>>(p);
+    merge_kernel<2><<<(unsigned)blocks, threads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -5,6 +5,11 @@
 
 namespace ra {
 
+// Element formats of the 16-bit inputs, as the kind::f16 MMA encodes them
+// (A and B always share one).
+constexpr int kFmtF16 = 0;
+constexpr int kFmtBF16 = 1;
+
 // One forward call, in the form every forward kernel consumes.  Rows of all
 // sequences are addressed as one token axis: token row r of sequence b is
 // global row seq_base(b) + r, with seq_base(b) = b * seqlen (dense) or

@@ -26,7 +26,7 @@ CONTIGUOUS, STRIPED = 0, 1
 @dataclass(frozen=True)
 class Workload:
     name: str
-    dtype: str              # "f32" or "bf16"
+    dtype: str              # "f32", "bf16" or "f16"
     batch: int
     heads: int
     seqlen: int             # per sequence (dense) or total rows (varlen)
@@ -53,12 +53,12 @@ class Workload:
 
     @property
     def torch_dtype(self):
-        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+        return {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}[self.dtype]
 
 
 # The five workloads of the benchmark description (sizes, seeds) plus small
-# variants used by the tests, and one grouped-query workload (8 query heads
-# per key/value head).
+# variants used by the tests, one grouped-query workload (8 query heads per
+# key/value head) and the headline shape in fp16.
 WORKLOADS = {
     "fp32_b1_h1_s1024_d16_noncausal_n16": Workload(
         "fp32_b1_h1_s1024_d16_noncausal_n16", "f32", 1, 1, 1024, 16, False, 16,
@@ -81,6 +81,9 @@ WORKLOADS = {
     "bf16_b1_h8_s262144_d128_causal_striped_n16_p4": Workload(
         "bf16_b1_h8_s262144_d128_causal_striped_n16_p4", "bf16", 1, 8, 262144, 128, True,
         16, STRIPED, 4, 5),
+    "f16_b2_h16_s8192_d128_noncausal_n8": Workload(
+        "f16_b2_h16_s8192_d128_noncausal_n8", "f16", 2, 16, 8192, 128, False, 8,
+        CONTIGUOUS, 8, 7),
     "bf16_b1_h32_kv4_s32768_d128_causal_n8_contiguous": Workload(
         "bf16_b1_h32_kv4_s32768_d128_causal_n8_contiguous", "bf16", 1, 32, 32768, 128, True,
         8, CONTIGUOUS, 8, 6, heads_kv=4),

@@ -66,7 +66,10 @@ typedef enum {
 
 typedef enum { RA_LAYOUT_CONTIGUOUS = 0, RA_LAYOUT_STRIPED = 1 } ra_layout;
 
-typedef enum { RA_F32 = 0, RA_BF16 = 1 } ra_dtype;
+/* Element type of q, k, v and out.  The "Tensorflow flash attention" page
+ * lists fp16 and bf16 as the flash-attention input types; fp32 is the gist's
+ * (and the fp32 workload's) type. */
+typedef enum { RA_F32 = 0, RA_BF16 = 1, RA_F16 = 2 } ra_dtype;
 
 /*
  * ring_attn_fwd -- exact attention forward, ring-ordered blockwise.
@@ -92,7 +95,8 @@ typedef enum { RA_F32 = 0, RA_BF16 = 1 } ra_dtype;
  *            cu_seqlens[batch] (the host never reads cu_seqlens, so the call
  *            stays asynchronous; the kernels check it).
  *  d_head    head dimension: RA_F32 accepts 16, 32, 64, 128;
- *            RA_BF16 accepts 64, 128.
+ *            RA_BF16 and RA_F16 accept 64, 128 (tensor cores; bf16 or fp16
+ *            products accumulated in fp32).
  *  n_ring_blocks  N >= 1, the number of virtual ring devices per sequence.
  *  layout    ra_layout; buffers are in that stored order and out/lse are
  *            returned in the same order.
@@ -200,8 +204,8 @@ ra_status ring_attn_fwd_simt(const void* q, const void* k, const void* v,
  *  out_a, out_b  dtype [batch, seqlen, heads, d_head] (varlen results: batch
  *                = 1, seqlen = total rows).  out_a is overwritten.
  *  lse_a, lse_b  float32 [batch, heads, seqlen].  lse_a is overwritten.
- *  d_head        RA_F32: 4, 8, 16, 32, 64 or 128; RA_BF16: 8, 16, 32, 64,
- *                128 or 256 (a row is 1 to 32 whole 16-byte chunks).
+ *  d_head        RA_F32: 4, 8, 16, 32, 64 or 128; RA_BF16 and RA_F16: 8, 16,
+ *                32, 64, 128 or 256 (a row is 1 to 32 whole 16-byte chunks).
  * Errors: RA_ERR_INVALID for null/misaligned pointers, non-positive sizes,
  * an unsupported d_head or dtype; RA_ERR_CUDA when the launch fails.
  */

@@ -8,7 +8,11 @@ import oracle
 import blockwise_exact_attention_attn_b200 as ra
 from blockwise_exact_attention_attn_b200 import inputs as gen
 
-TOL = {"f32": (1e-4, 1e-5), "bf16": (2e-2, 1e-3)}   # (max |dO|, max |dlse|)
+# (max |dO|, max |dlse|).  fp16: outputs are rounded to an 11-bit significand
+# (half an ulp is 2^-11 relative, under 2e-3 for |O| < 4) and P enters the
+# tensor cores in fp16 (2^-11 relative), so 4e-3 on O; lse is computed in fp32
+# as for bf16.
+TOL = {"f32": (1e-4, 1e-5), "bf16": (2e-2, 1e-3), "f16": (4e-3, 1e-3)}
 
 
 def run_gpu(w, inp, impl="tc", stream=None):

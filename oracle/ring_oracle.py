@@ -257,6 +257,44 @@ def merge(out_a, lse_a, out_b, lse_b):
     return out, lse
 
 
+def block_rows(L: int, N: int, layout: int, r: int) -> np.ndarray:
+    """Stored indices of ring block r of a sequence of length L."""
+    t = np.arange(L, dtype=np.int64)
+    return np.flatnonzero(ring_block(t, L, N, layout) == r)
+
+
+def ring_step(q, k, v, out_prev, lse_prev, L: int, N: int, layout: int, causal: bool,
+              scale: float, q_block: int, kv_block: int):
+    """One key/value-outer ring step, fp64: the queries of ring block q_block
+    fold the keys of ring block kv_block into their running result.
+
+    The issue thread "A ring attention with flash attention kernel
+    implementation" notes that with keys and values on the outer loop the
+    reduced outputs and lse of the queries are stored and passed back in on
+    the next ring pass; the fold is the merge above of the running result
+    with attention over the new block's keys.
+
+    q: [nq, H, D] rows of block q_block in stored order; k, v: [nk, H, D]
+    rows of block kv_block; out_prev [nq, H, D] and lse_prev [H, nq] the
+    running normalised output and lse (lse = -inf: nothing folded yet).  The
+    mask is the sequence's (causal in original positions); no pass limit
+    applies, the caller chooses the blocks.  Returns (out, lse) in the same
+    shapes.
+    """
+    tq = block_rows(L, N, layout, q_block)
+    tk = block_rows(L, N, layout, kv_block)
+    mask = allowed(tq[:, None], tk[None, :], L, N, layout, causal, N)
+    H = q.shape[1]
+    o_new = np.zeros(np.shape(q), dtype=np.float64)
+    l_new = np.zeros((H, tq.size), dtype=np.float64)
+    for h in range(H):
+        o_new[:, h, :], l_new[h] = masked_attention(q[:, h, :], k[:, h, :], v[:, h, :], mask,
+                                                    scale)
+    out, lse = merge(np.transpose(out_prev, (1, 0, 2)), lse_prev,
+                     np.transpose(o_new, (1, 0, 2)), l_new)
+    return np.transpose(out, (1, 0, 2)), lse
+
+
 # --------------------------------------------------------------------------
 # Helpers for tests and the CPU baseline
 # --------------------------------------------------------------------------
@@ -307,8 +345,8 @@ def row_flops(p: Problem, seq, head, row) -> float:
 
 
 __all__ = [
-    "CONTIGUOUS", "STRIPED", "Problem", "allowed", "allowed_matrix",
+    "CONTIGUOUS", "STRIPED", "Problem", "allowed", "allowed_matrix", "block_rows",
     "attention_full", "attention_rows", "blas_threads", "masked_attention",
-    "merge", "ring_block", "row_flops", "striped_block_sizes", "timed_rows",
+    "merge", "ring_block", "ring_step", "row_flops", "striped_block_sizes", "timed_rows",
     "kv_head", "token_pos", "unmasked_pairs",
 ]

@@ -237,6 +237,67 @@ def test_grouped_query_zero_queries_give_group_means():
 
 
 # ----------------------------------------------------------------------------
+# Key/value-outer ring step
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("layout,causal", [(0, True), (1, True), (0, False), (1, False)])
+def test_ring_steps_in_ring_order_reach_full_attention(layout, causal):
+    """Folding every key/value block into the queries of each block, in ring
+    order from an empty state, reaches full attention (the blockwise result
+    is exact)."""
+    L, N, H, D = 24, 4, 2, 5
+    rng = np.random.default_rng(21)
+    q, k, v = (rng.standard_normal((L, H, D)) for _ in range(3))
+    scale = 0.45
+    full_o, full_l = oracle.attention_full(problem(q, k, v, N, layout, causal, N, scale))
+    for i in range(N):
+        tq = oracle.block_rows(L, N, layout, i)
+        out = np.zeros((tq.size, H, D))
+        lse = np.full((H, tq.size), -np.inf)
+        for s in range(N):
+            j = (i - s) % N
+            tk = oracle.block_rows(L, N, layout, j)
+            out, lse = oracle.ring_step(q[tq], k[tk], v[tk], out, lse, L, N, layout, causal,
+                                        scale, i, j)
+        assert np.abs(out - full_o[tq]).max() < TIGHT
+        assert np.abs(lse - full_l[:, tq]).max() < TIGHT
+
+
+def test_ring_step_order_does_not_matter_and_one_step_is_block_attention():
+    L, N, H, D, layout = 30, 5, 1, 4, 1
+    rng = np.random.default_rng(22)
+    q, k, v = (rng.standard_normal((L, H, D)) for _ in range(3))
+    scale = 0.6
+    i = 3
+    tq = oracle.block_rows(L, N, layout, i)
+    results = []
+    for order in ([0, 1, 2, 3, 4], [4, 2, 0, 3, 1]):
+        out = np.zeros((tq.size, H, D))
+        lse = np.full((H, tq.size), -np.inf)
+        for j in order:
+            tk = oracle.block_rows(L, N, layout, j)
+            out, lse = oracle.ring_step(q[tq], k[tk], v[tk], out, lse, L, N, layout, True,
+                                        scale, i, j)
+        results.append((out, lse))
+    assert np.abs(results[0][0] - results[1][0]).max() < TIGHT
+    assert np.abs(results[0][1] - results[1][1]).max() < TIGHT
+    # one step from the empty state: attention over that block's keys, against
+    # torch SDPA with the explicit mask restricted to the block
+    j = 1
+    tk = oracle.block_rows(L, N, layout, j)
+    out, lse = oracle.ring_step(q[tq], k[tk], v[tk], np.zeros((tq.size, H, D)),
+                                np.full((H, tq.size), -np.inf), L, N, layout, True, scale, i, j)
+    mask = torch.from_numpy(explicit_mask(L, N, layout, True, N)[np.ix_(tq, tk)])
+    has = mask.any(dim=1).numpy()
+    qt, kt, vt = (torch.from_numpy(x[:, 0]) for x in (q[tq], k[tk], v[tk]))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        qt[has][None], kt[None], vt[None], attn_mask=mask[has][None], scale=scale)[0]
+    assert np.abs(out[has, 0] - ref.numpy()).max() < TIGHT
+    # rows without an allowed key in the block keep the empty state
+    assert np.all(out[~has] == 0.0) and np.all(np.isneginf(lse[0, ~has]))
+
+
+# ----------------------------------------------------------------------------
 # Brute force on tiny inputs (pure Python exp / normalise)
 # ----------------------------------------------------------------------------
 

@@ -289,6 +289,47 @@ def measure_workload(name, steps, warmup, dist, dev, peaks):
     return res, w, in_bytes, out_bytes, flops
 
 
+RING_STEPS_WORKLOAD = "bf16_b1_h32_s32768_d128_causal_n8_contiguous"
+
+
+def measure_ring_steps(steps, warmup, dist, dev, peaks):
+    """The 32K causal workload computed as key/value-outer ring steps: for
+    every query block i, the N blocks folded in ring order (N^2 step calls,
+    what N devices of a ring run between them), fp32 running state."""
+    import blockwise_exact_attention_attn_b200 as ra
+    from blockwise_exact_attention_attn_b200 import inputs as gen
+    w = gen.WORKLOADS[RING_STEPS_WORKLOAD]
+    inp = gen.make_device_inputs(w, dev, seed=w.seed + 1000 * dist.rank)
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    B, S, H, D = q.shape
+    N = w.n_ring
+    b = S // N
+    blk = [(q[:, r * b:(r + 1) * b], k[:, r * b:(r + 1) * b], v[:, r * b:(r + 1) * b])
+           for r in range(N)]
+    outs = [torch.empty(B, b, H, D, dtype=torch.float32, device=dev) for _ in range(N)]
+    lses = [torch.empty(B, H, b, dtype=torch.float32, device=dev) for _ in range(N)]
+
+    def step():
+        for i in range(N):
+            for st in range(N):
+                j = (i - st) % N
+                ra.ring_attn_fwd_step(blk[i][0], blk[j][1], blk[j][2], outs[i], lses[i], B, H,
+                                      S, D, N, i, j, st > 0, w.layout, w.causal,
+                                      w.softmax_scale)
+
+    flops = workload_flops(w, [S] * B)
+    ms = time_steps(step, steps, warmup, dist, dev, graph=True)
+    if ra.ring_attn_status() != ra.RA_OK:
+        raise RuntimeError("ring steps: device status not OK")
+    per = ms / steps
+    tflops = flops / (per * 1e-3) / 1e12
+    return {"workload": RING_STEPS_WORKLOAD + " as key/value-outer ring steps",
+            "step_calls": N * N, "ms_per_step": per, "tflops_per_gpu": tflops,
+            "tflops": tflops * dist.world,
+            "frac_of_measured_bf16_peak": tflops / peaks["bf16_tflops"],
+            "kernel": "fwd_tc step mode (tcgen05)"}
+
+
 def measure_merge(steps, warmup, dist, dev, peaks):
     """(O, lse) merge on fp32 partials shaped like the headline output."""
     import blockwise_exact_attention_attn_b200 as ra
@@ -465,6 +506,12 @@ def run_ours(args, dist):
             except Exception as e:  # report, never hide
                 extras.append({"workload": name, "error": str(e)})
     merge = measure_merge(args.steps, args.warmup, dist, dev, peaks)
+    ring_steps = None
+    if not args.no_extras:
+        try:
+            ring_steps = measure_ring_steps(max(3, min(args.steps, 10)), 3, dist, dev, peaks)
+        except Exception as e:  # report, never hide
+            ring_steps = {"workload": RING_STEPS_WORKLOAD + " as ring steps", "error": str(e)}
     e2e = measure_e2e(w, args.steps, args.warmup, dist, dev) if not w.varlen else None
 
     cpu = None
@@ -507,6 +554,7 @@ def run_ours(args, dist):
         "gpu_launches": args.steps,
         "e2e": e2e,
         "merge": merge,
+        "ring_steps": ring_steps,
         "workloads": extras,
         "cpu_baseline": cpu,
     }

@@ -22,6 +22,7 @@ from ._binding import (  # noqa: F401
     ring_attn_func,
     ring_attn_fwd,
     ring_attn_fwd_noalloc,
+    ring_attn_fwd_step,
     ring_attn_gqa_fwd,
     ring_attn_fwd_simt,
     ring_attn_merge,

@@ -26,6 +26,7 @@ F32, BF16, F16 = 0, 1, 2
 EXPORTS = (
     "ring_attn_fwd",
     "ring_attn_gqa_fwd",
+    "ring_attn_fwd_step",
     "ring_attn_qkvpacked_fwd",
     "ring_attn_fwd_simt",
     "ring_attn_fwd_noalloc",
@@ -69,6 +70,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib = ctypes.CDLL(path)
         lib.ring_attn_fwd.argtypes = _FWD_ARGS
         lib.ring_attn_fwd.restype = _c_int
+        lib.ring_attn_fwd_step.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int,
+                                           _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
+                                           _c_int, _c_int, _c_int, _c_int, _c_vp]
+        lib.ring_attn_fwd_step.restype = _c_int
         lib.ring_attn_gqa_fwd.argtypes = _GQA_ARGS
         lib.ring_attn_gqa_fwd.restype = _c_int
         lib.ring_attn_fwd_simt.argtypes = _FWD_ARGS
@@ -185,6 +190,25 @@ def ring_attn_gqa_fwd(q, k, v, out, lse, batch: int, heads: int, heads_kv: int, 
         _ptr(cu_seqlens, "cu_seqlens"), _dtype_code(q) if dtype is None else int(dtype),
         _stream(stream))
     _check("ring_attn_gqa_fwd", st)
+
+
+def ring_attn_fwd_step(q, k, v, out, lse, batch: int, heads: int, seqlen: int, d_head: int,
+                       n_ring_blocks: int, q_block: int, kv_block: int, accumulate: bool,
+                       layout=CONTIGUOUS, causal: bool = False,
+                       softmax_scale: Optional[float] = None, dtype: Optional[int] = None,
+                       stream=None) -> None:
+    """Fold ring block kv_block's keys into the running fp32 (out, lse) of
+    ring block q_block's queries (see ring_attn.h)."""
+    lib = load_library()
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d_head)
+    st = lib.ring_attn_fwd_step(
+        _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _ptr(out, "out"), _ptr(lse, "lse"),
+        int(batch), int(heads), int(seqlen), int(d_head), int(n_ring_blocks),
+        _layout_code(layout), int(bool(causal)), float(softmax_scale), int(q_block),
+        int(kv_block), int(bool(accumulate)), _dtype_code(q) if dtype is None else int(dtype),
+        _stream(stream))
+    _check("ring_attn_fwd_step", st)
 
 
 def ring_attn_fwd_simt(q, k, v, out, lse, batch: int, heads: int, seqlen: int, d_head: int,

@@ -135,6 +135,9 @@ ra::FwdParams make_params(const void* q, const void* k, const void* v, int64_t t
   }
   p.status = nullptr;
   p.work_counter = nullptr;
+  p.step = 0;
+  p.q_block = p.kv_block = p.step_rows = 0;
+  p.accumulate = 0;
   return p;
 }
 
@@ -195,6 +198,45 @@ ra_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out, 
                              n_ring_blocks, layout, causal, softmax_scale, max_ring_passes,
                              cu_seqlens),
                  dtype, stream, false);
+}
+
+ra_status ring_attn_fwd_step(const void* q, const void* k, const void* v, float* out,
+                             float* lse, int batch, int heads, int seqlen, int d_head,
+                             int n_ring_blocks, int layout, int causal, float softmax_scale,
+                             int q_block, int kv_block, int accumulate, int dtype,
+                             void* stream) {
+  if (!q || !k || !v || !out || !lse) return RA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return RA_ERR_INVALID;
+  ra_status st = validate_fwd(batch, heads, heads, seqlen, d_head, n_ring_blocks, layout,
+                              causal, softmax_scale, n_ring_blocks, nullptr, dtype);
+  if (st != RA_OK) return st;
+  if (q_block < 0 || q_block >= n_ring_blocks || kv_block < 0 || kv_block >= n_ring_blocks)
+    return RA_ERR_INVALID;
+  if (accumulate != 0 && accumulate != 1) return RA_ERR_INVALID;
+  // the step runs on the tensor cores only, with whole 128-row tiles per block
+  const int rows = seqlen / n_ring_blocks;
+  if (dtype == RA_F32 || softmax_scale == 0.f || rows % 128 != 0) return RA_ERR_UNSUPPORTED;
+  // An accumulating step over a block pair that the mask hides entirely
+  // leaves the state as it is: nothing to launch.
+  const ra::RingGeom g = ra::make_geom(seqlen, n_ring_blocks, layout, causal, n_ring_blocks);
+  if (accumulate && ra::classify(g, q_block * rows, (q_block + 1) * rows, kv_block * rows,
+                                 (kv_block + 1) * rows) == ra::CLS_EMPTY)
+    return RA_OK;
+  const int64_t hd = (int64_t)heads * d_head;
+  ra::FwdParams p = make_params(q, k, v, hd, heads, hd, out, lse, batch, heads, seqlen, d_head,
+                                n_ring_blocks, layout, causal, softmax_scale, n_ring_blocks,
+                                nullptr);
+  p.step = 1;
+  p.q_block = q_block;
+  p.kv_block = kv_block;
+  p.step_rows = rows;
+  p.accumulate = accumulate;
+  p.total_rows = batch * rows;
+  p.lse_seq_stride = (int64_t)heads * rows;
+  p.lse_head_stride = rows;
+  p.order = 0;
+  return run_fwd(p, dtype, stream, false);
 }
 
 ra_status ring_attn_gqa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,

@@ -407,15 +407,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const SeqWork it = find_work_item(p, kRows, item);
       if (!it.live) continue;
       if (lane == 0) {
+        // query rows of this sequence held in q: the sequence, or one ring block
+        const int nrows = p.step ? p.step_rows : it.L;
         const int q0 = it.qr * kRows;
-        const int qm = min(q0 + kTcBM, it.L), q1 = min(q0 + kRows, it.L);
+        const int qm = min(q0 + kTcBM, nrows), q1 = min(q0 + kRows, nrows);
         const RingGeom g = make_geom(it.L, p.n_ring, p.layout, p.causal, p.passes);
-        TileWalk walk;
-        walk.init(g, q0, qm, q1, kTcBN);
-        int kt, c0, c1;
         ok = put(item_header(item)) && put(it.b) && put(it.qr) && put(it.h) && put(it.base) &&
              put(it.L);
-        while (ok && walk.next(&kt, &c0, &c1)) ok = put((kt << 4) | (c1 << 2) | c0);
+        int kt, c0, c1;
+        if (!p.step) {
+          TileWalk walk;
+          walk.init(g, q0, qm, q1, kTcBN);
+          while (ok && walk.next(&kt, &c0, &c1)) ok = put((kt << 4) | (c1 << 2) | c0);
+        } else {
+          // one ring step: the tiles of key/value block kv_block (tile-aligned
+          // blocks; kt counts tiles inside the block)
+          const int qo = p.q_block * p.step_rows, ko = p.kv_block * p.step_rows;
+          for (kt = 0; ok && kt < p.step_rows / kTcBN; ++kt) {
+            const int k0 = ko + kt * kTcBN;
+            c0 = classify(g, qo + q0, qo + qm, k0, k0 + kTcBN);
+            c1 = classify(g, qo + qm, qo + q1, k0, k0 + kTcBN);
+            if (c0 != CLS_EMPTY || c1 != CLS_EMPTY) ok = put((kt << 4) | (c1 << 2) | c0);
+          }
+        }
         if (ok) ok = put(kItemEnd);
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -592,8 +606,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               tc_fence_after();
               if (!started[i]) wait_ofree(i);
               if (!ok) break;
+              // an accumulating ring step adds to the O loaded from the state
               issue_pv<D>(tmem + C::kColO + i * D, pdesc0 + i * kPStep,
-                          vdesc0 + slot_v * kSlotStep, idesc_o, started[i]);
+                          vdesc0 + slot_v * kSlotStep, idesc_o, started[i] || p.accumulate);
               umma_commit(&ctrl->pv_done[i]);
               started[i] = true;
             }
@@ -652,17 +667,52 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ok = read_item<true>(rd, &it, abort_flag);
       if (!ok) break;
       const int L = it.L;
+      // sq: row in q/out; sqg: its stored index in the sequence (they differ
+      // in a ring step, where q holds one block); kvo: same offset for keys
       const int sq = it.qr * kRows + tile * kTcBM + r;
-      const bool valid = sq < L;
+      const int qo = p.step ? p.q_block * p.step_rows : 0;
+      const int kvo = p.step ? p.kv_block * p.step_rows : 0;
+      const bool valid = sq < (p.step ? p.step_rows : L);
       int rq = 0, tq = 0;
       if (valid) {
         const RingGeom g = make_geom(L, p.n_ring, p.layout, p.causal, p.passes);
-        rq = block_of(g, sq);
-        tq = token_of(g, sq, rq);
+        rq = block_of(g, qo + sq);
+        tq = token_of(g, qo + sq, rq);
       }
+      const int64_t li = (int64_t)it.b * p.lse_seq_stride + (int64_t)it.h * p.lse_head_stride +
+                         (p.cu_seqlens ? it.base : 0) + sq;
       float m_ref = -INFINITY;  // reference max, log2 domain
       float l = 0.f;
       bool first = true;
+      // A ring step that accumulates starts from the running state: m = lse
+      // (log2 units) with l = 1 and O = the normalised output (O = 0 where
+      // nothing was folded yet); the first PV then adds to O.
+      const bool from_state = p.step && p.accumulate;
+      if (from_state) {
+        const float lp = valid ? p.lse[li] : -INFINITY;
+        const bool has = lp > -INFINITY;
+        if (has) {
+          m_ref = lp * 1.4426950408889634f;
+          l = 1.f;
+        }
+        const float* orow = static_cast<const float*>(p.out) +
+                            ((int64_t)(it.base + sq) * p.heads + it.h) * D;
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t o[32];
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            const float4 f = has ? *reinterpret_cast<const float4*>(orow + c + j)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+            o[j] = __float_as_uint(f.x);
+            o[j + 1] = __float_as_uint(f.y);
+            o[j + 2] = __float_as_uint(f.z);
+            o[j + 3] = __float_as_uint(f.w);
+          }
+          RA_TMEM_ST32(tO + c, o);
+        }
+        tmem_wait_st();
+      }
 
       while (true) {
         int e;
@@ -685,7 +735,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // S_tile is in registers: the next S may be computed into its columns
         tc_fence_before();
         mbar_arrive(&ctrl->s_free[tile]);
-        const int k0 = entry_tile(e) * kTcBN;
+        const int k0 = kvo + entry_tile(e) * kTcBN;  // stored index of the tile's first key
         const int nk = min(kTcBN, L - k0);
         if (cls == CLS_PARTIAL || nk < kTcBN) {
           apply_mask(x, p, L, valid, cls, rq, tq, k0, nk);
@@ -736,7 +786,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         l = l * alpha + ((f32x2_lo(sum2[0]) + f32x2_hi(sum2[0])) +
                          (f32x2_lo(sum2[1]) + f32x2_hi(sum2[1])));
-        if (!first && __any_sync(0xffffffffu, need)) {
+        if ((!first || from_state) && __any_sync(0xffffffffu, need)) {
           // O_row *= alpha (exactly 1.0 for rows that keep their reference)
 #pragma unroll
           for (int c = 0; c < D; c += 32) {
@@ -761,34 +811,53 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ok = warp_wait(&ctrl->o_full[tile], k & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
+      const int64_t orow_off = ((int64_t)(it.base + sq) * p.heads + it.h) * D;
       if (!first) {
         const float inv_l = valid ? 1.f / l : 0.f;
-        uint16_t* orow = static_cast<uint16_t*>(p.out) +
-                              ((int64_t)(it.base + sq) * p.heads + it.h) * D;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
           uint32_t o[32];
           RA_TMEM_LD32(tO + c, o);
           tmem_wait_ld();
-          uint32_t pk[16];
+          if (p.step) {
+            // ring step: the running output stays fp32
+            if (valid) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow_off + c);
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            pk[j] = pack_x2<kFmt>(__uint_as_float(o[2 * j]) * inv_l,
-                                __uint_as_float(o[2 * j + 1]) * inv_l);
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c);
+              for (int j = 0; j < 8; ++j)
+                dst[j] = make_float4(
+                    __uint_as_float(o[4 * j]) * inv_l, __uint_as_float(o[4 * j + 1]) * inv_l,
+                    __uint_as_float(o[4 * j + 2]) * inv_l, __uint_as_float(o[4 * j + 3]) * inv_l);
+            }
+          } else {
+            uint32_t pk[16];
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            for (int j = 0; j < 16; ++j)
+              pk[j] = pack_x2<kFmt>(__uint_as_float(o[2 * j]) * inv_l,
+                                    __uint_as_float(o[2 * j + 1]) * inv_l);
+            if (valid) {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + orow_off + c);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            }
           }
         }
+      } else if (p.step && !p.accumulate && valid) {
+        // no key of this block is visible to the row: the empty result
+        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow_off);
+#pragma unroll
+        for (int j = 0; j < D / 4; ++j) dst[j] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
       tc_fence_before();
       mbar_arrive(&ctrl->o_free[tile]);
-      if (!first && valid) {
-        const int64_t li = (int64_t)it.b * p.lse_seq_stride + (int64_t)it.h * p.lse_head_stride +
-                           (p.cu_seqlens ? it.base : 0) + sq;
-        p.lse[li] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
+      if (valid) {
+        if (!first) {
+          p.lse[li] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
+        } else if (p.step && !p.accumulate) {
+          p.lse[li] = -INFINITY;
+        }
+        // (an accumulating step without new keys leaves the state as it was)
       }
       ++k;
     }
@@ -851,7 +920,7 @@ template <int D, int kFmt>
 static cudaError_t launch_tc_t(const FwdParams& p, cudaStream_t stream) {
   using C = TcCfg<D>;
   FwdParams pp = p;
-  pp.n_qranges = (p.seqlen + kTcBM * kTcQT - 1) / (kTcBM * kTcQT);
+  pp.n_qranges = (q_rows_per_seq(p) + kTcBM * kTcQT - 1) / (kTcBM * kTcQT);
   set_striped_order(pp, kTcBM * kTcQT);
   const int64_t items = work_grid(pp, kTcBM * kTcQT);
   if (items == 0) return cudaSuccess;
@@ -865,8 +934,9 @@ static cudaError_t launch_tc_t(const FwdParams& p, cudaStream_t stream) {
     return cudaErrorInvalidDevice;
   // Dense causal work varies per item: one CTA per item, balanced by the
   // hardware block scheduler, measured faster than persistent CTAs there.
-  // Otherwise persistent CTAs (one per SM) claim items until none is left.
-  const bool per_item = p.causal && !p.cu_seqlens;
+  // Otherwise (and for ring steps, whose items are short) persistent CTAs
+  // (one per SM) claim items until none is left.
+  const bool per_item = p.causal && !p.cu_seqlens && !p.step;
   const int64_t grid = per_item ? items : (items < sms[dev] ? items : sms[dev]);
   const int claim_limit = per_item ? 1 : 0;
   TcMaps maps;

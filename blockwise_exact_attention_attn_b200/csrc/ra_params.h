@@ -38,7 +38,24 @@ struct FwdParams {
   float scale_log2;         // scale * log2(e)
   int* status;              // device status word (never NULL at launch)
   int* work_counter;        // persistent kernels: next work item (zeroed per launch)
+  // Key/value-outer ring step (ring_attn_fwd_step): q, out and lse hold the
+  // step_rows rows of ring block q_block of each sequence, k and v those of
+  // kv_block; seqlen stays the whole sequence (the ring geometry).  out is
+  // fp32; with accumulate the call folds into the running (out, lse).
+  int step;                 // 0: whole-sequence call
+  int q_block, kv_block, step_rows;
+  int accumulate;
 };
+
+// Query rows per dense sequence held by q/out: the whole sequence, or one
+// ring block in a step call.  (Varlen calls size each sequence from
+// cu_seqlens instead.)
+#if defined(__CUDACC__)
+__host__ __device__ __forceinline__
+#else
+inline
+#endif
+int q_rows_per_seq(const FwdParams& p) { return p.step ? p.step_rows : p.seqlen; }
 
 // Map a linear work index to (query range, batch, head).  The (batch, head)
 // pair is the slowest index, so the work running at one time shares the K/V

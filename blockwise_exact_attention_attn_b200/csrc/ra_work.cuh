@@ -39,9 +39,10 @@ __device__ __forceinline__ SeqWork find_work_item(const FwdParams& p, int rows_p
     w.b = it.b;
     w.qr = it.qr;
     w.h = it.h;
-    w.base = it.b * p.seqlen;
+    const int rows = q_rows_per_seq(p);
+    w.base = it.b * rows;
     w.L = p.seqlen;
-    w.live = (int64_t)it.qr * rows_per_cta < p.seqlen;
+    w.live = (int64_t)it.qr * rows_per_cta < rows;
     return w;
   }
   const int flat = item / p.heads;
@@ -95,7 +96,7 @@ __device__ __forceinline__ SeqWork find_work(const FwdParams& p, int rows_per_ct
 // Causal striped dense inputs whose ring blocks hold a whole number of work
 // items: order the items by local position (heaviest first).
 inline void set_striped_order(FwdParams& p, int rows_per_cta) {
-  if (p.cu_seqlens || !p.causal || p.layout != 1) return;
+  if (p.cu_seqlens || p.step || !p.causal || p.layout != 1) return;
   const int blk = p.seqlen / p.n_ring;
   if (blk % rows_per_cta != 0 || blk == 0) return;
   p.order = 2;
@@ -107,7 +108,7 @@ inline void set_striped_order(FwdParams& p, int rows_per_cta) {
 // sequences.
 inline int64_t work_grid(const FwdParams& p, int rows_per_cta) {
   if (!p.cu_seqlens) {
-    const int64_t nq = ((int64_t)p.seqlen + rows_per_cta - 1) / rows_per_cta;
+    const int64_t nq = ((int64_t)q_rows_per_seq(p) + rows_per_cta - 1) / rows_per_cta;
     return nq * p.batch * p.heads;
   }
   const int64_t nq = ((int64_t)p.total_rows + rows_per_cta - 1) / rows_per_cta + p.batch;

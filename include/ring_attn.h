@@ -154,6 +154,49 @@ ra_status ring_attn_gqa_fwd(const void* q, const void* k, const void* v,
                             void* stream);
 
 /*
+ * ring_attn_fwd_step -- one key/value-outer ring step: the queries of ring
+ * block q_block fold the keys and values of ring block kv_block into their
+ * running result (out, lse), in place.
+ *
+ * Source: issue thread "A ring attention with flash attention kernel
+ * implementation": with the keys and values iterated on the outer loop, the
+ * reduced outputs and lse of the queries are stored and passed back in on
+ * the next ring pass.  The fold is the online-softmax update started from
+ * the stored state (m = lse, l = 1, O = out), the same arithmetic as folding
+ * a partial result with ring_attn_merge.
+ *
+ *  q         dtype [batch, seqlen / n_ring_blocks, heads, d_head]: the rows
+ *            of ring block q_block in stored order (contiguous: tokens
+ *            [q_block * b, (q_block + 1) * b); striped: tokens q_block,
+ *            q_block + N, ...).
+ *  k, v      same shape: the rows of ring block kv_block.
+ *  out       float32, same shape as q: the running normalised output.  Read
+ *            when accumulate (rows with lse = -inf may hold anything), always
+ *            written for rows that see a key of the block; with accumulate =
+ *            0 rows that see none get 0.
+ *  lse       float32 [batch, heads, seqlen / n_ring_blocks]: the running
+ *            log-sum-exp, -inf for "nothing folded yet"; updated like out
+ *            (-inf written with accumulate = 0 for rows that see no key).
+ *  seqlen    tokens of the whole sequence (the ring geometry; causal masking
+ *            compares original positions over the whole sequence).
+ *  q_block, kv_block  ring blocks in [0, n_ring_blocks).
+ *  accumulate  1: fold into (out, lse); 0: start from the empty state.
+ * No pass limit applies: the caller chooses which blocks to fold.  An
+ * accumulating step over a block pair the mask hides entirely (causal
+ * contiguous, kv_block > q_block) returns RA_OK without launching anything.
+ * Errors: as ring_attn_fwd, plus RA_ERR_INVALID for a block index out of
+ * range or accumulate not in {0,1}; RA_ERR_UNSUPPORTED for RA_F32, a zero
+ * scale, or a block size seqlen / n_ring_blocks that is not a multiple of
+ * 128 (the step runs on the tensor cores with whole tiles per block).
+ */
+ra_status ring_attn_fwd_step(const void* q, const void* k, const void* v,
+                             float* out, float* lse, int batch, int heads,
+                             int seqlen, int d_head, int n_ring_blocks,
+                             int layout, int causal, float softmax_scale,
+                             int q_block, int kv_block, int accumulate,
+                             int dtype, void* stream);
+
+/*
  * ring_attn_qkvpacked_fwd -- same computation, q/k/v packed in one tensor.
  *
  * Source: issue thread "A ring attention with flash attention kernel

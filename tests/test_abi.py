@@ -86,6 +86,24 @@ def test_gqa_shares_the_forward_validation(lib):
                                  4, None, 1, None) == ra.RA_ERR_INVALID
 
 
+@pytest.mark.parametrize("over,want", [
+    (dict(q_block=4), "invalid"), (dict(kv_block=-1), "invalid"), (dict(acc=2), "invalid"),
+    (dict(seqlen=960), "unsupported"),       # blocks of 240 rows: not whole tiles
+    (dict(dtype=0), "unsupported"),          # fp32 has no tensor-core step
+    (dict(scale=0.0), "unsupported"),
+    (dict(out=None), "invalid"), (dict(seqlen=1002), "invalid"),   # not a multiple of N
+])
+def test_step_validation(lib, over, want):
+    a = dict(q=FAKE, out=FAKE, batch=1, heads=2, seqlen=1024, d=128, n=4, layout=0, causal=1,
+             scale=0.1, q_block=1, kv_block=0, acc=1, dtype=1)
+    a.update(over)
+    st = lib.ring_attn_fwd_step(a["q"], FAKE, FAKE, a["out"], FAKE, a["batch"], a["heads"],
+                                a["seqlen"], a["d"], a["n"], a["layout"], a["causal"],
+                                a["scale"], a["q_block"], a["kv_block"], a["acc"], a["dtype"],
+                                None)
+    assert st == {"invalid": ra.RA_ERR_INVALID, "unsupported": ra.RA_ERR_UNSUPPORTED}[want]
+
+
 @pytest.mark.parametrize("args", [
     (None, FAKE, FAKE, FAKE, 1, 1, 8, 128, 0),         # null
     (FAKE, FAKE + 4, FAKE, FAKE, 1, 1, 8, 128, 0),     # misaligned lse

@@ -295,6 +295,54 @@ def ring_step(q, k, v, out_prev, lse_prev, L: int, N: int, layout: int, causal: 
     return np.transpose(out, (1, 0, 2)), lse
 
 
+def attention_backward(p: Problem, dout):
+    """Gradients (dq, dk, dv) of sum(dout * O) for the forward of p, fp64,
+    from the plain definition, one (sequence, head) at a time.
+
+    The pages stop at the forward; the issue thread "A ring attention with
+    flash attention kernel implementation" notes that the backward is where
+    an implementation went wrong and that the returned lse is what the
+    blockwise method keeps.  The gradient itself is plain calculus on
+    O_i = sum_j P_ij v_j with P_ij = exp(s_ij - lse_i), s_ij = scale <q_i, k_j>
+    over the allowed keys:
+        dV_j = sum_i P_ij dO_i
+        dP_ij = <dO_i, v_j>,   D_i = <dO_i, O_i> = sum_j P_ij dP_ij
+        dS_ij = P_ij (dP_ij - D_i)
+        dQ_i = scale sum_j dS_ij k_j,   dK_j = scale sum_i dS_ij q_i
+    dout has q's shape [T, H, D]; k and v may have fewer heads (grouped
+    queries), their gradients summing over the query heads that share them.
+    """
+    q = np.asarray(p.q, dtype=np.float64)
+    k = np.asarray(p.k, dtype=np.float64)
+    v = np.asarray(p.v, dtype=np.float64)
+    do = np.asarray(dout, dtype=np.float64)
+    T, H, D = q.shape
+    Hk = k.shape[1]
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(len(p.seq_len)):
+        s0, L = int(p.seq_start[b]), int(p.seq_len[b])
+        mask = allowed_matrix(L, p.n_ring, p.layout, p.causal, p.passes)
+        for h in range(H):
+            hk = kv_head(h, H, Hk)
+            Q, K, V = q[s0:s0 + L, h], k[s0:s0 + L, hk], v[s0:s0 + L, hk]
+            dO = do[s0:s0 + L, h]
+            s = np.where(mask, p.scale * (Q @ K.T), -np.inf)
+            m = s.max(axis=1, keepdims=True)
+            m = np.where(np.isfinite(m), m, 0.0)
+            e = np.exp(s - m)
+            P = e / e.sum(axis=1, keepdims=True)
+            O = P @ V
+            dP = dO @ V.T
+            Dd = (dO * O).sum(axis=1, keepdims=True)
+            dS = P * (dP - Dd)
+            dq[s0:s0 + L, h] = p.scale * (dS @ K)
+            dk[s0:s0 + L, hk] += p.scale * (dS.T @ Q)
+            dv[s0:s0 + L, hk] += P.T @ dO
+    return dq, dk, dv
+
+
 # --------------------------------------------------------------------------
 # Helpers for tests and the CPU baseline
 # --------------------------------------------------------------------------
@@ -345,7 +393,8 @@ def row_flops(p: Problem, seq, head, row) -> float:
 
 
 __all__ = [
-    "CONTIGUOUS", "STRIPED", "Problem", "allowed", "allowed_matrix", "block_rows",
+    "CONTIGUOUS", "STRIPED", "Problem", "allowed", "allowed_matrix", "attention_backward",
+    "block_rows",
     "attention_full", "attention_rows", "blas_threads", "masked_attention",
     "merge", "ring_block", "ring_step", "row_flops", "striped_block_sizes", "timed_rows",
     "kv_head", "token_pos", "unmasked_pairs",

@@ -237,6 +237,48 @@ def test_grouped_query_zero_queries_give_group_means():
 
 
 # ----------------------------------------------------------------------------
+# Backward: gradients against torch autograd (fp64)
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("layout,causal,P,H,Hkv", [(0, True, 4, 2, 2), (1, True, 2, 2, 2),
+                                                   (0, False, 3, 4, 2), (1, False, 4, 3, 1)])
+def test_backward_matches_torch_autograd(layout, causal, P, H, Hkv):
+    L, N, D = 20, 4, 6
+    g = torch.Generator().manual_seed(31)
+    q = torch.randn(L, H, D, generator=g, dtype=torch.float64, requires_grad=True)
+    k = torch.randn(L, Hkv, D, generator=g, dtype=torch.float64, requires_grad=True)
+    v = torch.randn(L, Hkv, D, generator=g, dtype=torch.float64, requires_grad=True)
+    do = torch.randn(L, H, D, generator=g, dtype=torch.float64)
+    scale = 0.43
+    mask = torch.from_numpy(explicit_mask(L, N, layout, causal, P))
+    o = torch.nn.functional.scaled_dot_product_attention(
+        q.permute(1, 0, 2)[None], k.permute(1, 0, 2)[None], v.permute(1, 0, 2)[None],
+        attn_mask=mask[None, None], scale=scale, enable_gqa=True)[0].permute(1, 0, 2)
+    (o * do).sum().backward()
+    p = problem(q.detach().numpy(), k.detach().numpy(), v.detach().numpy(), N, layout, causal,
+                P, scale)
+    dq, dk, dv = oracle.attention_backward(p, do.numpy())
+    assert np.abs(dq - q.grad.numpy()).max() < TIGHT
+    assert np.abs(dk - k.grad.numpy()).max() < TIGHT
+    assert np.abs(dv - v.grad.numpy()).max() < TIGHT
+
+
+def test_backward_of_varlen_equals_each_sequence_alone():
+    rng = np.random.default_rng(33)
+    lens = [7, 12, 5]
+    T, H, D, N = sum(lens), 2, 3, 3
+    q, k, v, do = (rng.standard_normal((T, H, D)) for _ in range(4))
+    starts = np.concatenate([[0], np.cumsum(lens)[:-1]])
+    p = problem(q, k, v, N, 0, True, N, 0.7, starts=starts, lens=lens)
+    grads = oracle.attention_backward(p, do)
+    for s0, L in zip(starts, lens):
+        sl = slice(s0, s0 + L)
+        one = problem(q[sl], k[sl], v[sl], N, 0, True, N, 0.7)
+        for g_all, g_one in zip(grads, oracle.attention_backward(one, do[sl])):
+            assert np.array_equal(g_all[sl], g_one)
+
+
+# ----------------------------------------------------------------------------
 # Key/value-outer ring step
 # ----------------------------------------------------------------------------
 

@@ -330,6 +330,47 @@ def measure_ring_steps(steps, warmup, dist, dev, peaks):
             "kernel": "fwd_tc step mode (tcgen05)"}
 
 
+BWD_WORKLOAD = dict(batch=1, heads=8, seqlen=8192, d_head=128, causal=True, n_ring=8)
+# CUDA-core fp32 peak for the backward kernels (plain FMA arithmetic): 148
+# SMs x 128 fp32 lanes x 2 FLOP per FMA x 1.965 GHz
+CUDA_CORE_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def measure_backward(steps, warmup, dist, dev):
+    """Backward (ring_attn_bwd) of a bf16 causal workload: FLOPs counted as
+    10 * d_head per allowed (query, key) pair (recomputed scores, dP, dV, dQ,
+    dK: 2.5 times the forward's count)."""
+    import blockwise_exact_attention_attn_b200 as ra
+    c = BWD_WORKLOAD
+    B, H, S, D, N = c["batch"], c["heads"], c["seqlen"], c["d_head"], c["n_ring"]
+    g = torch.Generator(device=dev).manual_seed(8 + 1000 * dist.rank)
+    q, k, v, do = (torch.randn(B, S, H, D, generator=g, device=dev).to(torch.bfloat16)
+                   for _ in range(4))
+    out = torch.empty_like(q)
+    lse = torch.empty(B, H, S, device=dev)
+    scale = 1.0 / math.sqrt(D)
+    ra.ring_attn_fwd(q, k, v, out, lse, B, H, S, D, N, 0, c["causal"], scale, N)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def step():
+        ra.ring_attn_bwd(q, k, v, out, lse, do, dq, dk, dv, B, H, H, S, D, N, 0, c["causal"],
+                         scale, N)
+
+    from blockwise_exact_attention_attn_b200.flops import forward_flops
+    flops = 2.5 * forward_flops([S] * B, H, D, N, 0, c["causal"], N)
+    ms = time_steps(step, steps, warmup, dist, dev, graph=True)
+    if ra.ring_attn_status() != ra.RA_OK:
+        raise RuntimeError("backward: device status not OK")
+    per = ms / steps
+    tflops = flops / (per * 1e-3) / 1e12
+    return {"workload": f"bf16_b{B}_h{H}_s{S}_d{D}_causal_n{N} backward (dq, dk, dv)",
+            "ms_per_step": per, "tflops_per_gpu": tflops, "tflops": tflops * dist.world,
+            "flops_per_step": flops,
+            "roofline": {"bound": "alu", "achieved": tflops, "peak": CUDA_CORE_FP32_TFLOPS,
+                         "unit": "TFLOP/s", "frac": tflops / CUDA_CORE_FP32_TFLOPS},
+            "kernel": "bwd_dq + bwd_dkdv (CUDA cores, fp32 arithmetic)"}
+
+
 def measure_merge(steps, warmup, dist, dev, peaks):
     """(O, lse) merge on fp32 partials shaped like the headline output."""
     import blockwise_exact_attention_attn_b200 as ra
@@ -501,13 +542,21 @@ def run_ours(args, dist):
             if name == args.workload:
                 continue
             try:
-                r, *_ = measure_workload(name, max(3, min(args.steps, 10)), 3, dist, dev, peaks)
+                with ClockSampler(dist.local) as ck:
+                    r, *_ = measure_workload(name, max(3, min(args.steps, 10)), 3, dist, dev,
+                                             peaks)
+                r["clocks"] = ck.summary()   # long causal runs may meet the power cap
                 extras.append(r)
             except Exception as e:  # report, never hide
                 extras.append({"workload": name, "error": str(e)})
     merge = measure_merge(args.steps, args.warmup, dist, dev, peaks)
     ring_steps = None
+    backward = None
     if not args.no_extras:
+        try:
+            backward = measure_backward(max(3, min(args.steps, 5)), 2, dist, dev)
+        except Exception as e:  # report, never hide
+            backward = {"workload": "backward", "error": str(e)}
         try:
             ring_steps = measure_ring_steps(max(3, min(args.steps, 10)), 3, dist, dev, peaks)
         except Exception as e:  # report, never hide
@@ -555,6 +604,7 @@ def run_ours(args, dist):
         "e2e": e2e,
         "merge": merge,
         "ring_steps": ring_steps,
+        "backward": backward,
         "workloads": extras,
         "cpu_baseline": cpu,
     }

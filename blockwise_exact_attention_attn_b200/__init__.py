@@ -19,6 +19,7 @@ from ._binding import (  # noqa: F401
     RingAttnError,
     library_path,
     load_library,
+    ring_attn_bwd,
     ring_attn_func,
     ring_attn_fwd,
     ring_attn_fwd_noalloc,

@@ -14,6 +14,8 @@
 namespace ra {
 cudaError_t launch_fwd_tc(const FwdParams& p, int fmt, cudaStream_t stream);
 cudaError_t launch_fwd_simt(const FwdParams& p, int dtype, cudaStream_t stream);
+cudaError_t launch_bwd_simt(const FwdParams& f, const void* o, const void* dout, void* dq,
+                            void* dk, void* dv, int dtype, cudaStream_t stream);
 cudaError_t launch_merge(void* out_a, float* lse_a, const void* out_b, const float* lse_b,
                          int batch, int heads, int seqlen, int d_head, int dtype, int num_sms,
                          cudaStream_t stream);
@@ -237,6 +239,34 @@ ra_status ring_attn_fwd_step(const void* q, const void* k, const void* v, float*
   p.lse_head_stride = rows;
   p.order = 0;
   return run_fwd(p, dtype, stream, false);
+}
+
+ra_status ring_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                        const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                        int batch, int heads, int heads_kv, int seqlen, int d_head,
+                        int n_ring_blocks, int layout, int causal, float softmax_scale,
+                        int max_ring_passes, const int32_t* cu_seqlens, int dtype,
+                        void* stream) {
+  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv) return RA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) ||
+      !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return RA_ERR_INVALID;
+  ra_status st = validate_fwd(batch, heads, heads_kv, seqlen, d_head, n_ring_blocks, layout,
+                              causal, softmax_scale, max_ring_passes, cu_seqlens, dtype);
+  if (st != RA_OK) return st;
+  ra::FwdParams p = make_params(q, k, v, (int64_t)heads * d_head, heads_kv,
+                                (int64_t)heads_kv * d_head, nullptr, const_cast<float*>(lse),
+                                batch, heads, seqlen, d_head, n_ring_blocks, layout, causal,
+                                softmax_scale, max_ring_passes, cu_seqlens);
+  int* status = nullptr;
+  st = device_state(&status, nullptr);
+  if (st != RA_OK) return st;
+  p.status = status;
+  cudaError_t e = ra::launch_bwd_simt(p, out, dout, dq, dk, dv,
+                                      dtype == RA_F32 ? 0 : (dtype == RA_BF16 ? 1 : 2),
+                                      reinterpret_cast<cudaStream_t>(stream));
+  if (e == cudaErrorInvalidValue) return RA_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
 ra_status ring_attn_gqa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,

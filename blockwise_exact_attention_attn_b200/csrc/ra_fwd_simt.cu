@@ -20,6 +20,7 @@
 #include <cuda_runtime.h>
 
 #include "ra_common.cuh"
+#include "ra_convert.cuh"
 #include "ra_params.h"
 #include "ra_sched.h"
 #include "ra_work.cuh"
@@ -28,32 +29,6 @@ namespace ra {
 
 constexpr int kSimtThreads = 128;
 constexpr int kSimtBN = 64;
-
-template <typename T>
-__device__ __forceinline__ float to_f32(T x);
-template <>
-__device__ __forceinline__ float to_f32<float>(float x) { return x; }
-template <>
-__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
-  return __bfloat162float(x);
-}
-template <>
-__device__ __forceinline__ float to_f32<__half>(__half x) {
-  return __half2float(x);
-}
-
-template <typename T>
-__device__ __forceinline__ T from_f32(float x);
-template <>
-__device__ __forceinline__ float from_f32<float>(float x) { return x; }
-template <>
-__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
-  return __float2bfloat16_rn(x);
-}
-template <>
-__device__ __forceinline__ __half from_f32<__half>(float x) {
-  return __float2half_rn(x);
-}
 
 // Thread layout: 8 threads serve one query row, 16 rows per CTA.  The row's
 // dimensions are split over TPRD = D / min(D, 32) threads and its keys over

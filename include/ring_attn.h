@@ -197,6 +197,36 @@ ra_status ring_attn_fwd_step(const void* q, const void* k, const void* v,
                              int dtype, void* stream);
 
 /*
+ * ring_attn_bwd -- gradients of the forward: dq, dk, dv of sum(dout * out)
+ * for out = ring_attn_fwd (or ring_attn_gqa_fwd) of q, k, v.
+ *
+ * Source: issue thread "A ring attention with flash attention kernel
+ * implementation": the backward is the part an implementation got wrong,
+ * and the returned lse is what the blockwise method keeps.  The gradients
+ * are plain calculus on out_i = sum_j P_ij v_j, P_ij = exp(scale q_i.k_j -
+ * lse_i) over the allowed keys: dV = P^T dout, dS = P (dP - D) with dP =
+ * dout v^T and D_i = dout_i . out_i, dQ = scale dS K, dK = scale dS^T Q.
+ * P is recomputed from the forward's lse.  Computed on CUDA cores in fp32
+ * arithmetic (two kernels: query rows for dq, key rows for dk/dv).
+ *
+ *  q, k, v, out, lse  as passed to / returned by the forward (k, v with
+ *            heads_kv heads; heads_kv == heads for ring_attn_fwd).
+ *  dout      dtype, shape of out.
+ *  dq        dtype, shape of q; written.
+ *  dk, dv    dtype, shape of k / v; written (summed over the query heads
+ *            that share a key/value head).
+ * Other arguments as ring_attn_gqa_fwd; d_head in {16, 32, 64, 128} for
+ * every dtype.  Errors as ring_attn_gqa_fwd.
+ */
+ra_status ring_attn_bwd(const void* q, const void* k, const void* v,
+                        const void* out, const float* lse, const void* dout,
+                        void* dq, void* dk, void* dv, int batch, int heads,
+                        int heads_kv, int seqlen, int d_head,
+                        int n_ring_blocks, int layout, int causal,
+                        float softmax_scale, int max_ring_passes,
+                        const int32_t* cu_seqlens, int dtype, void* stream);
+
+/*
  * ring_attn_qkvpacked_fwd -- same computation, q/k/v packed in one tensor.
  *
  * Source: issue thread "A ring attention with flash attention kernel

@@ -395,9 +395,9 @@ def measure_merge(steps, warmup, dist, dev, peaks):
 
 
 def measure_e2e(w, steps, warmup, dist, dev):
-    """Same metric through the public API from pinned host buffers: the host
-    to device copy of q/k/v and the device to host copy of out/lse are inside
-    the timed region."""
+    """Same metric through the public API from pinned host buffers
+    (ring_attn_func_host): the host to device copy of q/k/v and the device
+    to host copy of out/lse are inside the timed region."""
     import blockwise_exact_attention_attn_b200 as ra
     from blockwise_exact_attention_attn_b200 import inputs as gen
     assert not w.varlen
@@ -408,11 +408,11 @@ def measure_e2e(w, steps, warmup, dist, dev):
     lse_h = torch.empty(w.batch, w.heads, w.seqlen, dtype=torch.float32).pin_memory()
 
     def step():
-        q, k, v = (t.to(dev, non_blocking=True) for t in host)
-        out, lse = ra.ring_attn_func(q, k, v, w.n_ring, w.causal, w.layout, w.softmax_scale,
-                                     w.passes)
-        out_h.copy_(out, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
+        # the host-input call: per sequence, copies in, forward, copies out on
+        # three streams, so one sequence's transfers overlap another's forward
+        ra.ring_attn_func_host(host[0], host[1], host[2], w.n_ring, w.causal, w.layout,
+                               w.softmax_scale, w.passes, out=out_h, lse=lse_h, chunk=1,
+                               device=dev)
 
     n = max(1, min(steps, 10))
     ms = time_steps(step, n, min(warmup, 3), dist, dev)

@@ -21,6 +21,7 @@ from ._binding import (  # noqa: F401
     load_library,
     ring_attn_bwd,
     ring_attn_func,
+    ring_attn_func_host,
     ring_attn_fwd,
     ring_attn_fwd_noalloc,
     ring_attn_fwd_step,

@@ -359,6 +359,80 @@ def ring_attn_func(q, k, v, n_ring_blocks: int, causal: bool = False, layout=CON
     return out, lse
 
 
+def ring_attn_func_host(q, k, v, n_ring_blocks: int, causal: bool = False, layout=CONTIGUOUS,
+                        softmax_scale: Optional[float] = None,
+                        max_ring_passes: Optional[int] = None, out=None, lse=None,
+                        chunk: int = 1, device=None):
+    """ring_attn_func on pinned HOST tensors q, k, v [batch, seqlen, heads,
+    d_head]: returns (out, lse) on the host (pinned).  The batch is processed
+    in chunks of `chunk` sequences on three CUDA streams -- host-to-device
+    copies, the forward, device-to-host copies -- with two device buffers, so
+    the copies of one chunk overlap the forward of another.  Returns after
+    the results are on the host."""
+    import torch
+    B, S, H, D = q.shape
+    Hkv = k.shape[2]
+    if not (q.is_pinned() and k.is_pinned() and v.is_pinned()):
+        raise ValueError("q, k, v must be pinned host tensors")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    if out is None:
+        out = torch.empty(B, S, H, D, dtype=q.dtype).pin_memory()
+    if lse is None:
+        lse = torch.empty(B, H, S, dtype=torch.float32).pin_memory()
+    chunk = max(1, min(int(chunk), B))
+    nchunks = (B + chunk - 1) // chunk
+    nbuf = min(2, nchunks)
+    bufs = [dict(q=torch.empty(chunk, S, H, D, dtype=q.dtype, device=dev),
+                 k=torch.empty(chunk, S, Hkv, D, dtype=k.dtype, device=dev),
+                 v=torch.empty(chunk, S, Hkv, D, dtype=v.dtype, device=dev),
+                 out=torch.empty(chunk, S, H, D, dtype=q.dtype, device=dev),
+                 lse=torch.empty(chunk, H, S, dtype=torch.float32, device=dev))
+            for _ in range(nbuf)]
+    s_in, s_run, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    start = torch.cuda.current_stream(dev)
+    for st in (s_in, s_run, s_out):
+        st.wait_stream(start)
+    ran = [None] * nbuf      # forward of the buffer's previous chunk done
+    drained = [None] * nbuf  # its results copied out
+    for c in range(nchunks):
+        b0, b1 = c * chunk, min(B, (c + 1) * chunk)
+        n = b1 - b0
+        bf = bufs[c % nbuf]
+        with torch.cuda.stream(s_in):
+            if ran[c % nbuf] is not None:
+                s_in.wait_event(ran[c % nbuf])
+            for name, src in (("q", q), ("k", k), ("v", v)):
+                bf[name][:n].copy_(src[b0:b1], non_blocking=True)
+            loaded = torch.cuda.Event()
+            loaded.record(s_in)
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(loaded)
+            if drained[c % nbuf] is not None:
+                s_run.wait_event(drained[c % nbuf])
+            qc, kc, vc = bf["q"][:n], bf["k"][:n], bf["v"][:n]
+            oc, lc = bf["out"][:n], bf["lse"][:n]
+            if Hkv == H:
+                ring_attn_fwd(qc, kc, vc, oc, lc, n, H, S, D, n_ring_blocks, layout, causal,
+                              softmax_scale, max_ring_passes, None, None, s_run)
+            else:
+                ring_attn_gqa_fwd(qc, kc, vc, oc, lc, n, H, Hkv, S, D, n_ring_blocks, layout,
+                                  causal, softmax_scale, max_ring_passes, None, None, s_run)
+            done = torch.cuda.Event()
+            done.record(s_run)
+            ran[c % nbuf] = done
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done)
+            out[b0:b1].copy_(oc, non_blocking=True)
+            lse[b0:b1].copy_(lc, non_blocking=True)
+            fin = torch.cuda.Event()
+            fin.record(s_out)
+            drained[c % nbuf] = fin
+    # the caller's stream orders after the last copy out; the host waits for it
+    start.wait_stream(s_out)
+    s_out.synchronize()
+    return out, lse
+
+
 def ring_attn_qkvpacked_func(qkv, n_ring_blocks: int, causal: bool = False,
                              layout=CONTIGUOUS, softmax_scale: Optional[float] = None,
                              max_ring_passes: Optional[int] = None, stream=None):

@@ -44,9 +44,11 @@ struct BwdParams {
 constexpr int kBwdThreads = 128;
 constexpr int kBwdBN = 64;  // keys (dq) or queries (dkdv) per shared-memory tile
 
-template <int D>
+// kMaxDPT: dims per thread at most (the dk/dv kernel keeps four row vectors
+// per thread and uses 16 to stay within its registers)
+template <int D, int kMaxDPT = 32>
 struct BwdShape {
-  static constexpr int DPT = D < 32 ? D : 32;          // dims per thread
+  static constexpr int DPT = D < kMaxDPT ? D : kMaxDPT;  // dims per thread
   static constexpr int TPRD = D / DPT;                 // threads per row (dims)
   static constexpr int LANES = 8 / TPRD;               // key / query lanes per row
   static constexpr int ROWS = kBwdThreads / 8;         // rows per CTA
@@ -146,7 +148,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(const BwdParams bp)
       dp = row_sum<TPRD>(dp);
       bool ok = valid && c < nk;
       if (ok && c0 == CLS_PARTIAL) ok = allowed(g, sq, rq, tq, k0 + c);
-      const float P = ok ? exp2f(fmaf(s, p.scale_log2, -lse2)) : 0.f;
+      const float P = ok ? ex2_approx(fmaf(s, p.scale_log2, -lse2)) : 0.f;
       const float ds = P * (dp - Drow);
 #pragma unroll
       for (int d = 0; d < DPT; ++d) dq[d] = fmaf(ds, kr[d], dq[d]);
@@ -166,7 +168,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(const BwdParams bp)
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const BwdParams bp) {
-  using Sh = BwdShape<D>;
+  using Sh = BwdShape<D, 16>;
   constexpr int DPT = Sh::DPT, TPRD = Sh::TPRD, LANES = Sh::LANES, ROWS = Sh::ROWS;
   constexpr int PER = Sh::PER, BQ = kBwdBN, ST = Sh::ST;
   const FwdParams& p = bp.f;  // heads = key/value heads here (work decode)
@@ -252,7 +254,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const BwdParams b
           const int ri = block_of(g, i);
           ok = allowed(g, i, ri, token_of(g, i, ri), sk);
         }
-        const float P = ok ? exp2f(fmaf(s, p.scale_log2, -lse_s[c])) : 0.f;
+        const float P = ok ? ex2_approx(fmaf(s, p.scale_log2, -lse_s[c])) : 0.f;
         const float ds = P * (dp - D_s[c]);
 #pragma unroll
         for (int d = 0; d < DPT; ++d) {
@@ -285,6 +287,8 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const BwdParams b
 template <typename T, int D>
 static cudaError_t launch_bwd_t(const BwdParams& bp, cudaStream_t stream) {
   using Sh = BwdShape<D>;
+  using ShK = BwdShape<D, 16>;
+  static_assert(Sh::ROWS == ShK::ROWS && Sh::ST == ShK::ST, "shared tile shapes");
   // dq: work items over (sequence, query head, 16 query rows)
   BwdParams pq = bp;
   pq.f.n_qranges = (bp.f.seqlen + Sh::ROWS - 1) / Sh::ROWS;

@@ -151,16 +151,6 @@ __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64
       : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem desc].
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                        uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
 
 // Arrive on `bar` once every tcgen05.mma issued so far by this thread is done.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -225,15 +215,6 @@ __host__ __device__ constexpr uint32_t idesc_f16kind_f32(int M, int N, int b_mn_
       "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])            \
       : "memory")
 
-#define RA_TMEM_ST16(taddr, r)                                                          \
-  asm volatile(                                                                         \
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "                                   \
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),         \
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),     \
-      "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),  \
-      "r"(r[14]), "r"(r[15])                                                            \
-      : "memory")
-
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -294,22 +275,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
-}
-
-// 2^x on the FMA and integer pipes, for x <= 126: x = j + f with j =
-// round(x) (the 1.5 * 2^23 addition leaves j in the low mantissa bits) and
-// |f| <= 1/2; 2^f from a cubic with constant term exactly 1, fitted to the
-// relative error of 2^f on [-1/2, 1/2] (Lawson-weighted least squares; max
-// relative error 1.02e-4 in fp32 Horner form); j is added to the exponent
-// field.  x <= -127 (and -inf) gives exactly +0; x = 0 gives exactly 1.
-__device__ __forceinline__ float exp2_poly3(float x) {
-  x = fmaxf(x, -127.0f);
-  const float t = __fadd_rn(x, 12582912.0f);
-  const float f = __fsub_rn(x, __fsub_rn(t, 12582912.0f));
-  const float p = fmaf(fmaf(fmaf(0.05500892922282219f, f, 0.2422109693288803f), f,
-                            0.6932829022407532f),
-                       f, 1.0f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

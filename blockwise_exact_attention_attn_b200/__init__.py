@@ -32,6 +32,7 @@ from ._binding import (  # noqa: F401
     ring_attn_qkvpacked_func,
     ring_attn_schedule,
     ring_attn_status,
+    ring_attn_test_withhold_q,
     ring_attn_status_string,
     ring_attn_varlen_qkvpacked_func,
 )

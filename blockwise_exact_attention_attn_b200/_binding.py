@@ -35,6 +35,7 @@ EXPORTS = (
     "ring_attn_status",
     "ring_attn_status_string",
     "ring_attn_schedule",
+    "ring_attn_test_withhold_q",
 )
 
 
@@ -95,6 +96,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.ring_attn_schedule.argtypes = [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                            _c_int, _c_vp, _c_vp, _c_vp, _c_i64]
         lib.ring_attn_schedule.restype = _c_i64
+        lib.ring_attn_test_withhold_q.argtypes = [_c_int]
+        lib.ring_attn_test_withhold_q.restype = _c_int
         _lib = lib
         return lib
 
@@ -309,6 +312,13 @@ def ring_attn_merge(out_a, lse_a, out_b, lse_b, batch: int, heads: int, seqlen: 
 def ring_attn_status(stream=None) -> int:
     """Synchronize the stream; return and clear the device status word."""
     return int(load_library().ring_attn_status(_stream(stream)))
+
+
+def ring_attn_test_withhold_q(on: bool) -> bool:
+    """Failure-detection test hook: while on, tensor-core forward launches load
+    no query tile, so their bounded wait expires and RA_ERR_TIMEOUT is latched.
+    Returns the previous setting."""
+    return bool(load_library().ring_attn_test_withhold_q(1 if on else 0))
 
 
 def ring_attn_schedule(seqlen: int, n_ring_blocks: int, layout=CONTIGUOUS,

@@ -3,6 +3,7 @@
 // choice of kernel (tensor-core kernel for bf16, CUDA-core kernel for fp32).
 #include <cmath>
 #include <cstdint>
+#include <atomic>
 #include <mutex>
 
 #include <cuda_runtime.h>
@@ -33,6 +34,8 @@ std::mutex g_mu;
 int* g_status[kMaxDevices] = {nullptr};
 int g_num_sms[kMaxDevices] = {0};
 unsigned g_next_slot[kMaxDevices] = {0};
+// Failure-detection test hook, read by every forward call (ring_attn_test_withhold_q).
+std::atomic<int> g_withhold_q{0};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -140,6 +143,7 @@ ra::FwdParams make_params(const void* q, const void* k, const void* v, int64_t t
   p.step = 0;
   p.q_block = p.kv_block = p.step_rows = 0;
   p.accumulate = 0;
+  p.withhold_q = g_withhold_q.load(std::memory_order_relaxed);
   return p;
 }
 
@@ -357,6 +361,10 @@ ra_status ring_attn_status(void* stream) {
     return RA_ERR_CUDA;
   if (v != 0 && cudaMemset(status, 0, sizeof(int)) != cudaSuccess) return RA_ERR_CUDA;
   return static_cast<ra_status>(v);
+}
+
+int ring_attn_test_withhold_q(int on) {
+  return g_withhold_q.exchange(on ? 1 : 0);
 }
 
 const char* ring_attn_status_string(int status) {

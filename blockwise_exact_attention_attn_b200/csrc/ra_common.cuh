@@ -15,7 +15,9 @@ namespace ra {
 enum : int { ST_OK = 0, ST_INVALID = 1, ST_UNSUPPORTED = 2, ST_CUDA = 3, ST_TIMEOUT = 4 };
 
 // Bound on every in-kernel wait, in SM clock cycles (~1 s at 2 GHz).  No wait
-// of a healthy launch comes close: the longest is one K/V tile or one MMA.
+// of a healthy launch comes close: the longest, the schedule builder waiting
+// for the previous work item to start, lasts about one work item
+// (milliseconds).
 constexpr long long kWaitCycles = 2000000000LL;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

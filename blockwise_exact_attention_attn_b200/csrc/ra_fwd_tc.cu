@@ -448,7 +448,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tma_prefetch_desc(&maps.k);
       tma_prefetch_desc(&maps.v);
     }
-    int n = 0, k = 0;
+    int n = 0, k = 0, nq = 0;  // K/V tiles, items and query loads issued
     bool ok = true;
     auto load = [&](const CUtensorMap* map, int h, int row) -> bool {
       const int slot = n % KVS;
@@ -477,7 +477,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int hk = it.h / p.kv_group;  // key/value head of this query head
         if (ok && e >= 0) ok = load(&maps.k, hk, it.base + entry_tile(e) * kTcBN);
         if (ok && k > 0) ok = mbar_wait(&ctrl->q_free, (k - 1) & 1, abort_flag);
-        if (ok) {
+        if (ok && !p.withhold_q) {
           uint8_t* qs = smem + C::kQOff;
           const int q0 = it.qr * kRows;
           mbar_arrive_expect_tx(&ctrl->q_full, kTcQT * C::kTileBytes);
@@ -485,6 +485,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int pn = 0; pn < C::kPanels; ++pn)
               tma_load_3d(qs + i * C::kTileBytes + pn * C::kPanelBytes, &maps.q,
                           &ctrl->q_full, pn * 64, it.h, it.base + q0 + i * kTcBM);
+          ++nq;
         }
         int prev = e;
         while (ok && prev >= 0) {
@@ -504,7 +505,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // let the copies already issued land before the CTA can exit
       for (int u = (n > KVS ? n - KVS : 0); u < n; ++u)
         mbar_wait(&ctrl->kv_full[u % KVS], (u / KVS) & 1, nullptr);
-      if (k > 0) mbar_wait(&ctrl->q_full, (k - 1) & 1, nullptr);
+      if (nq > 0) mbar_wait(&ctrl->q_full, (nq - 1) & 1, nullptr);
     }
     __syncwarp();
    } else if (warp == kTcMmaWarp || kTcIssuers == 2) {

@@ -45,6 +45,10 @@ struct FwdParams {
   int step;                 // 0: whole-sequence call
   int q_block, kv_block, step_rows;
   int accumulate;
+  // Failure-detection test hook (0 in normal use): the tensor-core kernel's
+  // producer issues no query-tile load, so the MMA issuers' bounded wait for
+  // Q expires and the launch unwinds with ST_TIMEOUT.
+  int withhold_q;
 };
 
 // Query rows per dense sequence held by q/out: the whole sequence, or one

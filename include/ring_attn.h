@@ -330,6 +330,21 @@ ra_status ring_attn_fwd_noalloc(const void* q, const void* k, const void* v,
  */
 ra_status ring_attn_status(void* stream);
 
+/*
+ * ring_attn_test_withhold_q -- failure-detection test hook; leave it off (0)
+ * in normal use.  While on, every tensor-core forward launch made by this
+ * process (bf16/fp16 ring_attn_fwd, _gqa_fwd, _fwd_step, _qkvpacked_fwd,
+ * _fwd_noalloc) loads no query tile: the MMA warps' bounded wait for Q gives
+ * up after about one second, every role of the CTA unwinds (copies and MMAs
+ * already issued are drained, tensor memory is freed) and RA_ERR_TIMEOUT is
+ * latched in the status word; the output is left unspecified.  The device
+ * context stays usable.  Host-only: the setting is read when a call builds
+ * its launch parameters, so it can be toggled without a GPU.
+ *  on  nonzero = on, 0 = off.
+ * Returns the previous setting (0 or 1).  Never fails.
+ */
+int ring_attn_test_withhold_q(int on);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* ring_attn_status_string(int status);
 

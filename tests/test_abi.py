@@ -41,6 +41,15 @@ def test_status_strings(lib):
     assert lib.ring_attn_status_string(99).decode() == "RA_ERR_UNKNOWN"
 
 
+def test_withhold_hook_toggles_on_the_host(lib):
+    # host-only setting: returns the previous value, never touches CUDA
+    assert lib.ring_attn_test_withhold_q(1) == 0
+    assert lib.ring_attn_test_withhold_q(7) == 1
+    assert lib.ring_attn_test_withhold_q(0) == 1
+    assert lib.ring_attn_test_withhold_q(0) == 0
+    assert ra.ring_attn_test_withhold_q(False) is False
+
+
 def fwd(lib, **over):
     a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, batch=1, heads=2, seqlen=256, d_head=128,
              n=4, layout=0, causal=1, scale=0.1, passes=4, cu=None, dtype=1, stream=None)

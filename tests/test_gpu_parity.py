@@ -178,6 +178,32 @@ def test_varlen_sequence_alone_is_bitwise_identical():
         assert torch.equal(lse[:, s0:s0 + L], l1)
 
 
+@pytest.mark.parametrize("impl", ["tc", "simt"])
+def test_varlen_empty_sequences(impl):
+    """Zero-length sequences (allowed: cu_seqlens only has to be
+    non-decreasing) at the start, in the middle and at the end contribute no
+    work: every row matches the oracle, and the result is bit for bit the
+    one of the same tokens without the empty sequences."""
+    lens = [0, 300, 0, 0, 129, 1, 0]
+    cu = torch.zeros(len(lens) + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(torch.tensor(lens), 0)
+    T = int(cu[-1])
+    g = torch.Generator().manual_seed(12)
+    qkv = torch.randn(T, 3, 2, 128, generator=g).to(torch.bfloat16)
+    mk = lambda n, c: (gen.Workload("vl_empty", "bf16", n, 2, T, 128, True, 4, 1, 3, seed=12,
+                                    varlen=True, packed=impl == "tc", n_seqs=n),
+                       dict(qkv=qkv, cu_seqlens=c, q=qkv[:, 0], k=qkv[:, 1], v=qkv[:, 2]))
+    w, inp = mk(len(lens), cu)
+    out, lse = run_gpu(w, inp, impl=impl)
+    check(w, *compare_full(w, inp, out, lse))
+    kept = [L for L in lens if L > 0]
+    cu2 = torch.zeros(len(kept) + 1, dtype=torch.int32)
+    cu2[1:] = torch.cumsum(torch.tensor(kept), 0)
+    w2, inp2 = mk(len(kept), cu2)
+    out2, lse2 = run_gpu(w2, inp2, impl=impl)
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
+
+
 def test_rows_outside_the_sequences_stay_untouched():
     dev = torch.device("cuda", 0)
     lens = [300, 200]

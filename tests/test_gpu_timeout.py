@@ -12,9 +12,11 @@ oracle.
 
 import time
 
+import numpy as np
 import pytest
 import torch
 
+import oracle
 import blockwise_exact_attention_attn_b200 as ra
 from blockwise_exact_attention_attn_b200 import inputs as gen
 from gpu_util import TOL, compare_full, run_gpu
@@ -60,3 +62,57 @@ def test_expired_wait_latches_timeout_and_context_recovers(case):
     err_o, err_l = compare_full(w, inp, out2, lse2)
     to, tl = TOL[w.dtype]
     assert err_o <= to and err_l <= tl, (err_o, err_l)
+
+
+def test_cuda_core_kernel_ignores_the_hook():
+    # fp32 runs on the CUDA-core kernel, which has no query-load pipeline:
+    # the hook changes nothing there
+    w = gen.Workload("timeout_f32", "f32", 1, 2, 256, 64, True, 4, 0, 4, seed=31)
+    inp = gen.make_inputs(w)
+    prev = ra.ring_attn_test_withhold_q(True)
+    try:
+        out, lse = run_gpu(w, inp)  # asserts RA_OK
+    finally:
+        ra.ring_attn_test_withhold_q(prev)
+    err_o, err_l = compare_full(w, inp, out, lse)
+    to, tl = TOL[w.dtype]
+    assert err_o <= to and err_l <= tl, (err_o, err_l)
+
+
+def test_ring_step_unwinds_from_a_loaded_state():
+    """An accumulating ring step loads the running state into tensor memory
+    before its first wait; with the hook on it must unwind the same way, and
+    a whole ring of steps with the hook off must then reach full attention."""
+    dev = torch.device("cuda", 0)
+    B, H, L, N, D, layout = 1, 2, 1024, 4, 128, 0
+    scale = 1.0 / np.sqrt(D)
+    g = torch.Generator().manual_seed(41)
+    q, k, v = (torch.randn(B, L, H, D, generator=g).to(torch.bfloat16) for _ in range(3))
+    blk = [[t[:, oracle.block_rows(L, N, layout, r)].contiguous().to(dev) for r in range(N)]
+           for t in (q, k, v)]
+    b = L // N
+    i = 2
+    out = torch.zeros(B, b, H, D, device=dev)
+    lse = torch.zeros(B, H, b, device=dev)  # a running state: one unit of weight, O = 0
+    prev = ra.ring_attn_test_withhold_q(True)
+    try:
+        ra.ring_attn_fwd_step(blk[0][i], blk[1][1], blk[2][1], out, lse, B, H, L, D, N, i, 1,
+                              True, layout, True, scale)
+        st = ra.ring_attn_status()
+    finally:
+        ra.ring_attn_test_withhold_q(prev)
+    assert st == ra.RA_ERR_TIMEOUT, ra.ring_attn_status_string(st)
+
+    for s in range(N):
+        j = (i - s) % N
+        ra.ring_attn_fwd_step(blk[0][i], blk[1][j], blk[2][j], out, lse, B, H, L, D, N, i, j,
+                              s > 0, layout, True, scale)
+    assert ra.ring_attn_status() == ra.RA_OK
+    p = oracle.Problem(q=q[0].float().numpy(), k=k[0].float().numpy(), v=v[0].float().numpy(),
+                       seq_start=np.array([0]), seq_len=np.array([L]), n_ring=N, layout=layout,
+                       causal=True, passes=N, scale=scale)
+    full_o, full_l = oracle.attention_full(p)
+    rows = oracle.block_rows(L, N, layout, i)
+    to, tl = TOL["bf16"]
+    assert float(np.abs(out[0].cpu().numpy() - full_o[rows]).max()) <= to
+    assert float(np.abs(lse[0].cpu().numpy() - full_l[:, rows]).max()) <= tl

@@ -562,6 +562,24 @@ def test_varlen_equals_each_sequence_alone():
         assert np.array_equal(o[sl], o1) and np.array_equal(lse[:, sl], l1)
 
 
+def test_zero_length_sequences_contribute_nothing():
+    # cu_seqlens only has to be non-decreasing: an empty sequence owns no row
+    # and no key, so the others come out exactly as without it (both layouts,
+    # a pass cap below N)
+    rng = np.random.default_rng(16)
+    lens = [0, 6, 0, 0, 11, 0]
+    starts = np.concatenate([[0], np.cumsum(lens)[:-1]])
+    kept = [L for L in lens if L > 0]
+    kstarts = np.concatenate([[0], np.cumsum(kept)[:-1]])
+    T, H, D, N = sum(lens), 2, 4, 3
+    q, k, v = (rng.standard_normal((T, H, D)) for _ in range(3))
+    for layout in (oracle.CONTIGUOUS, oracle.STRIPED):
+        o, lse = oracle.attention_full(problem(q, k, v, N, layout, True, 2, 0.5, starts, lens))
+        o2, l2 = oracle.attention_full(problem(q, k, v, N, layout, True, 2, 0.5, kstarts, kept))
+        assert np.array_equal(o, o2) and np.array_equal(lse, l2)
+        assert np.isfinite(o).all() and np.isfinite(lse).all()
+
+
 def test_row_sample_equals_full():
     rng = np.random.default_rng(8)
     T, H, D, N = 50, 3, 4, 5

@@ -523,6 +523,18 @@ def oracle_sample(w, budget_s: float, rows_cap: int = 1 << 20):
     return fl / t / 1e12, t, n, oracle.blas_threads()
 
 
+def full_config_flops(w) -> float:
+    """Unmasked FLOPs of the whole workload (varlen lengths drawn as the
+    input recipe draws them, without the values)."""
+    from blockwise_exact_attention_attn_b200 import inputs as gen
+    if w.varlen:
+        g = torch.Generator().manual_seed(w.seed)
+        lens = gen.varlen_lengths(g, w.n_seqs, w.seqlen, *w.len_range).tolist()
+    else:
+        lens = [w.seqlen] * w.batch
+    return workload_flops(w, lens)
+
+
 def run_reference(args, dist):
     """Reference arm: the fp64 oracle as it stands, on the host cores, on the
     same workload and metric; each step is a bounded row sample."""
@@ -549,7 +561,9 @@ def run_reference(args, dist):
         "config": {"workload": w.name, "sample": f"{rows} random query rows of head 0, "
                    "full key range each, over all steps"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": f"~{per_step_budget:.1f} s of fp64 rows per step"},
+                         "sample": f"~{per_step_budget:.1f} s of fp64 rows per step",
+                         "extrapolated_full_config_s":
+                             full_config_flops(w) / (value * 1e12) if value > 0 else None},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -632,7 +646,9 @@ def run_ours(args, dist):
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         v, t, n, cores = oracle_sample(w, 15.0)
         cpu = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-               "sample": f"{n} random query rows of head 0 (full key range each), {t:.1f} s"}
+               "sample": f"{n} random query rows of head 0 (full key range each), {t:.1f} s",
+               # the whole workload at the sampled rate (not run)
+               "extrapolated_full_config_s": flops / (v * 1e12) if v > 0 else None}
 
     if dist.rank != 0:
         return

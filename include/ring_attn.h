@@ -107,8 +107,9 @@ typedef enum { RA_F32 = 0, RA_BF16 = 1, RA_F16 = 2 } ra_dtype;
  *  cu_seqlens  NULL for dense, else DEVICE int32[batch + 1] (4-byte aligned),
  *            cu_seqlens[0] = 0, non-decreasing, cu_seqlens[batch] = seqlen.
  *            Sequence b is rows [cu_seqlens[b], cu_seqlens[b+1]); its ring
- *            blocks follow its own length (any length >= 1, no divisibility
- *            requirement).  A negative length or an offset beyond seqlen
+ *            blocks follow its own length (any length >= 0, no divisibility
+ *            requirement; a zero-length sequence owns no row and is
+ *            skipped).  A negative length or an offset beyond seqlen
  *            latches RA_ERR_INVALID in the status word and that sequence's
  *            rows are left unwritten; a wrong cu_seqlens[0] or
  *            cu_seqlens[batch] latches RA_ERR_INVALID too.
@@ -119,7 +120,9 @@ typedef enum { RA_F32 = 0, RA_BF16 = 1, RA_F16 = 2 } ra_dtype;
  * size, seqlen % n_ring_blocks != 0 (dense), max_ring_passes < 1, a
  * non-finite softmax_scale, causal not in {0,1}, an unknown layout/dtype, or
  * a d_head outside {16,32,64,128}; RA_ERR_UNSUPPORTED for a d_head the dtype
- * has no kernel for; RA_ERR_CUDA when a launch fails.
+ * has no kernel for, or for sizes past 32-bit row indices (dense
+ * batch * seqlen, or batch * heads, above 2^31 - 1); RA_ERR_CUDA when a launch
+ * fails.
  */
 ra_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out,
                         float* lse, int batch, int heads, int seqlen,
@@ -280,7 +283,8 @@ ra_status ring_attn_fwd_simt(const void* q, const void* k, const void* v,
  *  d_head        RA_F32: 4, 8, 16, 32, 64 or 128; RA_BF16 and RA_F16: 8, 16,
  *                32, 64, 128 or 256 (a row is 1 to 32 whole 16-byte chunks).
  * Errors: RA_ERR_INVALID for null/misaligned pointers, non-positive sizes,
- * an unsupported d_head or dtype; RA_ERR_CUDA when the launch fails.
+ * an unsupported d_head or dtype; RA_ERR_UNSUPPORTED when batch * seqlen *
+ * heads rows exceed 2^31 - 1; RA_ERR_CUDA when the launch fails.
  */
 ra_status ring_attn_merge(void* out_a, float* lse_a, const void* out_b,
                           const float* lse_b, int batch, int heads, int seqlen,

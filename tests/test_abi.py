@@ -71,6 +71,23 @@ def test_fwd_rejects_invalid_arguments(lib, over):
     assert fwd(lib, **over) == ra.RA_ERR_INVALID
 
 
+@pytest.mark.parametrize("over", [
+    dict(batch=2, seqlen=1 << 30),       # batch * seqlen = 2^31 rows: past 32-bit row indices
+    dict(batch=1 << 16, heads=1 << 15, seqlen=4),   # batch * heads = 2^31
+])
+def test_fwd_refuses_sizes_past_32_bit_indices(lib, over):
+    # maximum sizes: refused on the host before any CUDA call
+    assert fwd(lib, **over) == ra.RA_ERR_UNSUPPORTED
+
+
+def test_merge_refuses_rows_past_32_bit_indices(lib):
+    # batch * seqlen * heads = 2^31 rows
+    assert lib.ring_attn_merge(FAKE, FAKE, FAKE, FAKE, 2, 1 << 10, 1 << 20, 128, 0,
+                               None) == ra.RA_ERR_UNSUPPORTED
+    assert lib.ring_attn_merge(FAKE, FAKE, FAKE, FAKE, 1, 1 << 11, 1 << 20, 128, 0,
+                               None) == ra.RA_ERR_UNSUPPORTED
+
+
 def test_qkvpacked_and_simt_reject_invalid_arguments(lib):
     st = lib.ring_attn_qkvpacked_fwd(None, FAKE, FAKE, 1, 2, 256, 128, 4, 0, 1, 0.1, 4, None, 1,
                                      None)

@@ -94,7 +94,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.ring_attn_status_string.argtypes = [_c_int]
         lib.ring_attn_status_string.restype = ctypes.c_char_p
         lib.ring_attn_schedule.argtypes = [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
-                                           _c_int, _c_vp, _c_vp, _c_vp, _c_i64]
+                                           _c_int, _c_int, _c_vp, _c_vp, _c_vp, _c_i64]
         lib.ring_attn_schedule.restype = _c_i64
         lib.ring_attn_test_withhold_q.argtypes = [_c_int]
         lib.ring_attn_test_withhold_q.restype = _c_int
@@ -323,14 +323,16 @@ def ring_attn_test_withhold_q(on: bool) -> bool:
 
 def ring_attn_schedule(seqlen: int, n_ring_blocks: int, layout=CONTIGUOUS,
                        causal: bool = False, max_ring_passes: Optional[int] = None,
-                       q_tile: int = 128, kv_tile: int = 128):
+                       q_tile: int = 128, kv_tile: int = 128, q_tiles_per_item: int = 1):
     """Visited (q_tile, kv_tile, class) triples of the ring scheduler, as
-    three numpy arrays in visit order (class 1 = FULL, 2 = PARTIAL)."""
+    three numpy arrays in visit order (class 1 = FULL, 2 = PARTIAL).  With
+    q_tiles_per_item = 2, pairs of q-tiles walk one key/value stream, as the
+    tensor-core kernel's work items do."""
     lib = load_library()
     if max_ring_passes is None:
         max_ring_passes = n_ring_blocks
     args = (int(seqlen), int(n_ring_blocks), _layout_code(layout), int(bool(causal)),
-            int(max_ring_passes), int(q_tile), int(kv_tile))
+            int(max_ring_passes), int(q_tile), int(kv_tile), int(q_tiles_per_item))
     n = lib.ring_attn_schedule(*args, None, None, None, 0)
     if n < 0:
         raise RingAttnError("ring_attn_schedule", RA_ERR_INVALID)

@@ -379,27 +379,38 @@ const char* ring_attn_status_string(int status) {
 }
 
 int64_t ring_attn_schedule(int seqlen, int n_ring_blocks, int layout, int causal,
-                           int max_ring_passes, int q_tile, int kv_tile, int32_t* out_q,
-                           int32_t* out_kv, int8_t* out_class, int64_t capacity) {
+                           int max_ring_passes, int q_tile, int kv_tile, int q_tiles_per_item,
+                           int32_t* out_q, int32_t* out_kv, int8_t* out_class,
+                           int64_t capacity) {
   if (seqlen < 1 || n_ring_blocks < 1 || max_ring_passes < 1 || q_tile < 1 || kv_tile < 1)
     return -1;
+  if (q_tiles_per_item != 1 && q_tiles_per_item != 2) return -1;
   if (layout != RA_LAYOUT_CONTIGUOUS && layout != RA_LAYOUT_STRIPED) return -1;
   if (causal != 0 && causal != 1) return -1;
   if (capacity > 0 && (!out_q || !out_kv || !out_class)) return -1;
   const ra::RingGeom g = ra::make_geom(seqlen, n_ring_blocks, layout, causal, max_ring_passes);
   int64_t n = 0;
-  for (int q0 = 0; q0 < seqlen; q0 += q_tile) {
-    const int q1 = q0 + q_tile < seqlen ? q0 + q_tile : seqlen;
+  auto emit = [&](int qt, int kt, int c) {
+    if (n < capacity) {
+      out_q[n] = qt;
+      out_kv[n] = kt;
+      out_class[n] = (int8_t)c;
+    }
+    ++n;
+  };
+  const int64_t item_rows = (int64_t)q_tile * q_tiles_per_item;
+  for (int64_t i0 = 0; i0 < seqlen; i0 += item_rows) {
+    // one work item: query tiles [q0, qm) and [qm, q1), walked together over
+    // one key/value stream as the tensor-core kernel's schedule builder does
+    const int q0 = (int)i0;
+    const int qm = (int)(i0 + q_tile < seqlen ? i0 + q_tile : seqlen);
+    const int q1 = (int)(i0 + item_rows < seqlen ? i0 + item_rows : seqlen);
     ra::TileWalk w;
-    w.init(g, q0, q1, q1, kv_tile);
+    w.init(g, q0, qm, q1, kv_tile);
     int kt, c0, c1;
     while (w.next(&kt, &c0, &c1)) {
-      if (n < capacity) {
-        out_q[n] = q0 / q_tile;
-        out_kv[n] = kt;
-        out_class[n] = (int8_t)c0;
-      }
-      ++n;
+      if (c0 != ra::CLS_EMPTY) emit(q0 / q_tile, kt, c0);
+      if (c1 != ra::CLS_EMPTY && qm < q1) emit(q0 / q_tile + 1, kt, c1);
     }
   }
   return n;

@@ -360,10 +360,17 @@ const char* ring_attn_status_string(int status);
  *   1 = FULL (every query/key pair of the two tiles is allowed, no mask),
  *   2 = PARTIAL (mixed; the element mask is applied).
  * EMPTY pairs (no allowed pair) are not visited and not listed.
- * The classification is exact whenever the two tiles together touch at most
- * 64 (q-block, kv-block) pairs of ring blocks; beyond that a pair that is
+ * The classification is exact whenever the ring-block index ranges the two
+ * tiles span, multiplied, are at most 64 (empty blocks inside a range, which
+ * exist when a sequence is shorter than N, count); beyond that a pair that is
  * really EMPTY or FULL may be listed as PARTIAL (never the reverse).
  *
+ *  q_tiles_per_item  1: each q-tile walks alone.  2: consecutive pairs of
+ *                 q-tiles (the tensor-core kernel's work items of
+ *                 2 * q_tile rows; the last may hold one tile) walk one
+ *                 shared key/value stream, in the ring order of the pair's
+ *                 first row; each tile's visited pairs are listed in stream
+ *                 order, the first tile's entry before the second's.
  *  out_q, out_kv  int32 tile indices; out_class int8.  HOST arrays of
  *                 `capacity` entries (may be NULL when capacity is 0).
  * Returns the total number of visited pairs (which may exceed capacity; only
@@ -371,8 +378,9 @@ const char* ring_attn_status_string(int status);
  */
 int64_t ring_attn_schedule(int seqlen, int n_ring_blocks, int layout,
                            int causal, int max_ring_passes, int q_tile,
-                           int kv_tile, int32_t* out_q, int32_t* out_kv,
-                           int8_t* out_class, int64_t capacity);
+                           int kv_tile, int q_tiles_per_item, int32_t* out_q,
+                           int32_t* out_kv, int8_t* out_class,
+                           int64_t capacity);
 
 #ifdef __cplusplus
 }

@@ -7,6 +7,7 @@ import itertools
 
 import numpy as np
 import pytest
+from hypothesis import given, settings, strategies as st
 
 import oracle
 from blockwise_exact_attention_attn_b200 import ring_attn_schedule
@@ -31,12 +32,14 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("per_item", [1, 2])
 @pytest.mark.parametrize("L,N,tq,tk", CASES)
 @pytest.mark.parametrize("layout", [oracle.CONTIGUOUS, oracle.STRIPED])
 @pytest.mark.parametrize("causal", [False, True])
-def test_schedule_equals_brute_force(L, N, tq, tk, layout, causal):
+def test_schedule_equals_brute_force(L, N, tq, tk, layout, causal, per_item):
+    # per_item 2 is the tensor-core kernel's walk: two q-tiles, one stream
     for P in sorted({1, 2, max(1, N // 2), N}):
-        qt, kt, cl = ring_attn_schedule(L, N, layout, causal, P, tq, tk)
+        qt, kt, cl = ring_attn_schedule(L, N, layout, causal, P, tq, tk, per_item)
         got = {}
         for a, b, c in zip(qt.tolist(), kt.tolist(), cl.tolist()):
             assert (a, b) not in got, "a kv tile was visited twice"
@@ -92,3 +95,45 @@ def test_schedule_rejects_bad_arguments():
         ring_attn_schedule(0, 4)
     with pytest.raises(RingAttnError):
         ring_attn_schedule(128, 0)
+
+
+def block_pairs(blk, L, a, tq, b, tk):
+    """Product of the ring-block index ranges q-tile a and kv-tile b span
+    (stored rows are in block order in both layouts; empty blocks inside a
+    range, which exist when a sequence is shorter than N, count)."""
+    qa, qb = blk[a * tq], blk[min(L, (a + 1) * tq) - 1]
+    ka, kb = blk[b * tk], blk[min(L, (b + 1) * tk) - 1]
+    return (qb - qa + 1) * (kb - ka + 1)
+
+
+@settings(max_examples=300, deadline=None)
+@given(L=st.integers(1, 600), N=st.integers(1, 20), layout=st.sampled_from([0, 1]),
+       causal=st.booleans(), p_extra=st.integers(0, 20),
+       tq=st.sampled_from([16, 32, 64, 128]), tk=st.sampled_from([16, 32, 64, 128]),
+       per_item=st.sampled_from([1, 2]))
+def test_schedule_properties_on_random_geometry(L, N, layout, causal, p_extra, tq, tk,
+                                                per_item):
+    P = 1 + p_extra % (N + 1)          # 1 .. N+1 (values above N clamp to N)
+    qt, kt, cl = ring_attn_schedule(L, N, layout, causal, P, tq, tk, per_item)
+    ref = brute(L, N, layout, causal, P, tq, tk)
+    mask = oracle.allowed_matrix(L, N, layout, causal, P)
+    blk = oracle.ring_block(np.arange(L), L, N, layout)
+    got = {}
+    for a, b, c in zip(qt.tolist(), kt.tolist(), cl.tolist()):
+        assert (a, b) not in got, "a kv tile was visited twice"
+        assert c in (1, 2)
+        got[(a, b)] = c
+    for key in ref:
+        assert key in got, ("non-empty pair skipped", key)
+    for (a, b), c in got.items():
+        sub = mask[a * tq:(a + 1) * tq, b * tk:(b + 1) * tk]
+        if c == 1:
+            assert sub.all(), ("false FULL", a, b)
+        if block_pairs(blk, L, a, tq, b, tk) <= 64:
+            assert ref.get((a, b)) == c, ("inexact class in the exact regime", a, b)
+    # ring order: per q-tile, the step of each visited kv tile (block of its
+    # first key, relative to the block of the item's first row) never falls
+    for a in np.unique(qt):
+        item0 = (a // per_item) * per_item * tq
+        steps = [(blk[item0] - blk[b * tk]) % N for b in kt[qt == a]]
+        assert steps == sorted(steps)

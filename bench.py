@@ -612,8 +612,12 @@ def run_ours(args, dist):
     peak = peaks["bf16_tflops"] if w.dtype == "bf16" else None
     traffic = profiled_traffic(w.name) if w.dtype == "bf16" else None
 
+    # The extra workloads, ring steps and backward are per-GPU figures: they
+    # run at N = 1 only, so a multi-rank run stays short and its line carries
+    # what scaling is computed from (value), plus merge and e2e.
+    run_extras = not args.no_extras and dist.world == 1
     extras = []
-    if not args.no_extras:
+    if run_extras:
         for name in EXTRAS:
             if name == args.workload:
                 continue
@@ -631,7 +635,7 @@ def run_ours(args, dist):
     merge = measure_merge(args.steps, args.warmup, dist, dev, peaks)
     ring_steps = None
     backward = None
-    if not args.no_extras:
+    if run_extras:
         try:
             backward = measure_backward(max(3, min(args.steps, 5)), 2, dist, dev)
         except Exception as e:  # report, never hide

@@ -37,6 +37,23 @@ def device_fold(q, k, v, out, lse, q_block: int, kv_block: int, accumulate: bool
                        accumulate, layout, causal, scale)
 
 
+def check_device_fold(q, softmax_scale: float) -> None:
+    """Raise ValueError when ring_attn_fwd_step would refuse this rank's
+    block: 16-bit inputs, d_head 64 or 128, a block of whole 128-row tiles and
+    a nonzero scale.  Checked before the first exchange, so that every rank
+    (same shapes on all of them) fails before any transfer is in flight."""
+    import torch
+    B, b, H, D = q.shape
+    if q.dtype not in (torch.bfloat16, torch.float16):
+        raise ValueError(f"the device ring step takes bf16 or fp16 inputs, not {q.dtype}")
+    if D not in (64, 128):
+        raise ValueError(f"the device ring step takes d_head 64 or 128, not {D}")
+    if b % 128 != 0:
+        raise ValueError(f"the device ring step needs blocks of whole 128-row tiles, not {b}")
+    if softmax_scale == 0.0:
+        raise ValueError("the device ring step needs a nonzero softmax scale")
+
+
 def ring_attention_forward(q, k, v, *, causal: bool = False, layout: int = CONTIGUOUS,
                            softmax_scale: Optional[float] = None,
                            max_ring_passes: Optional[int] = None, group=None,
@@ -60,6 +77,8 @@ def ring_attention_forward(q, k, v, *, causal: bool = False, layout: int = CONTI
     L = b * N
     P = N if max_ring_passes is None else max(1, min(int(max_ring_passes), N))
     scale = 1.0 / math.sqrt(D) if softmax_scale is None else float(softmax_scale)
+    if fold is device_fold:
+        check_device_fold(q, scale)
     # the running state is fp32 (what the device step keeps); fp64 inputs
     # (host checks) keep it in fp64
     state = torch.float64 if q.dtype == torch.float64 else torch.float32

@@ -93,3 +93,22 @@ def test_ring_across_ranks_equals_full_attention(world, case):
     assert all(p.exitcode == 0 for p in procs)
     err_o, err_l = result.get(timeout=10)
     assert err_o < 1e-12 and err_l < 1e-12
+
+
+@pytest.mark.parametrize("dtype,shape,scale", [
+    (torch.float32, (1, 128, 2, 128), 0.1),      # fp32 has no device ring step
+    (torch.bfloat16, (1, 128, 2, 32), 0.1),      # d_head 32
+    (torch.bfloat16, (1, 100, 2, 128), 0.1),     # block not whole 128-row tiles
+    (torch.bfloat16, (1, 128, 2, 128), 0.0),     # zero scale
+])
+def test_device_fold_arguments_are_refused_before_any_exchange(dtype, shape, scale):
+    # the check needs no process group: every rank refuses before communicating
+    from blockwise_exact_attention_attn_b200.ring import check_device_fold
+    with pytest.raises(ValueError):
+        check_device_fold(torch.zeros(*shape, dtype=dtype), scale)
+
+
+def test_device_fold_arguments_accepted():
+    from blockwise_exact_attention_attn_b200.ring import check_device_fold
+    for dt, D in ((torch.bfloat16, 128), (torch.float16, 64)):
+        check_device_fold(torch.zeros(2, 256, 3, D, dtype=dt), -0.5)

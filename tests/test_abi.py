@@ -149,3 +149,44 @@ def test_binding_refuses_host_tensors():
     lse = torch.zeros(1, 1, 128)
     with pytest.raises(ValueError):
         ra.ring_attn_fwd(x, x, x, x, lse, 1, 1, 128, 64, 1)
+
+
+C_CONSUMER = r"""
+#include <stdio.h>
+#include <string.h>
+#include "ring_attn.h"
+int main(void) {
+  int32_t qt[8], kt[8];
+  int8_t cl[8];
+  int64_t n;
+  if (strcmp(ring_attn_status_string(RA_ERR_TIMEOUT), "RA_ERR_TIMEOUT") != 0) return 1;
+  if (ring_attn_fwd(NULL, NULL, NULL, NULL, NULL, 1, 1, 128, 128, 1, RA_LAYOUT_CONTIGUOUS, 0,
+                    0.1f, 1, NULL, RA_BF16, NULL) != RA_ERR_INVALID)
+    return 2;
+  /* causal, 256 rows, 128-row tiles: (0,0) partial, (1,0) full, (1,1) partial */
+  n = ring_attn_schedule(256, 2, RA_LAYOUT_CONTIGUOUS, 1, 2, 128, 128, 1, qt, kt, cl, 8);
+  if (n != 3 || cl[0] != 2) return 3;
+  if (ring_attn_test_withhold_q(0) != 0) return 4;
+  printf("ok\n");
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    # the boundary from C itself: strict C99 against the header, linked to the
+    # library, host-only calls (no CUDA call is made)
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "consumer.c"
+    src.write_text(C_CONSUMER)
+    exe = tmp_path / "consumer"
+    libdir = os.path.dirname(ra.library_path())
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.dirname(HEADER), str(src), "-L", libdir, "-lringattn",
+                    "-Wl,-rpath," + libdir, "-o", str(exe)], check=True, capture_output=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)

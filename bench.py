@@ -7,7 +7,7 @@
 A step is one forward call (ring schedule, Q/K/V tiles, QK^T, mask, online
 softmax, PV, epilogue -- one kernel launch) over the workload's inputs, which
 are resident in HBM and larger than L2.  The merge kernel is timed in its own
-region on fp32 partial results shaped like the headline workload's output.
+region on fp32 partial results shaped like the 2 x 8192 x 16 x 128 output.
 Rank 0 prints one JSON line.  Under torchrun every rank runs its own copy of
 the workload (independent (batch, head) units, no collective on the data
 path) and the throughput is the sum over ranks divided by the slowest rank's
@@ -32,12 +32,15 @@ if ROOT not in sys.path:
 
 import torch  # noqa: E402
 
-HEADLINE = "bf16_b2_h16_s8192_d128_noncausal_n8"
+# The largest single-GPU workload: 262144 tokens, causal, striped over 16
+# ring blocks, every ring pass (one of the two causal workloads the target
+# names).  The others are reported beside it.
+HEADLINE = "bf16_b1_h8_s262144_d128_causal_striped_n16_p16"
 EXTRAS = [
+    "bf16_b2_h16_s8192_d128_noncausal_n8",
     "bf16_b1_h32_s32768_d128_causal_n8_contiguous",
     "bf16_b1_h32_s32768_d128_causal_n8_striped",
     "bf16_varlen_t65536_s16_h16_d128_causal_n4_packed",
-    "bf16_b1_h8_s262144_d128_causal_striped_n16_p16",
     "bf16_b1_h8_s262144_d128_causal_striped_n16_p4",
     "bf16_b1_h32_kv4_s32768_d128_causal_n8_contiguous",
     "f16_b2_h16_s8192_d128_noncausal_n8",
@@ -177,7 +180,10 @@ def profiled_traffic(workload: str):
     if kv.get("workload") != workload:
         return None
     try:
-        return float(kv["dram_bytes_per_launch"])
+        # a capture on fewer heads than the workload scales by the heads
+        # (every head's items read that head's q/k/v the same way)
+        scale = float(kv.get("scale_to_workload", "1"))
+        return float(kv["dram_bytes_per_launch"]) * scale
     except (KeyError, ValueError):
         return None
 
@@ -457,34 +463,40 @@ def measure_merge(steps, warmup, dist, dev, peaks):
 
 
 def measure_e2e(w, steps, warmup, dist, dev):
-    """Same metric through the public API from pinned host buffers
-    (ring_attn_func_host): the host to device copy of q/k/v and the device
-    to host copy of out/lse are inside the timed region."""
+    """Same metric end to end through the C ABI's host-input call
+    (ring_attn_fwd_host): every step copies q/k/v from page-locked host
+    memory, runs the forward and copies out/lse back, chunks of heads
+    overlapping on three streams; all of it is inside the timed region.  The
+    device workspace is allocated once, outside it, as a caller would."""
     import blockwise_exact_attention_attn_b200 as ra
-    from blockwise_exact_attention_attn_b200 import inputs as gen
-    assert not w.varlen
+    assert not w.varlen and w.kv_heads == w.heads
     shape = (w.batch, w.seqlen, w.heads, w.d_head)
-    g = torch.Generator().manual_seed(w.seed)
-    host = [torch.randn(*shape, generator=g).to(w.torch_dtype).pin_memory() for _ in range(3)]
+    g = torch.Generator(device=dev).manual_seed(w.seed + 1000 * dist.rank)
+    host = [torch.randn(*shape, generator=g, device=dev).to(w.torch_dtype).cpu().pin_memory()
+            for _ in range(3)]
     out_h = torch.empty(*shape, dtype=w.torch_dtype).pin_memory()
     lse_h = torch.empty(w.batch, w.heads, w.seqlen, dtype=torch.float32).pin_memory()
+    code = {"bf16": ra.BF16, "f16": ra.F16, "f32": ra.F32}[w.dtype]
+    ws = torch.empty(ra.ring_attn_fwd_host_workspace(w.batch, w.heads, w.seqlen, w.d_head, code,
+                                                     0), dtype=torch.uint8, device=dev)
 
     def step():
-        # the host-input call: per sequence, copies in, forward, copies out on
-        # three streams, so one sequence's transfers overlap another's forward
-        ra.ring_attn_func_host(host[0], host[1], host[2], w.n_ring, w.causal, w.layout,
-                               w.softmax_scale, w.passes, out=out_h, lse=lse_h, chunk=1,
-                               device=dev)
+        ra.ring_attn_fwd_host(host[0], host[1], host[2], out_h, lse_h, w.batch, w.heads,
+                              w.seqlen, w.d_head, w.n_ring, w.layout, w.causal, w.softmax_scale,
+                              w.passes, ws)
 
     n = max(1, min(steps, 10))
     ms = time_steps(step, n, min(warmup, 3), dist, dev)
+    if ra.ring_attn_status() != ra.RA_OK:
+        raise RuntimeError("e2e: device status not OK")
     per = ms / n
     flops = workload_flops(w, [w.seqlen] * w.batch)
     h2d = sum(t.numel() * t.element_size() for t in host)
     d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * 4
-    del gen
     return {"value": flops * dist.world / (per * 1e-3) / 1e12, "unit": "TFLOP/s",
-            "ms_per_step": per, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "ms_per_step": per, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "api": "ring_attn_fwd_host (C ABI; page-locked host q/k/v/out/lse)",
+            "h2d_plus_d2h_GBps": (h2d + d2h) / (per * 1e-3) / 1e9}
 
 
 # ----------------------------------------------------------------------------- oracle
@@ -492,9 +504,14 @@ def measure_e2e(w, steps, warmup, dist, dev):
 def oracle_sample(w, budget_s: float, rows_cap: int = 1 << 20):
     """Time the fp64 oracle on sampled rows of the workload (host cores).
     Returns (TFLOP/s, seconds, rows, description)."""
+    import dataclasses
     import numpy as np
     import oracle
     from blockwise_exact_attention_attn_b200 import inputs as gen
+    if not w.varlen:
+        # one head of the workload: a row's cost depends on its keys and
+        # d_head only, and the host arrays stay small
+        w = dataclasses.replace(w, heads=1, heads_kv=0)
     inp = gen.make_inputs(w)
     starts, lens = gen.seq_offsets(w, inp)
     if w.varlen:
@@ -609,7 +626,16 @@ def run_ours(args, dist):
             break
         attempt += 1
     value = head["tflops"]
-    peak = peaks["bf16_tflops"] if w.dtype == "bf16" else None
+    # A timed region of back-to-back launches lasting a second or more runs
+    # under the power cap: its denominator is cuBLAS measured the same way
+    # (bf16_tflops_sustained); a shorter region is held to the burst figure.
+    timed_s = head["ms_per_step"] * args.steps / 1e3
+    burst = peaks["bf16_tflops"] if w.dtype == "bf16" else None
+    sustained = timed_s >= 1.0 and "bf16_tflops_sustained" in peaks
+    peak = (peaks["bf16_tflops_sustained"] if sustained else burst) if burst else None
+    peak_desc = (f"{peak_kind} sustained bf16 (cuBLAS back to back under the power cap; "
+                 f"the timed region runs {timed_s:.1f} s)" if sustained
+                 else f"{peak_kind} burst bf16 (cuBLAS)")
     traffic = profiled_traffic(w.name) if w.dtype == "bf16" else None
 
     # The extra workloads, ring steps and backward are per-GPU figures: they
@@ -650,7 +676,8 @@ def run_ours(args, dist):
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         v, t, n, cores = oracle_sample(w, 15.0)
         cpu = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-               "sample": f"{n} random query rows of head 0 (full key range each), {t:.1f} s",
+               "sample": f"{n} random query rows of one head (full key range each) of the "
+                         f"same workload, {t:.1f} s",
                # the whole workload at the sampled rate (not run)
                "extrapolated_full_config_s": flops / (v * 1e12) if v > 0 else None}
 
@@ -679,11 +706,14 @@ def run_ours(args, dist):
                    "l2": f"no flush: inputs {in_bytes / 2**20:.0f} MiB > L2 126 MiB",
                    "timing": "CUDA graph of the timed launches, CUDA events"},
         "pct_of_peak": 100.0 * value / dist.world / peak if peak else None,
+        "pct_of_measured_burst_peak": 100.0 * value / dist.world / burst if burst else None,
         "roofline": {"bound": "tensor", "achieved": value / dist.world, "peak": peak,
                      "unit": "TFLOP/s", "frac": value / dist.world / peak if peak else None,
-                     "peak_kind": f"{peak_kind} burst bf16 (cuBLAS)",
+                     "peak_kind": peak_desc,
+                     "frac_of_measured_burst": value / dist.world / burst if burst else None,
                      "datasheet_frac": value / dist.world / DATASHEET_BF16_TFLOPS,
-                     "traffic": traffic},
+                     "traffic": traffic,
+                     "algorithmic_bytes": in_bytes + out_bytes},
         "clocks": clocks.summary(),
         "gpu_launches": args.steps,
         "e2e": e2e,

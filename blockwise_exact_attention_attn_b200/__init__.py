@@ -23,7 +23,10 @@ from ._binding import (  # noqa: F401
     ring_attn_func,
     ring_attn_func_host,
     ring_attn_fwd,
+    ring_attn_fwd_host,
+    ring_attn_fwd_host_workspace,
     ring_attn_fwd_noalloc,
+    ring_attn_noalloc_status,
     ring_attn_fwd_step,
     ring_attn_gqa_fwd,
     ring_attn_fwd_simt,

@@ -31,6 +31,9 @@ EXPORTS = (
     "ring_attn_qkvpacked_fwd",
     "ring_attn_fwd_simt",
     "ring_attn_fwd_noalloc",
+    "ring_attn_noalloc_status",
+    "ring_attn_fwd_host",
+    "ring_attn_fwd_host_workspace",
     "ring_attn_merge",
     "ring_attn_status",
     "ring_attn_status_string",
@@ -84,6 +87,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.ring_attn_fwd_simt.restype = _c_int
         lib.ring_attn_fwd_noalloc.argtypes = _FWD_ARGS
         lib.ring_attn_fwd_noalloc.restype = _c_int
+        lib.ring_attn_noalloc_status.argtypes = [_c_vp]
+        lib.ring_attn_noalloc_status.restype = _c_int
+        lib.ring_attn_fwd_host.argtypes = (_FWD_ARGS[:14] + [_c_int, _c_int, _c_vp,
+                                                             ctypes.c_size_t, _c_vp])
+        lib.ring_attn_fwd_host.restype = _c_int
+        lib.ring_attn_fwd_host_workspace.argtypes = [_c_int] * 6
+        lib.ring_attn_fwd_host_workspace.restype = ctypes.c_size_t
         lib.ring_attn_qkvpacked_fwd.argtypes = [_c_vp, _c_vp, _c_vp] + _FWD_ARGS[5:]
         lib.ring_attn_qkvpacked_fwd.restype = _c_int
         lib.ring_attn_merge.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
@@ -278,6 +288,52 @@ def ring_attn_fwd_noalloc(q, k, v, out, lse, batch: int, heads: int, seqlen: int
     _check("ring_attn_fwd_noalloc", st)
 
 
+def ring_attn_noalloc_status(stream=None) -> int:
+    """Synchronize the stream; return and clear the status word of the
+    allocation-free calls (see ring_attn.h)."""
+    return int(load_library().ring_attn_noalloc_status(_stream(stream)))
+
+
+def _host_ptr(t, name: str) -> int:
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def ring_attn_fwd_host_workspace(batch: int, heads: int, seqlen: int, d_head: int,
+                                 dtype: int, head_chunk: int = 0) -> int:
+    """Bytes of device workspace ring_attn_fwd_host needs (see ring_attn.h)."""
+    return int(load_library().ring_attn_fwd_host_workspace(
+        int(batch), int(heads), int(seqlen), int(d_head), int(dtype), int(head_chunk)))
+
+
+def ring_attn_fwd_host(q, k, v, out, lse, batch: int, heads: int, seqlen: int, d_head: int,
+                       n_ring_blocks: int, layout=CONTIGUOUS, causal: bool = False,
+                       softmax_scale: Optional[float] = None,
+                       max_ring_passes: Optional[int] = None, workspace=None,
+                       head_chunk: int = 0, dtype: Optional[int] = None, stream=None) -> None:
+    """Forward on page-locked HOST tensors through a caller-owned device
+    workspace (a uint8 CUDA tensor); asynchronous on the stream (see
+    ring_attn.h)."""
+    lib = load_library()
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d_head)
+    if max_ring_passes is None:
+        max_ring_passes = n_ring_blocks
+    if workspace is None:
+        raise ValueError("workspace is required (see ring_attn_fwd_host_workspace)")
+    st = lib.ring_attn_fwd_host(
+        _host_ptr(q, "q"), _host_ptr(k, "k"), _host_ptr(v, "v"), _host_ptr(out, "out"),
+        _host_ptr(lse, "lse"), int(batch), int(heads), int(seqlen), int(d_head),
+        int(n_ring_blocks), _layout_code(layout), int(bool(causal)), float(softmax_scale),
+        int(max_ring_passes), _dtype_code(q) if dtype is None else int(dtype), int(head_chunk),
+        _ptr(workspace, "workspace"), int(workspace.numel() * workspace.element_size()),
+        _stream(stream))
+    _check("ring_attn_fwd_host", st)
+
+
 def ring_attn_qkvpacked_fwd(qkv, out, lse, batch: int, heads: int, seqlen: int, d_head: int,
                             n_ring_blocks: int, layout=CONTIGUOUS, causal: bool = False,
                             softmax_scale: Optional[float] = None,
@@ -374,74 +430,31 @@ def ring_attn_func(q, k, v, n_ring_blocks: int, causal: bool = False, layout=CON
 def ring_attn_func_host(q, k, v, n_ring_blocks: int, causal: bool = False, layout=CONTIGUOUS,
                         softmax_scale: Optional[float] = None,
                         max_ring_passes: Optional[int] = None, out=None, lse=None,
-                        chunk: int = 1, device=None):
-    """ring_attn_func on pinned HOST tensors q, k, v [batch, seqlen, heads,
-    d_head]: returns (out, lse) on the host (pinned).  The batch is processed
-    in chunks of `chunk` sequences on three CUDA streams -- host-to-device
-    copies, the forward, device-to-host copies -- with two device buffers, so
-    the copies of one chunk overlap the forward of another.  Returns after
-    the results are on the host."""
+                        head_chunk: int = 0, workspace=None, device=None):
+    """ring_attn_func on page-locked HOST tensors q, k, v [batch, seqlen,
+    heads, d_head] (same head count): returns (out, lse) on the host
+    (page-locked).  Runs ring_attn_fwd_host, which moves chunks of heads in
+    and out on its own streams while other chunks compute; `workspace`
+    (a uint8 CUDA tensor of ring_attn_fwd_host_workspace bytes) is allocated
+    when not given.  Returns after the results are on the host."""
     import torch
     B, S, H, D = q.shape
-    Hkv = k.shape[2]
-    if not (q.is_pinned() and k.is_pinned() and v.is_pinned()):
-        raise ValueError("q, k, v must be pinned host tensors")
+    if k.shape[2] != H:
+        raise ValueError("the host-input forward takes as many key/value heads as query heads")
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
     if out is None:
         out = torch.empty(B, S, H, D, dtype=q.dtype).pin_memory()
     if lse is None:
         lse = torch.empty(B, H, S, dtype=torch.float32).pin_memory()
-    chunk = max(1, min(int(chunk), B))
-    nchunks = (B + chunk - 1) // chunk
-    nbuf = min(2, nchunks)
-    bufs = [dict(q=torch.empty(chunk, S, H, D, dtype=q.dtype, device=dev),
-                 k=torch.empty(chunk, S, Hkv, D, dtype=k.dtype, device=dev),
-                 v=torch.empty(chunk, S, Hkv, D, dtype=v.dtype, device=dev),
-                 out=torch.empty(chunk, S, H, D, dtype=q.dtype, device=dev),
-                 lse=torch.empty(chunk, H, S, dtype=torch.float32, device=dev))
-            for _ in range(nbuf)]
-    s_in, s_run, s_out = (torch.cuda.Stream(dev) for _ in range(3))
-    start = torch.cuda.current_stream(dev)
-    for st in (s_in, s_run, s_out):
-        st.wait_stream(start)
-    ran = [None] * nbuf      # forward of the buffer's previous chunk done
-    drained = [None] * nbuf  # its results copied out
-    for c in range(nchunks):
-        b0, b1 = c * chunk, min(B, (c + 1) * chunk)
-        n = b1 - b0
-        bf = bufs[c % nbuf]
-        with torch.cuda.stream(s_in):
-            if ran[c % nbuf] is not None:
-                s_in.wait_event(ran[c % nbuf])
-            for name, src in (("q", q), ("k", k), ("v", v)):
-                bf[name][:n].copy_(src[b0:b1], non_blocking=True)
-            loaded = torch.cuda.Event()
-            loaded.record(s_in)
-        with torch.cuda.stream(s_run):
-            s_run.wait_event(loaded)
-            if drained[c % nbuf] is not None:
-                s_run.wait_event(drained[c % nbuf])
-            qc, kc, vc = bf["q"][:n], bf["k"][:n], bf["v"][:n]
-            oc, lc = bf["out"][:n], bf["lse"][:n]
-            if Hkv == H:
-                ring_attn_fwd(qc, kc, vc, oc, lc, n, H, S, D, n_ring_blocks, layout, causal,
-                              softmax_scale, max_ring_passes, None, None, s_run)
-            else:
-                ring_attn_gqa_fwd(qc, kc, vc, oc, lc, n, H, Hkv, S, D, n_ring_blocks, layout,
-                                  causal, softmax_scale, max_ring_passes, None, None, s_run)
-            done = torch.cuda.Event()
-            done.record(s_run)
-            ran[c % nbuf] = done
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(done)
-            out[b0:b1].copy_(oc, non_blocking=True)
-            lse[b0:b1].copy_(lc, non_blocking=True)
-            fin = torch.cuda.Event()
-            fin.record(s_out)
-            drained[c % nbuf] = fin
-    # the caller's stream orders after the last copy out; the host waits for it
-    start.wait_stream(s_out)
-    s_out.synchronize()
+    code = _dtype_code(q)
+    if workspace is None:
+        nbytes = ring_attn_fwd_host_workspace(B, H, S, D, code, head_chunk)
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        stream = torch.cuda.current_stream(dev)
+        ring_attn_fwd_host(q, k, v, out, lse, B, H, S, D, n_ring_blocks, layout, causal,
+                           softmax_scale, max_ring_passes, workspace, head_chunk, code, stream)
+        stream.synchronize()
     return out, lse
 
 

@@ -419,6 +419,191 @@ int64_t ring_attn_schedule(int seqlen, int n_ring_blocks, int layout, int causal
 }  // extern "C"
 
 // ---------------------------------------------------------------------------
+// Forward on host buffers (ring_attn_fwd_host).
+//
+// The heads are processed in chunks.  Each chunk's q/k/v columns are copied
+// from the page-locked host tensors into one of two device slots of the
+// caller's workspace (a strided 2-D copy: the chunk's heads of every token
+// row), the forward runs on the slot, and out/lse go back into the host
+// tensors' columns.  Copies in, forwards and copies out run on three streams
+// (two library streams per device and the caller's), so chunk c's forward
+// overlaps chunk c+1's copy in and chunk c-1's copy out.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+constexpr int kHostSlots = 2;
+constexpr size_t kHostAlign = 256;
+
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+  cudaEvent_t loaded[kHostSlots] = {}, computed[kHostSlots] = {}, drained[kHostSlots] = {};
+};
+HostPipe g_pipe[kMaxDevices];
+// Held while a call enqueues its work: the per-device streams and events are
+// shared, and each event must be waited on right after it is recorded.
+std::mutex g_pipe_mu;
+
+size_t align_up(size_t x) { return (x + kHostAlign - 1) & ~(kHostAlign - 1); }
+
+// Heads per chunk: the caller's choice, or about eight chunks.
+int host_head_chunk(int heads, int head_chunk) {
+  if (head_chunk > 0) return head_chunk < heads ? head_chunk : heads;
+  const int hc = (heads + 7) / 8;
+  return hc < 1 ? 1 : hc;
+}
+
+// Byte offsets of q, k, v, out, lse inside one slot, and the slot size.
+size_t host_slot_layout(int batch, int seqlen, int hc, int d_head, int esize, size_t off[5]) {
+  const size_t tens = (size_t)batch * seqlen * hc * d_head * esize;
+  const size_t lse = (size_t)batch * hc * seqlen * sizeof(float);
+  size_t o = 0;
+  for (int i = 0; i < 4; ++i) {
+    off[i] = o;
+    o += align_up(tens);
+  }
+  off[4] = o;
+  return o + align_up(lse);
+}
+
+bool is_host_pinned(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();  // clear the sticky-free error of an unknown pointer
+    return false;
+  }
+  return a.type == cudaMemoryTypeHost;
+}
+
+bool is_device(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeDevice;
+}
+
+ra_status host_pipe(HostPipe** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RA_ERR_CUDA;
+  HostPipe& hp = g_pipe[dev];
+  if (!hp.ready) {
+    bool ok = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.done, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; ok && i < kHostSlots; ++i)
+      ok = cudaEventCreateWithFlags(&hp.loaded[i], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&hp.computed[i], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&hp.drained[i], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) return RA_ERR_CUDA;  // (created handles are kept for the next try)
+    hp.ready = true;
+  }
+  *out = &hp;
+  return RA_OK;
+}
+
+}  // namespace
+
+extern "C" size_t ring_attn_fwd_host_workspace(int batch, int heads, int seqlen, int d_head,
+                                               int dtype, int head_chunk) {
+  if (batch < 1 || heads < 1 || seqlen < 1 || d_head < 1) return 0;
+  if (dtype != RA_F32 && dtype != RA_BF16 && dtype != RA_F16) return 0;
+  const int hc = host_head_chunk(heads, head_chunk);
+  const int nchunks = (heads + hc - 1) / hc;
+  size_t off[5];
+  const size_t slot =
+      host_slot_layout(batch, seqlen, hc, d_head, dtype == RA_F32 ? 4 : 2, off);
+  return slot * (size_t)(nchunks < kHostSlots ? nchunks : kHostSlots);
+}
+
+extern "C" ra_status ring_attn_fwd_host(const void* q, const void* k, const void* v, void* out,
+                                        float* lse, int batch, int heads, int seqlen,
+                                        int d_head, int n_ring_blocks, int layout, int causal,
+                                        float softmax_scale, int max_ring_passes, int dtype,
+                                        int head_chunk, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !out || !lse || !workspace) return RA_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kHostAlign - 1)) != 0) return RA_ERR_INVALID;
+  ra_status st = validate_fwd(batch, heads, heads, seqlen, d_head, n_ring_blocks, layout,
+                              causal, softmax_scale, max_ring_passes, nullptr, dtype);
+  if (st != RA_OK) return st;
+  if (head_chunk < 0) return RA_ERR_INVALID;
+  const int esize = dtype == RA_F32 ? 4 : 2;
+  const int hc = host_head_chunk(heads, head_chunk);
+  const int nchunks = (heads + hc - 1) / hc;
+  const int nslots = nchunks < kHostSlots ? nchunks : kHostSlots;
+  size_t off[5];
+  const size_t slot_bytes = host_slot_layout(batch, seqlen, hc, d_head, esize, off);
+  if (workspace_bytes < slot_bytes * nslots) return RA_ERR_INVALID;
+  if (!is_host_pinned(q) || !is_host_pinned(k) || !is_host_pinned(v) || !is_host_pinned(out) ||
+      !is_host_pinned(lse) || !is_device(workspace))
+    return RA_ERR_INVALID;
+  // the per-chunk rows: each token row holds `heads` head vectors
+  const size_t row_bytes = (size_t)heads * d_head * esize;
+  const size_t rows = (size_t)batch * seqlen;
+
+  HostPipe* hp = nullptr;
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  st = host_pipe(&hp);
+  if (st != RA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  auto ck = [](cudaError_t e) { return e == cudaSuccess; };
+  // the copy streams start after the work already on the caller's stream
+  if (!ck(cudaEventRecord(hp->start, s)) || !ck(cudaStreamWaitEvent(hp->h2d, hp->start, 0)) ||
+      !ck(cudaStreamWaitEvent(hp->d2h, hp->start, 0)))
+    return RA_ERR_CUDA;
+  char* ws = static_cast<char*>(workspace);
+  for (int c = 0; c < nchunks; ++c) {
+    const int b = c % nslots;
+    const int h0 = c * hc;
+    const int nh = heads - h0 < hc ? heads - h0 : hc;
+    char* sl = ws + (size_t)b * slot_bytes;
+    const size_t w = (size_t)nh * d_head * esize;  // bytes of the chunk in one token row
+    const size_t col = (size_t)h0 * d_head * esize;
+    // copies in: wait until the slot's previous forward has read its inputs
+    if (c >= nslots && !ck(cudaStreamWaitEvent(hp->h2d, hp->computed[b], 0))) return RA_ERR_CUDA;
+    const void* src[3] = {q, k, v};
+    for (int t = 0; t < 3; ++t)
+      if (!ck(cudaMemcpy2DAsync(sl + off[t], w, static_cast<const char*>(src[t]) + col,
+                                row_bytes, w, rows, cudaMemcpyHostToDevice, hp->h2d)))
+        return RA_ERR_CUDA;
+    if (!ck(cudaEventRecord(hp->loaded[b], hp->h2d)) ||
+        !ck(cudaStreamWaitEvent(s, hp->loaded[b], 0)))
+      return RA_ERR_CUDA;
+    // forward: wait until the slot's previous results have been copied out
+    if (c >= nslots && !ck(cudaStreamWaitEvent(s, hp->drained[b], 0))) return RA_ERR_CUDA;
+    const int64_t hd = (int64_t)nh * d_head;
+    ra::FwdParams p = make_params(sl + off[0], sl + off[1], sl + off[2], hd, nh, hd,
+                                  sl + off[3], reinterpret_cast<float*>(sl + off[4]), batch, nh,
+                                  seqlen, d_head, n_ring_blocks, layout, causal, softmax_scale,
+                                  max_ring_passes, nullptr);
+    st = run_fwd(p, dtype, stream, false);
+    if (st != RA_OK) return st;
+    if (!ck(cudaEventRecord(hp->computed[b], s)) ||
+        !ck(cudaStreamWaitEvent(hp->d2h, hp->computed[b], 0)))
+      return RA_ERR_CUDA;
+    // copies out: out columns of every token row, lse rows of every sequence
+    if (!ck(cudaMemcpy2DAsync(static_cast<char*>(out) + col, row_bytes, sl + off[3], w, w, rows,
+                              cudaMemcpyDeviceToHost, hp->d2h)))
+      return RA_ERR_CUDA;
+    const size_t lw = (size_t)nh * seqlen * sizeof(float);
+    if (!ck(cudaMemcpy2DAsync(lse + (size_t)h0 * seqlen, (size_t)heads * seqlen * sizeof(float),
+                              sl + off[4], lw, lw, (size_t)batch, cudaMemcpyDeviceToHost,
+                              hp->d2h)))
+      return RA_ERR_CUDA;
+    if (!ck(cudaEventRecord(hp->drained[b], hp->d2h))) return RA_ERR_CUDA;
+  }
+  // the caller's stream orders after the last copy out
+  if (!ck(cudaEventRecord(hp->done, hp->d2h)) || !ck(cudaStreamWaitEvent(s, hp->done, 0)))
+    return RA_ERR_CUDA;
+  return RA_OK;
+}
+
+// ---------------------------------------------------------------------------
 // Allocation-free variant of ring_attn_fwd.
 //
 // The tensor-core forward needs a little device scratch: the word that
@@ -492,9 +677,29 @@ extern "C" ra_status ring_attn_fwd_noalloc(const void* q, const void* k, const v
   p.work_counter = scratch + kNoAllocCounter;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // the array keeps the previous call's contents: start from zero
-  if (cudaMemsetAsync(scratch + kNoAllocStatus, 0, sizeof(int), s) != cudaSuccess ||
-      cudaMemsetAsync(scratch + kNoAllocCounter, 0, sizeof(int), s) != cudaSuccess)
+  // The array keeps the previous call's contents.  The counter starts from
+  // zero for every launch; the status word is left alone, so an error
+  // latched by an earlier call stays readable (ring_attn_noalloc_status)
+  // until it is read.
+  if (cudaMemsetAsync(scratch + kNoAllocCounter, 0, sizeof(int), s) != cudaSuccess)
     return RA_ERR_CUDA;
   return dispatch(p, dtype, false, s);
+}
+
+// Reads and clears the status word of the allocation-free calls.  It uses no
+// allocation either: a synchronous copy into a local variable and, only when
+// an error was latched, a synchronous clear.
+extern "C" ra_status ring_attn_noalloc_status(void* stream) {
+  int* scratch = nullptr;
+  ra_status st = noalloc_scratch(&scratch);
+  if (st != RA_OK) return st;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return RA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, scratch + kNoAllocStatus, sizeof(int), cudaMemcpyDeviceToHost) !=
+      cudaSuccess)
+    return RA_ERR_CUDA;
+  if (v != 0 && cudaMemset(scratch + kNoAllocStatus, 0, sizeof(int)) != cudaSuccess)
+    return RA_ERR_CUDA;
+  return static_cast<ra_status>(v);
 }

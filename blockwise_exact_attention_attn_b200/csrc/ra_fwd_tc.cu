@@ -47,6 +47,8 @@
 // (in log2 units); until then exponentials are taken against the stale max
 // (values <= 2^kRescaleLog2), which is exact up to rounding because the same
 // reference is used for O and l.
+#include <atomic>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -925,19 +927,25 @@ static cudaError_t launch_tc_t(const FwdParams& p, cudaStream_t stream) {
   const int64_t items = work_grid(pp, kTcBM * kTcQT);
   if (items == 0) return cudaSuccess;
   if (items > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  // persistent: one CTA per SM (shared memory and tensor memory allow one)
-  static int sms[64] = {0};
+  // persistent: one CTA per SM (shared memory and tensor memory allow one).
+  // The SM count is cached per device; host threads may launch concurrently,
+  // so the cache is atomic (a racing first lookup stores the same value).
+  static std::atomic<int> sms_cache[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!sms[dev] && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) !=
-                       cudaSuccess)
-    return cudaErrorInvalidDevice;
+  int num_sms = sms_cache[dev].load(std::memory_order_relaxed);
+  if (!num_sms) {
+    if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        num_sms < 1)
+      return cudaErrorInvalidDevice;
+    sms_cache[dev].store(num_sms, std::memory_order_relaxed);
+  }
   // Dense causal work varies per item: one CTA per item, balanced by the
   // hardware block scheduler, measured faster than persistent CTAs there.
   // Otherwise (and for ring steps, whose items are short) persistent CTAs
   // (one per SM) claim items until none is left.
   const bool per_item = p.causal && !p.cu_seqlens && !p.step;
-  const int64_t grid = per_item ? items : (items < sms[dev] ? items : sms[dev]);
+  const int64_t grid = per_item ? items : (items < num_sms ? items : num_sms);
   const int claim_limit = per_item ? 1 : 0;
   TcMaps maps;
   if (!make_map(&maps.q, p.q, p.total_rows, p.heads, D, p.tok_stride, kFmt) ||

@@ -96,6 +96,14 @@ def ring_attention_forward(q, k, v, *, causal: bool = False, layout: int = CONTI
         j = (r - s) % N
         works = []
         if s + 1 < P:
+            # Buffer reuse: bufs[s % 2] was last read by the fold of step
+            # s - 1, enqueued on the current stream before this call.  With
+            # NCCL, batch_isend_irecv makes its communication stream wait for
+            # the work already on the current stream when the ops are issued,
+            # so the receive cannot overwrite the buffer before that fold has
+            # read it; with gloo the ops run on the host after the (host)
+            # fold returned.  The w.wait() below orders the next fold after
+            # this receive in the other direction.
             nk, nv = bufs[s % 2]
             ops = [dist.P2POp(dist.isend, cur_k, peer(1), group),
                    dist.P2POp(dist.isend, cur_v, peer(1), group),

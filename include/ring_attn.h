@@ -50,6 +50,7 @@
 #ifndef RING_ATTN_H
 #define RING_ATTN_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -291,34 +292,38 @@ ra_status ring_attn_merge(void* out_a, float* lse_a, const void* out_b,
                           int d_head, int dtype, void* stream);
 
 /*
- * ring_attn_fwd_noalloc -- ring_attn_fwd that allocates nothing.  (No
- * counterpart in the pages: this is a deployment variant of the same call.)
+ * ring_attn_fwd_noalloc -- ring_attn_fwd that allocates no device memory.
+ * (The pages have no counterpart: this is a deployment variant of the same
+ * call.)
  *
- * For callers that cannot allocate device memory: code being captured into a
- * CUDA graph in a mode that forbids allocation, processes whose device memory
- * is owned by a fixed pool or budget, and runtimes that must not touch the
- * allocator after start-up.  ring_attn_fwd allocates a small device scratch
- * (error status word, work counters) with cudaMalloc on its first call on a
- * device; this entry point uses a 256-byte array that is part of the
- * library's device image instead (every device that loads the library holds
- * it until the process exits), and calls no cudaMalloc, cudaFree or other
- * allocating routine.
+ * Who needs it: callers whose device memory is all handed out up front and
+ * must not move afterwards -- inference servers and runtimes that reserve a
+ * fixed pool or budget at start-up and treat any later cudaMalloc as a leak
+ * or an out-of-memory risk, and code that runs where a cudaMalloc would
+ * synchronize the device or is not permitted at all.  ring_attn_fwd
+ * allocates a small device scratch (the error status word and the work
+ * counters) with cudaMalloc on its first call on a device; this entry point
+ * uses a 256-byte array that is part of the library's device image instead
+ * (every device that loads the library holds it until the process exits) and
+ * calls no cudaMalloc, cudaFree or other allocating routine.
  *
  *  - Arguments, layouts, ownership and host-side errors are those of
- *    ring_attn_fwd; results are identical to it.
+ *    ring_attn_fwd, and so are the results (the same kernels run).
  *  - Scratch limit: 256 bytes, of which each call uses the status word and
  *    one work counter.  No problem size changes that; a call that would need
  *    more than the array holds returns RA_ERR_UNSUPPORTED.
- *  - The first call on each device looks the array up (cudaGetSymbolAddress)
- *    with that device current; make that first call before any stream
- *    capture.
+ *  - Set-up: the first call on each device looks the array's device address
+ *    up (cudaGetSymbolAddress) with that device current.  Make that first
+ *    call before any stream capture.
  *  - All calls share the array, which keeps the last call's contents: each
- *    call clears the status word and the counter at its start (in-stream
- *    memsets).  Calls that overlap on the GPU (e.g. on different streams)
- *    race on the array and may compute wrong results; issue them on one
- *    stream or order them.
+ *    call zeroes the work counter on its stream before its kernel starts.
+ *    Calls that overlap on the GPU (e.g. on different streams) race on the
+ *    array and may compute wrong results; issue them on one stream or order
+ *    them.
  *  - Device-side errors (malformed cu_seqlens, an expired wait) are latched in
- *    the array's status word, which ring_attn_status does not read.
+ *    the array's status word (the first error wins) and stay there until
+ *    ring_attn_noalloc_status reads and clears them; ring_attn_status does
+ *    not see them.
  */
 ra_status ring_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                                 void* out, float* lse, int batch, int heads,
@@ -326,6 +331,62 @@ ra_status ring_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                                 int layout, int causal, float softmax_scale,
                                 int max_ring_passes, const int32_t* cu_seqlens,
                                 int dtype, void* stream);
+
+/*
+ * ring_attn_noalloc_status -- synchronize `stream`, then return and clear the
+ * status word of the ring_attn_fwd_noalloc calls on the current device
+ * (RA_OK when none latched an error since the last read).  Allocates nothing
+ * either: it copies the word into a host variable and clears it with
+ * synchronous CUDA calls.  Returns RA_ERR_CUDA when a CUDA call fails.
+ */
+ra_status ring_attn_noalloc_status(void* stream);
+
+/*
+ * ring_attn_fwd_host -- ring_attn_fwd on HOST buffers, with the transfers
+ * overlapped with the computation.
+ *
+ * Source: "Ring Attention" glossary, "Come funziona la ring attention": a
+ * device computes on the block it holds while the next block is in flight,
+ * so the transfer hides behind the computation.  Here the blocks are groups
+ * of heads moving between host memory and the GPU: the heads are split into
+ * chunks of head_chunk heads; chunk c's q/k/v are copied in while chunk c-1
+ * is computed and chunk c-2's out/lse are copied out, on two library
+ * streams plus `stream`, through two device slots of `workspace`.
+ *
+ *  q, k, v   HOST, page-locked (cudaHostAlloc / cudaHostRegister) dtype
+ *            [batch, seqlen, heads, d_head].
+ *  out       HOST, page-locked, same shape and dtype; written.
+ *  lse       HOST, page-locked float32 [batch, heads, seqlen]; written.
+ *  head_chunk  heads per chunk (>= 1), or 0 to let the library choose
+ *            (ceil(heads / 8)).
+ *  workspace DEVICE memory of at least ring_attn_fwd_host_workspace(...)
+ *            bytes, 256-byte aligned, owned by the caller; one call at a
+ *            time may use it.
+ * Other arguments as ring_attn_fwd (dense inputs; no cu_seqlens).
+ * Asynchronous on `stream`: the call returns once everything is enqueued;
+ * out and lse are complete when `stream` is synchronized (then read device
+ * errors with ring_attn_status).  Work already on `stream` runs first.
+ * Calls from several host threads are serialised while they enqueue.
+ * Errors: as ring_attn_fwd, plus RA_ERR_INVALID when a host buffer is not
+ * page-locked, the workspace is not device memory, is misaligned or too
+ * small, or head_chunk < 0.
+ */
+ra_status ring_attn_fwd_host(const void* q, const void* k, const void* v,
+                             void* out, float* lse, int batch, int heads,
+                             int seqlen, int d_head, int n_ring_blocks,
+                             int layout, int causal, float softmax_scale,
+                             int max_ring_passes, int dtype, int head_chunk,
+                             void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/*
+ * ring_attn_fwd_host_workspace -- bytes of device workspace ring_attn_fwd_host
+ * needs for these sizes (two slots of one chunk's q, k, v, out and lse; one
+ * slot when there is a single chunk).  Returns 0 for invalid sizes.  Host
+ * only; never fails otherwise.
+ */
+size_t ring_attn_fwd_host_workspace(int batch, int heads, int seqlen,
+                                    int d_head, int dtype, int head_chunk);
 
 /*
  * ring_attn_status -- synchronize `stream`, then return and clear the current

@@ -190,3 +190,36 @@ def test_header_is_plain_c_and_links(tmp_path):
                     "-Wl,-rpath," + libdir, "-o", str(exe)], check=True, capture_output=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
+
+
+def test_host_workspace_size_is_two_slots_of_one_chunk(lib):
+    # one slot: q, k, v, out of one chunk ([B, S, hc, D] each, 256-byte
+    # rounded) and its lse ([B, hc, S] fp32); two slots unless one chunk
+    def slot(B, S, hc, D, es):
+        up = lambda x: (x + 255) // 256 * 256
+        return 4 * up(B * S * hc * D * es) + up(B * hc * S * 4)
+    assert lib.ring_attn_fwd_host_workspace(2, 8, 1024, 128, ra.BF16, 0) == 2 * slot(2, 1024, 1, 128, 2)
+    assert lib.ring_attn_fwd_host_workspace(1, 16, 512, 64, ra.F16, 0) == 2 * slot(1, 512, 2, 64, 2)
+    assert lib.ring_attn_fwd_host_workspace(1, 5, 100, 16, ra.F32, 3) == 2 * slot(1, 100, 3, 16, 4)
+    assert lib.ring_attn_fwd_host_workspace(1, 2, 256, 128, ra.BF16, 8) == slot(1, 256, 2, 128, 2)
+    for bad in [(0, 1, 1, 16, ra.F32, 0), (1, 1, 1, 16, 9, 0), (1, 0, 1, 16, ra.F32, 0)]:
+        assert lib.ring_attn_fwd_host_workspace(*bad) == 0
+
+
+def test_host_call_rejects_invalid_arguments_before_cuda(lib):
+    def call(**over):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, batch=1, heads=2, seqlen=256,
+                 d_head=128, n=4, layout=0, causal=1, scale=0.1, passes=4, dtype=1, hc=0,
+                 ws=FAKE * 16, nbytes=1 << 30, stream=None)
+        a.update(over)
+        return lib.ring_attn_fwd_host(a["q"], a["k"], a["v"], a["out"], a["lse"], a["batch"],
+                                      a["heads"], a["seqlen"], a["d_head"], a["n"], a["layout"],
+                                      a["causal"], a["scale"], a["passes"], a["dtype"], a["hc"],
+                                      a["ws"], a["nbytes"], a["stream"])
+    for over in [dict(q=None), dict(ws=None), dict(ws=FAKE + 16), dict(seqlen=250),
+                 dict(hc=-1), dict(nbytes=0), dict(d_head=48)]:
+        assert call(**over) == ra.RA_ERR_INVALID, over
+
+
+def test_noalloc_status_is_exported_with_a_stream_argument(lib):
+    assert lib.ring_attn_noalloc_status.argtypes == [ctypes.c_void_p]

@@ -25,7 +25,7 @@
 //              shared-memory slots in the order K(0), K(1), V(0), K(2), V(1),
 //              ... (the order in which the MMA issuers consume them)
 //   warps 9,11 MMA issuers, one per query tile i: S_i = Q_i K^T into tensor
-//              memory and O_i += P_i V with P_i from shared memory, as
+//              memory and O_i += P_i V with P_i read from tensor memory, as
 //              tcgen05.mma; completion signalled with tcgen05.commit.  Two
 //              issuers keep the tensor pipe fed while one of them waits on a
 //              barrier (a tcgen05.mma group issues at about the rate it runs).
@@ -34,14 +34,18 @@
 //              class into a shared-memory ring of small list chunks
 // The control warpgroup (warps 8-11) hands registers to the softmax
 // warpgroups with setmaxnreg.
-// Tensor memory (512 columns): S_0 | S_1 | O_0 | O_1.  Shared memory: Q_0,
-// Q_1, the K/V ring, P_0, P_1 (input format, 128-byte swizzle), the list.
+// Tensor memory (512 columns): S_0 | S_1 | O_0 | O_1, with P_i (16-bit,
+// two keys per column) written over the first half of S_i once S_i is in
+// registers.  Shared memory: Q_0, Q_1, the K/V ring, the list.
 //
-// Per kv tile t issuer i issues S_i(t+1) as soon as softmax i has loaded
-// S_i(t) into registers (s_free), then PV_i(t) once P_i(t) is in shared
-// memory (p_full).  The tensor core so computes the next scores while the
-// softmax warps still work on the current ones.  pv_done tells softmax i that
-// PV_i(t) finished: P_i may be overwritten and O_i is stable for a rescale.
+// Per kv tile t issuer i waits until softmax i has written P_i(t) (p_full),
+// then issues PV_i(t) followed by S_i(t+1).  The tensor core runs the MMAs
+// of one thread in issue order, so S_i(t+1) overwrites the P_i(t) columns
+// only after PV_i(t) has read them, and the commit that announces S_i(t+1)
+// (s_full) also covers PV_i(t): when softmax i sees S_i(t+1), P_i(t) is free
+// and O_i is stable for a rescale.  While softmax i works on its tile the
+// tensor core runs the other query tile's PV and S, so the two softmax
+// warpgroups take turns on the exponential unit.
 //
 // The running max is only moved when it grows by more than kRescaleLog2
 // (in log2 units); until then exponentials are taken against the stale max
@@ -69,7 +73,7 @@ constexpr int kTcMmaWarp = 9;      // MMA issuer (allocates TMEM)
 constexpr int kTcMmaWarp1 = 11;    // second MMA issuer when kTcIssuers == 2
 constexpr int kTcListWarp = 10;
 // MMA issuer warps: 2 = one per query tile, 1 = warp 9 issues for both tiles
-constexpr int kTcIssuers = 2;
+constexpr int kTcIssuers = 1;
 constexpr int kListChunk = 16;      // entries per schedule-list chunk (published at once)
 constexpr int kListBufs = 16;       // chunks in the shared-memory ring
 constexpr int kListConsumers = 9 + kTcIssuers;  // producer, issuers, 8 softmax warps
@@ -85,29 +89,27 @@ struct TcCfg {
   static constexpr int kPanels = D / 64;                    // 128-byte swizzle panels
   static constexpr int kPanelBytes = kTcBM * 128;           // 128 rows x 128 B
   static constexpr int kTileBytes = kPanels * kPanelBytes;  // one Q/K/V tile
-  static constexpr int kStages = D == 128 ? 3 : 6;          // K/V ring slots
-  static constexpr int kPBytes = kTcBM * kTcBN * 2;         // one P tile (2 panels)
+  static constexpr int kStages = D == 128 ? 5 : 10;         // K/V ring slots
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = kTcQT * kTileBytes;
-  static constexpr int kPOff = kKVOff + kStages * kTileBytes;
-  static constexpr int kListOff = kPOff + kTcQT * kPBytes;
+  static constexpr int kListOff = kKVOff + kStages * kTileBytes;
   static constexpr int kCtrlOff = kListOff + kListBufs * kListChunk * 4;
-  static constexpr int kCtrlBytes = 512;
+  static constexpr int kCtrlBytes = 1024;
   static constexpr int kSmemBytes = kCtrlOff + kCtrlBytes + 1024;  // + align slack
   static constexpr uint32_t kColS = 0;                      // S_i at i * 128
   static constexpr uint32_t kColO = 256;                    // O_i at 256 + i * D
+  static constexpr int kSlots = 10;                         // ring slots the barriers allow
+  static_assert(kStages <= kSlots, "K/V ring barriers");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
 struct TcCtrl {
   uint64_t q_full;
   uint64_t q_free;
-  uint64_t kv_full[6];
-  uint64_t kv_empty[6];
+  uint64_t kv_full[10];
+  uint64_t kv_empty[10];
   uint64_t s_full[kTcQT];
-  uint64_t s_free[kTcQT];
   uint64_t p_full[kTcQT];
-  uint64_t pv_done[kTcQT];
   uint64_t o_full[kTcQT];
   uint64_t o_free[kTcQT];
   uint64_t list_full[kListBufs];
@@ -116,7 +118,7 @@ struct TcCtrl {
   uint32_t tmem_base;
   int abort;
 };
-static_assert(sizeof(TcCtrl) <= 512, "control block");
+static_assert(sizeof(TcCtrl) <= 1024, "control block");
 
 struct TcMaps {
   CUtensorMap q, k, v;
@@ -163,19 +165,17 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t qdesc, uint64
   }
 }
 
-// O (+)= P V for one query tile: A = P from shared memory (128 x 128 bf16,
-// K-major in two 64-key panels, like Q), B = V tile MN-major (N = D split in
-// 64-element panels, LBO = panel stride; 8-key groups 1024 bytes apart).
-// Step kk covers 16 keys.
+// O (+)= P V for one query tile: A = P from tensor memory (128 lanes x 64
+// columns, two 16-bit keys per column; 16 keys = 8 columns per step), B = V
+// tile MN-major (N = D split in 64-element panels, LBO = panel stride; 8-key
+// groups 1024 bytes apart).  Step kk covers 16 keys.
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint64_t pdesc, uint64_t vdesc,
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t vdesc,
                                          uint32_t idesc, bool accumulate) {
 #pragma unroll
-  for (int kk = 0; kk < kTcBN / 16; ++kk) {
-    const uint64_t aoff = (uint64_t)((kk >> 2) * ((kTcBM * 128) >> 4) + (kk & 3) * 2);
-    umma_ss(d_tmem, pdesc + aoff, vdesc + (uint64_t)(kk * 128), idesc,
+  for (int kk = 0; kk < kTcBN / 16; ++kk)
+    umma_ts(d_tmem, p_tmem + (uint32_t)(kk * 8), vdesc + (uint64_t)(kk * 128), idesc,
             (accumulate || kk > 0) ? 1u : 0u);
-  }
 }
 
 // Bits [lo, hi) of a 32-bit word, 0 <= lo < hi <= 32.
@@ -328,9 +328,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int i = 0; i < kTcQT; ++i) {
       mbar_init(&ctrl->s_full[i], 1);
-      mbar_init(&ctrl->s_free[i], kTcBM);
       mbar_init(&ctrl->p_full[i], kTcBM);
-      mbar_init(&ctrl->pv_done[i], 1);
       mbar_init(&ctrl->o_full[i], 1);
       mbar_init(&ctrl->o_free[i], kTcBM);
       mbar_init(&ctrl->drain[i], 1);
@@ -443,8 +441,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
    } else if (warp == kTcProducerWarp) {
     // ---------------------------------------------------------- producer
-    // Ring order K(0), K(1), V(0), K(2), V(1), ...: a K tile is needed one
-    // kv tile before the V tile of the same position.
+    // Ring order K(0), V(0), K(1), V(1), ...: the order in which the issuers
+    // consume the tiles (PV(t) comes before S(t+1)).
     if (lane == 0) {
       tma_prefetch_desc(&maps.q);
       tma_prefetch_desc(&maps.k);
@@ -489,13 +487,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                           &ctrl->q_full, pn * 64, it.h, it.base + q0 + i * kTcBM);
           ++nq;
         }
-        int prev = e;
-        while (ok && prev >= 0) {
+        if (ok && e >= 0) ok = load(&maps.v, hk, it.base + entry_tile(e) * kTcBN);
+        while (ok && e >= 0) {
           ok = rd.next(&e, abort_flag);
-          if (!ok) break;
-          if (e >= 0) ok = load(&maps.k, hk, it.base + entry_tile(e) * kTcBN);
-          if (ok) ok = load(&maps.v, hk, it.base + entry_tile(prev) * kTcBN);
-          prev = e;
+          if (!ok || e < 0) break;
+          ok = load(&maps.k, hk, it.base + entry_tile(e) * kTcBN);
+          if (ok) ok = load(&maps.v, hk, it.base + entry_tile(e) * kTcBN);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -512,25 +509,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
    } else if (warp == kTcMmaWarp || kTcIssuers == 2) {
     // ---------------------------------------------------------- MMA issuers
-    // Issuer of query tiles [i0, i1), per kv tile t: S_i(t+1) as soon as
-    // softmax i has read S_i(t) (s_free), then PV_i(t) once P_i(t) is
-    // written (p_full).  Every issuer walks the K/V ring in load order; a
-    // slot is released by one commit of each issuer.
+    // Issuer of query tiles [i0, i1): S_i(0), then per kv tile t, once
+    // softmax i has written P_i(t) into tensor memory (p_full), PV_i(t) and
+    // S_i(t+1).  Both are issued by this thread, so they run in that order:
+    // S_i(t+1) overwrites the P_i(t) columns after PV_i(t) has read them.
+    // Every issuer walks the K/V ring in load order; a slot is released by
+    // one commit of each issuer.
     const int i0 = (kTcIssuers == 2 && warp == kTcMmaWarp1) ? 1 : 0;
     const int i1 = kTcIssuers == 2 ? i0 + 1 : kTcQT;
     // a negative softmax scale is applied as S = (-Q) K^T times |scale|
     const uint32_t idesc_s =
         idesc_f16kind_f32(kTcBM, kTcBN, 0, kFmt) | (p.scale_log2 < 0.f ? (1u << 13) : 0u);
     constexpr uint32_t idesc_o = idesc_f16kind_f32(kTcBM, D, 1, kFmt);
-    // base descriptors: K-major tiles (Q, K, P) and MN-major tiles (V)
+    // base descriptors: K-major tiles (Q, K) and MN-major tiles (V)
     const uint64_t qdesc0 = smem_desc_sw128(smem_u32(smem + C::kQOff), 16, 1024);
-    const uint64_t pdesc0 = smem_desc_sw128(smem_u32(smem + C::kPOff), 16, 1024);
     const uint64_t kdesc0 = smem_desc_sw128(smem_u32(smem + C::kKVOff), 16, 1024);
     const uint64_t vdesc0 = smem_desc_sw128(smem_u32(smem + C::kKVOff), C::kPanelBytes, 1024);
     constexpr uint64_t kSlotStep = (uint64_t)(C::kTileBytes >> 4);
     constexpr uint64_t kQStep = (uint64_t)(C::kTileBytes >> 4);
-    constexpr uint64_t kPStep = (uint64_t)(C::kPBytes >> 4);
-    uint32_t ns[kTcQT] = {0, 0};  // S_i issued so far
     uint32_t pphase[kTcQT] = {0, 0};
     int n = 0, k = 0;
     bool ok = true, issued_any = false;
@@ -542,24 +538,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (ok) tc_fence_after();
       return slot;
     };
-    // S_i = Q_i K^T for this issuer's query tiles that visit kv tile entry e
-    auto issue_s = [&](int e) {
-      const int slot = take();
-      if (!ok) return;
-      for (int i = i0; i < i1; ++i) {
-        if (entry_cls(e, i) == CLS_EMPTY) continue;
-        if (ns[i] > 0) {
-          ok = mbar_wait(&ctrl->s_free[i], (ns[i] - 1) & 1, abort_flag);
-          if (!ok) return;
-          tc_fence_after();
-        }
-        issue_qk<D>(tmem + C::kColS + i * kTcBN, qdesc0 + i * kQStep,
-                    kdesc0 + slot * kSlotStep, idesc_s);
-        umma_commit(&ctrl->s_full[i]);
-        ++ns[i];
-        issued_any = true;
-      }
-      umma_commit(&ctrl->kv_empty[slot]);
+    auto issue_s_tile = [&](int e, int i, int slot) {
+      if (entry_cls(e, i) == CLS_EMPTY) return;
+      issue_qk<D>(tmem + C::kColS + i * kTcBN, qdesc0 + i * kQStep, kdesc0 + slot * kSlotStep,
+                  idesc_s);
+      umma_commit(&ctrl->s_full[i]);
+      issued_any = true;
     };
     while (ok) {
       int h = 0;
@@ -585,38 +569,44 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         int e = -1;
         if (ok) ok = rd.next(&e, abort_flag);
         if (ok && e >= 0) {
-          issue_s(e);
-          int ep = e;
+          // S_i(0) for every tile of this issuer, tile 0 first
+          const int slot_k0 = take();
+          if (ok) {
+            for (int i = i0; i < i1; ++i) issue_s_tile(e, i, slot_k0);
+            umma_commit(&ctrl->kv_empty[slot_k0]);
+          }
+          int ep = e;  // entry of kv tile t
           while (ok) {
-            ok = rd.next(&e, abort_flag);
+            ok = rd.next(&e, abort_flag);  // kv tile t + 1, or the item's end
             if (!ok) break;
             const bool has = e >= 0;
-            if (has) {
-              issue_s(e);
-              if (!ok) break;
-            } else {
-              // every S of this item is issued: Q may be replaced once they finish
-              umma_commit(&ctrl->q_free);
-            }
-            const int slot_v = take();
+            // every S of this item is issued: Q may be replaced once they finish
+            if (!has) umma_commit(&ctrl->q_free);
+            const int slot_v = take();             // V(t)
+            const int slot_k = ok && has ? take() : 0;  // K(t + 1)
             if (!ok) break;
+            // per tile, PV_i(t) then S_i(t + 1): with one issuer the tensor
+            // core runs PV_0 S_0 PV_1 S_1, so while softmax 0 works on S_0(t+1)
+            // the tensor core computes tile 1's products, and the other way round
             for (int i = i0; i < i1 && ok; ++i) {
-              if (entry_cls(ep, i) == CLS_EMPTY) continue;
-              ok = mbar_wait(&ctrl->p_full[i], pphase[i], abort_flag);
-              pphase[i] ^= 1;
-              if (!ok) break;
-              tc_fence_after();
-              if (!started[i]) wait_ofree(i);
-              if (!ok) break;
-              // an accumulating ring step adds to the O loaded from the state
-              issue_pv<D>(tmem + C::kColO + i * D, pdesc0 + i * kPStep,
-                          vdesc0 + slot_v * kSlotStep, idesc_o, started[i] || p.accumulate);
-              umma_commit(&ctrl->pv_done[i]);
-              started[i] = true;
+              if (entry_cls(ep, i) != CLS_EMPTY) {
+                ok = mbar_wait(&ctrl->p_full[i], pphase[i], abort_flag);
+                pphase[i] ^= 1;
+                if (!ok) break;
+                tc_fence_after();
+                if (!started[i]) wait_ofree(i);
+                if (!ok) break;
+                // an accumulating ring step adds to the O loaded from the state
+                issue_pv<D>(tmem + C::kColO + i * D, tmem + C::kColS + i * kTcBN,
+                            vdesc0 + slot_v * kSlotStep, idesc_o, started[i] || p.accumulate);
+                started[i] = true;
+              }
+              if (has) issue_s_tile(e, i, slot_k);
             }
             if (!ok) break;
             umma_commit(&ctrl->kv_empty[slot_v]);
             if (!has) break;
+            umma_commit(&ctrl->kv_empty[slot_k]);
             ep = e;
           }
         } else if (ok) {
@@ -651,13 +641,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::kColS + tile * kTcBN;
     const uint32_t tO = tmem + lane_off + C::kColO + tile * D;
-    // this row of P_tile: 128-byte rows, 16-byte chunks XOR-swizzled by row % 8,
-    // keys 0-63 in the first 16 KB panel and keys 64-127 in the second
-    const uint32_t prow = smem_u32(smem + C::kPOff + tile * C::kPBytes) + (uint32_t)r * 128u;
-    const uint32_t pswz = (uint32_t)(r & 7);
+    // P_tile goes over the first kTcBN / 2 columns of S_tile (two keys per column)
+    const uint32_t tP = tS;
     const float sl2 = fabsf(p.scale_log2);  // > 0; the sign is folded into the MMA
     uint32_t sphase = 0;
-    uint32_t np = 0;  // P tiles written so far
     int k = 0;
     bool ok = true;
 
@@ -734,9 +721,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int c = 0; c < kTcBN; c += 32) RA_TMEM_LD32(tS + c, (xr + c));
           tmem_wait_ld();
         }
-        // S_tile is in registers: the next S may be computed into its columns
-        tc_fence_before();
-        mbar_arrive(&ctrl->s_free[tile]);
         const int k0 = kvo + entry_tile(e) * kTcBN;  // stored index of the tile's first key
         const int nk = min(kTcBN, L - k0);
         if (cls == CLS_PARTIAL || nk < kTcBN) {
@@ -759,8 +743,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           m_ref = m_tile;
         }
         const float msub = m_ref == -INFINITY ? 0.f : m_ref;
-        // P row in registers (16-bit pairs) while the previous PV still runs;
-        // scale-and-subtract and the row sums in paired fp32 instructions
+        // P row in registers (16-bit pairs); scale-and-subtract and the row
+        // sums in paired fp32 instructions
         const uint64_t sc2 = f32x2_pack(sl2, sl2), ms2 = f32x2_pack(-msub, -msub);
         uint64_t sum2[2] = {0ull, 0ull};  // two independent (even, odd) partial sums
         uint32_t pk[kTcBN / 2];
@@ -773,19 +757,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           sum2[j & 1] = fadd2(sum2[j & 1], a, b);
           pk[j] = pack_x2<kFmt>(a, b);
         }
-        // the previous PV of this query tile has finished reading P and
-        // writing O
-        if (np > 0) {
-          ok = warp_wait(&ctrl->pv_done[tile], (np - 1) & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-        }
+        // P into tensor memory, over the scores just read (the previous PV of
+        // this tile finished before this S was announced)
 #pragma unroll
-        for (int g8 = 0; g8 < kTcBN / 8; ++g8) {
-          const uint32_t addr =
-              prow + (uint32_t)(g8 >> 3) * (kTcBM * 128u) + ((((uint32_t)g8 & 7u) ^ pswz) << 4);
-          st_shared_v4(addr, pk[4 * g8], pk[4 * g8 + 1], pk[4 * g8 + 2], pk[4 * g8 + 3]);
-        }
+        for (int c = 0; c < kTcBN / 2; c += 32) RA_TMEM_ST32(tP + c, (pk + c));
         l = l * alpha + ((f32x2_lo(sum2[0]) + f32x2_hi(sum2[0])) +
                          (f32x2_lo(sum2[1]) + f32x2_hi(sum2[1])));
         if ((!first || from_state) && __any_sync(0xffffffffu, need)) {
@@ -799,12 +774,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
             RA_TMEM_ST32(tO + c, o);
           }
-          tmem_wait_st();
         }
-        fence_proxy_async_smem();
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&ctrl->p_full[tile]);
-        ++np;
         first = false;
       }
       if (!ok) break;

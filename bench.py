@@ -399,15 +399,14 @@ def measure_ring_steps(steps, warmup, dist, dev, peaks):
 
 
 BWD_WORKLOAD = dict(batch=1, heads=8, seqlen=8192, d_head=128, causal=True, n_ring=8)
-# CUDA-core fp32 peak for the backward kernels (plain FMA arithmetic): 148
-# SMs x 128 fp32 lanes x 2 FLOP per FMA x 1.965 GHz
-CUDA_CORE_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
-def measure_backward(steps, warmup, dist, dev):
-    """Backward (ring_attn_bwd) of a bf16 causal workload: FLOPs counted as
-    10 * d_head per allowed (query, key) pair (recomputed scores, dP, dV, dQ,
-    dK: 2.5 times the forward's count)."""
+def measure_backward(steps, warmup, dist, dev, peaks):
+    """Backward (ring_attn_bwd: the tensor-core dq and dk/dv kernels) of a
+    bf16 causal workload.  FLOPs are the useful ones, 10 * d_head per allowed
+    (query, key) pair (scores, dP, dV, dQ, dK: 2.5 times the forward's
+    count); the kernels execute 14 * d_head (the dq kernel recomputes the
+    scores and dP), reported beside it."""
     import blockwise_exact_attention_attn_b200 as ra
     c = BWD_WORKLOAD
     B, H, S, D, N = c["batch"], c["heads"], c["seqlen"], c["d_head"], c["n_ring"]
@@ -425,18 +424,22 @@ def measure_backward(steps, warmup, dist, dev):
                          scale, N)
 
     from blockwise_exact_attention_attn_b200.flops import forward_flops
-    flops = 2.5 * forward_flops([S] * B, H, D, N, 0, c["causal"], N)
+    fwd = forward_flops([S] * B, H, D, N, 0, c["causal"], N)
+    flops = 2.5 * fwd
     ms = time_steps(step, steps, warmup, dist, dev, graph=True)
     if ra.ring_attn_status() != ra.RA_OK:
         raise RuntimeError("backward: device status not OK")
     per = ms / steps
     tflops = flops / (per * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
     return {"workload": f"bf16_b{B}_h{H}_s{S}_d{D}_causal_n{N} backward (dq, dk, dv)",
             "ms_per_step": per, "tflops_per_gpu": tflops, "tflops": tflops * dist.world,
             "flops_per_step": flops,
-            "roofline": {"bound": "alu", "achieved": tflops, "peak": CUDA_CORE_FP32_TFLOPS,
-                         "unit": "TFLOP/s", "frac": tflops / CUDA_CORE_FP32_TFLOPS},
-            "kernel": "bwd_dq + bwd_dkdv (CUDA cores, fp32 arithmetic)"}
+            "executed_mma_tflops": 3.5 * fwd / (per * 1e-3) / 1e12,
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak,
+                         "unit": "TFLOP/s", "frac": tflops / peak,
+                         "peak_kind": "measured burst bf16 (cuBLAS)"},
+            "kernel": "bwd_dq + bwd_dkdv (tcgen05)"}
 
 
 def measure_merge(steps, warmup, dist, dev, peaks):
@@ -663,7 +666,7 @@ def run_ours(args, dist):
     backward = None
     if run_extras:
         try:
-            backward = measure_backward(max(3, min(args.steps, 5)), 2, dist, dev)
+            backward = measure_backward(max(3, min(args.steps, 10)), 3, dist, dev, peaks)
         except Exception as e:  # report, never hide
             backward = {"workload": "backward", "error": str(e)}
         try:

@@ -20,6 +20,7 @@ from ._binding import (  # noqa: F401
     library_path,
     load_library,
     ring_attn_bwd,
+    ring_attn_bwd_simt,
     ring_attn_func,
     ring_attn_func_host,
     ring_attn_fwd,

@@ -28,6 +28,7 @@ EXPORTS = (
     "ring_attn_gqa_fwd",
     "ring_attn_fwd_step",
     "ring_attn_bwd",
+    "ring_attn_bwd_simt",
     "ring_attn_qkvpacked_fwd",
     "ring_attn_fwd_simt",
     "ring_attn_fwd_noalloc",
@@ -81,6 +82,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.ring_attn_fwd_step.restype = _c_int
         lib.ring_attn_bwd.argtypes = [_c_vp] * 9 + _GQA_ARGS[5:]
         lib.ring_attn_bwd.restype = _c_int
+        lib.ring_attn_bwd_simt.argtypes = [_c_vp] * 9 + _GQA_ARGS[5:]
+        lib.ring_attn_bwd_simt.restype = _c_int
         lib.ring_attn_gqa_fwd.argtypes = _GQA_ARGS
         lib.ring_attn_gqa_fwd.restype = _c_int
         lib.ring_attn_fwd_simt.argtypes = _FWD_ARGS
@@ -233,19 +236,39 @@ def ring_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, batch: int, heads: int, h
                   max_ring_passes: Optional[int] = None, cu_seqlens=None,
                   dtype: Optional[int] = None, stream=None) -> None:
     """Gradients dq, dk, dv of the forward (see ring_attn.h)."""
+    _bwd("ring_attn_bwd", q, k, v, out, lse, dout, dq, dk, dv, batch, heads, heads_kv, seqlen,
+         d_head, n_ring_blocks, layout, causal, softmax_scale, max_ring_passes, cu_seqlens,
+         dtype, stream)
+
+
+def ring_attn_bwd_simt(q, k, v, out, lse, dout, dq, dk, dv, batch: int, heads: int,
+                       heads_kv: int, seqlen: int, d_head: int, n_ring_blocks: int,
+                       layout=CONTIGUOUS, causal: bool = False,
+                       softmax_scale: Optional[float] = None,
+                       max_ring_passes: Optional[int] = None, cu_seqlens=None,
+                       dtype: Optional[int] = None, stream=None) -> None:
+    """Same contract as ring_attn_bwd on the CUDA-core kernels."""
+    _bwd("ring_attn_bwd_simt", q, k, v, out, lse, dout, dq, dk, dv, batch, heads, heads_kv,
+         seqlen, d_head, n_ring_blocks, layout, causal, softmax_scale, max_ring_passes,
+         cu_seqlens, dtype, stream)
+
+
+def _bwd(fn, q, k, v, out, lse, dout, dq, dk, dv, batch, heads, heads_kv, seqlen, d_head,
+         n_ring_blocks, layout, causal, softmax_scale, max_ring_passes, cu_seqlens, dtype,
+         stream) -> None:
     lib = load_library()
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(d_head)
     if max_ring_passes is None:
         max_ring_passes = n_ring_blocks
-    st = lib.ring_attn_bwd(
+    st = getattr(lib, fn)(
         _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _ptr(out, "out"), _ptr(lse, "lse"),
         _ptr(dout, "dout"), _ptr(dq, "dq"), _ptr(dk, "dk"), _ptr(dv, "dv"),
         int(batch), int(heads), int(heads_kv), int(seqlen), int(d_head), int(n_ring_blocks),
         _layout_code(layout), int(bool(causal)), float(softmax_scale), int(max_ring_passes),
         _ptr(cu_seqlens, "cu_seqlens"), _dtype_code(q) if dtype is None else int(dtype),
         _stream(stream))
-    _check("ring_attn_bwd", st)
+    _check(fn, st)
 
 
 def ring_attn_fwd_simt(q, k, v, out, lse, batch: int, heads: int, seqlen: int, d_head: int,

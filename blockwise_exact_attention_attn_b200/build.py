@@ -24,7 +24,8 @@ INCLUDE = os.path.join(ROOT, "include")
 OBJDIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libringattn.so")
 
-SOURCES = ["ra_api.cu", "ra_fwd_simt.cu", "ra_fwd_tc.cu", "ra_merge.cu", "ra_bwd_simt.cu"]
+SOURCES = ["ra_api.cu", "ra_fwd_simt.cu", "ra_fwd_tc.cu", "ra_merge.cu", "ra_bwd_simt.cu",
+           "ra_bwd_tc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",
          "--expt-relaxed-constexpr", "-I" + INCLUDE, "-I" + CSRC]

@@ -17,6 +17,9 @@ cudaError_t launch_fwd_tc(const FwdParams& p, int fmt, cudaStream_t stream);
 cudaError_t launch_fwd_simt(const FwdParams& p, int dtype, cudaStream_t stream);
 cudaError_t launch_bwd_simt(const FwdParams& f, const void* o, const void* dout, void* dq,
                             void* dk, void* dv, int dtype, cudaStream_t stream);
+cudaError_t launch_bwd_tc(const FwdParams& f, const void* o, const void* dout, void* dq,
+                          void* dk, void* dv, float* dsum, int fmt, int num_sms,
+                          cudaStream_t stream);
 cudaError_t launch_merge(void* out_a, float* lse_a, const void* out_b, const float* lse_b,
                          int batch, int heads, int seqlen, int d_head, int dtype, int num_sms,
                          cudaStream_t stream);
@@ -245,12 +248,17 @@ ra_status ring_attn_fwd_step(const void* q, const void* k, const void* v, float*
   return run_fwd(p, dtype, stream, false);
 }
 
-ra_status ring_attn_bwd(const void* q, const void* k, const void* v, const void* out,
-                        const float* lse, const void* dout, void* dq, void* dk, void* dv,
-                        int batch, int heads, int heads_kv, int seqlen, int d_head,
-                        int n_ring_blocks, int layout, int causal, float softmax_scale,
-                        int max_ring_passes, const int32_t* cu_seqlens, int dtype,
-                        void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The backward: the tensor-core kernels for 16-bit inputs with d_head 64 or
+// 128 (unless force_simt), the CUDA-core kernels otherwise.
+ra_status run_bwd(const void* q, const void* k, const void* v, const void* out,
+                  const float* lse, const void* dout, void* dq, void* dk, void* dv, int batch,
+                  int heads, int heads_kv, int seqlen, int d_head, int n_ring_blocks,
+                  int layout, int causal, float softmax_scale, int max_ring_passes,
+                  const int32_t* cu_seqlens, int dtype, void* stream, bool force_simt) {
   if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv) return RA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) ||
       !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
@@ -263,14 +271,61 @@ ra_status ring_attn_bwd(const void* q, const void* k, const void* v, const void*
                                 batch, heads, seqlen, d_head, n_ring_blocks, layout, causal,
                                 softmax_scale, max_ring_passes, cu_seqlens);
   int* status = nullptr;
-  st = device_state(&status, nullptr);
+  int sms = 0;
+  st = device_state(&status, &sms);
   if (st != RA_OK) return st;
   p.status = status;
-  cudaError_t e = ra::launch_bwd_simt(p, out, dout, dq, dk, dv,
-                                      dtype == RA_F32 ? 0 : (dtype == RA_BF16 ? 1 : 2),
-                                      reinterpret_cast<cudaStream_t>(stream));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  const bool tc = !force_simt && (dtype == RA_BF16 || dtype == RA_F16) &&
+                  (d_head == 64 || d_head == 128);
+  if (tc) {
+    // D = <dO, O> per query row passes from the dq kernel to the dk/dv
+    // kernel through stream-ordered scratch in lse layout
+    const size_t n_lse = cu_seqlens ? (size_t)heads * seqlen : (size_t)batch * heads * seqlen;
+    float* dsum = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void**>(&dsum), n_lse * sizeof(float), s) !=
+        cudaSuccess)
+      return RA_ERR_CUDA;
+    p.work_counter = next_counter(status);
+    e = cudaMemsetAsync(p.work_counter, 0, sizeof(int), s);
+    if (e == cudaSuccess)
+      e = ra::launch_bwd_tc(p, out, dout, dq, dk, dv, dsum,
+                            dtype == RA_BF16 ? ra::kFmtBF16 : ra::kFmtF16, sms, s);
+    const cudaError_t ef = cudaFreeAsync(dsum, s);
+    if (e == cudaSuccess) e = ef;
+  } else {
+    e = ra::launch_bwd_simt(p, out, dout, dq, dk, dv,
+                            dtype == RA_F32 ? 0 : (dtype == RA_BF16 ? 1 : 2), s);
+  }
   if (e == cudaErrorInvalidValue) return RA_ERR_UNSUPPORTED;
   return e == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+ra_status ring_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                        const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                        int batch, int heads, int heads_kv, int seqlen, int d_head,
+                        int n_ring_blocks, int layout, int causal, float softmax_scale,
+                        int max_ring_passes, const int32_t* cu_seqlens, int dtype,
+                        void* stream) {
+  return run_bwd(q, k, v, out, lse, dout, dq, dk, dv, batch, heads, heads_kv, seqlen, d_head,
+                 n_ring_blocks, layout, causal, softmax_scale, max_ring_passes, cu_seqlens,
+                 dtype, stream, false);
+}
+
+ra_status ring_attn_bwd_simt(const void* q, const void* k, const void* v, const void* out,
+                             const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                             int batch, int heads, int heads_kv, int seqlen, int d_head,
+                             int n_ring_blocks, int layout, int causal, float softmax_scale,
+                             int max_ring_passes, const int32_t* cu_seqlens, int dtype,
+                             void* stream) {
+  return run_bwd(q, k, v, out, lse, dout, dq, dk, dv, batch, heads, heads_kv, seqlen, d_head,
+                 n_ring_blocks, layout, causal, softmax_scale, max_ring_passes, cu_seqlens,
+                 dtype, stream, true);
 }
 
 ra_status ring_attn_gqa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,

@@ -1,0 +1,1369 @@
+// ra_bwd_tc.cu -- backward of the ring-ordered blockwise attention on the
+// sm_100a tensor cores (tcgen05 + TMEM), bf16 or fp16 inputs, fp32
+// accumulation: dq, dk, dv of sum(dout * out).
+//
+// The gradients are plain calculus on out_i = sum_j P_ij v_j with P_ij =
+// exp(scale q_i.k_j - lse_i) over the allowed keys: dV = P^T dO, dP = dO V^T,
+// dS = P (dP - D) with D_i = <dO_i, O_i>, dQ = scale dS K, dK = scale dS^T Q.
+// P is recomputed from the forward's lse, the quantity the issue thread "A
+// ring attention with flash attention kernel implementation" says the
+// blockwise method keeps (and the backward is the part that thread found
+// wrong in an implementation).  Two kernels, so every gradient element has
+// one writer and no atomics are needed:
+//
+//  bwd_dq_kernel (query-outer, the forward's ring walk over 64-key tiles):
+//   per kv tile S = Q K^T and dP = dO V^T into tensor memory, the gradient
+//   warps form dS = P (dP - D) and store it as 16-bit to shared memory, then
+//   dQ += dS K.  It also writes D per query row for the second kernel.
+//   warps 0-3 / 4-7  gradient warps of query tile 0 / 1 (one TMEM lane each)
+//   warp  8          TMA producer: Q, dO per item; (K, V) pairs into a ring
+//   warps 9, 11      MMA issuers, one per query tile
+//   warp  10         schedule builder (the ring walk with 64-key tiles)
+//   TMEM: S_0 | S_1 | dP_0 | dP_1 | dQ_0 | dQ_1 (64, 64, 64, 64, D, D).
+//
+//  bwd_dkdv_kernel (key/value-outer): a CTA owns 128 keys of one (sequence,
+//   key/value head), one TMEM lane each, and walks the 64-row query tiles
+//   of every query head of its group that see them:
+//   S^T = K Q^T and dP^T = V dO^T into tensor memory, the gradient warps form
+//   P^T and dS^T = P^T (dP^T - D) into shared memory, then dV += P^T dO and
+//   dK += dS^T Q.
+//   warps 0-3 / 4-7  gradient warps for query columns 0-31 / 32-63
+//   warp  8          TMA producer (and the per-tile lse / D vectors)
+//   warp  9          MMA issuer;  warp 10 schedule builder;  warp 11 idle
+//   TMEM: S^T 64 | dP^T 64 | dV D | dK D.
+// Every wait is bounded like the forward's: an expired wait latches
+// ST_TIMEOUT, the CTA drains what it issued and frees its tensor memory.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "ra_common.cuh"
+#include "ra_params.h"
+#include "ra_sched.h"
+#include "ra_work.cuh"
+
+namespace ra {
+namespace tcb {
+
+constexpr int BM = 128;   // query rows per tile
+constexpr int QT = 2;     // query tiles per CTA
+constexpr int BN = 64;    // keys per kv tile
+constexpr int kThreads = 384;
+constexpr int kProducer = 8, kMma0 = 9, kBuilder = 10, kMma1 = 11;
+constexpr int kChunk = 16, kBufs = 16;
+constexpr int kConsumers = 11;  // producer, 2 issuers, 8 gradient warps
+constexpr int kStages = 2;      // (K, V) pairs in the ring
+constexpr int kRegsGrad = 184, kRegsControl = 136;  // 256*184 + 128*136 = 384*168
+constexpr uint32_t kTmemCols = 512;
+
+template <int D>
+struct Cfg {
+  static constexpr int kPanels = D / 64;
+  static constexpr int kQPanel = BM * 128;
+  static constexpr int kQTile = kPanels * kQPanel;
+  static constexpr int kKPanel = BN * 128;
+  static constexpr int kKTile = kPanels * kKPanel;
+  static constexpr int kDSBytes = BM * BN * 2;  // one 128-byte panel of 64 keys
+  static constexpr int kQOff = 0;
+  static constexpr int kDOOff = kQOff + QT * kQTile;
+  static constexpr int kKVOff = kDOOff + QT * kQTile;  // slot s: K at +0, V at +kKTile
+  static constexpr int kDSOff = kKVOff + kStages * 2 * kKTile;
+  static constexpr int kListOff = kDSOff + QT * kDSBytes;
+  static constexpr int kCtrlOff = kListOff + kBufs * kChunk * 4;
+  static constexpr int kSmemBytes = kCtrlOff + 512 + 1024;
+  static constexpr uint32_t kColS = 0;      // S_i at i * 64
+  static constexpr uint32_t kColDP = 128;   // dP_i at 128 + i * 64
+  static constexpr uint32_t kColDQ = 256;   // dQ_i at 256 + i * D
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kColDQ + QT * D <= kTmemCols, "tensor memory budget");
+};
+
+struct Ctrl {
+  uint64_t q_full, q_free;
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t s_full[QT], s_free[QT];
+  uint64_t ds_full[QT], ds_done[QT];
+  uint64_t dq_full[QT], dq_free[QT];
+  uint64_t list_full[kBufs], list_empty[kBufs];
+  uint64_t drain[QT];
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(Ctrl) <= 512, "control block");
+
+struct Maps {
+  CUtensorMap q, dout, k, v;
+};
+
+// Launch parameters of both kernels.  f holds the forward's inputs,
+// geometry, lse, status word and work counter; for the dK/dV kernel f.heads
+// counts the key/value heads (the work decode runs over them).
+struct Params {
+  FwdParams f;
+  int heads_q;      // query heads
+  const void* o;    // forward output, q's layout
+  const void* dout; // q's layout
+  void* dq;         // q's layout
+  void* dk;         // k's layout
+  void* dv;         // v's layout
+  float* dsum;      // D = <dO, O> per query row, lse layout (written by bwd_dq_kernel)
+};
+
+constexpr int kItemEnd = -1, kAllDone = -2, kPad = -3, kItemInfo = 5;
+__device__ __forceinline__ int item_header(int item) { return -(item + 8); }
+__device__ __forceinline__ int entry_tile(int e) { return e >> 4; }
+__device__ __forceinline__ int entry_cls(int e, int i) { return (e >> (2 * i)) & 3; }
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const bool ok = mbar_wait(bar, parity, abort);
+  return __all_sync(0xffffffffu, ok);
+}
+
+struct ListReader {
+  const int* list;
+  uint64_t* full;
+  uint64_t* empty;
+  int n;
+  __device__ __forceinline__ bool next_raw(int* e, volatile int* abort) {
+    const int pos = n % kChunk, c = n / kChunk, b = c % kBufs;
+    if (pos == 0 && !mbar_wait(&full[b], (c / kBufs) & 1, abort)) return false;
+    *e = list[b * kChunk + pos];
+    ++n;
+    if (pos == kChunk - 1) mbar_arrive(&empty[b]);
+    return true;
+  }
+  __device__ __forceinline__ bool next_warp_raw(int* e, volatile int* abort) {
+    const int pos = n % kChunk, c = n / kChunk, b = c % kBufs;
+    if (pos == 0 && !warp_wait(&full[b], (c / kBufs) & 1, abort)) return false;
+    *e = list[b * kChunk + pos];
+    ++n;
+    if (pos == kChunk - 1) {
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[b]);
+    }
+    return true;
+  }
+  __device__ __forceinline__ bool next(int* e, volatile int* abort) {
+    do {
+      if (!next_raw(e, abort)) return false;
+    } while (*e == kPad);
+    return true;
+  }
+  __device__ __forceinline__ bool next_warp(int* e, volatile int* abort) {
+    do {
+      if (!next_warp_raw(e, abort)) return false;
+    } while (*e == kPad);
+    return true;
+  }
+};
+
+template <bool kWarp>
+__device__ __forceinline__ bool read_item(ListReader& rd, SeqWork* it, volatile int* abort) {
+  int v[kItemInfo];
+#pragma unroll
+  for (int i = 0; i < kItemInfo; ++i)
+    if (!(kWarp ? rd.next_warp_raw(&v[i], abort) : rd.next_raw(&v[i], abort))) return false;
+  it->b = v[0];
+  it->qr = v[1];
+  it->h = v[2];
+  it->base = v[3];
+  it->L = v[4];
+  it->live = true;
+  return true;
+}
+
+// Leading allowed columns of kv tile [k0, k0 + nk) for query (rq, tq) when the
+// tile lies in ring block rk (allowed keys of one block form a prefix).
+__device__ __forceinline__ int block_limit(const RingGeom& g, int rq, int tq, int rk, int k0,
+                                           int nk) {
+  if (!pass_ok(g, rq, rk)) return 0;
+  if (!g.causal) return nk;
+  int last;
+  if (g.layout == LAYOUT_CONTIGUOUS) {
+    last = tq;
+  } else {
+    if (tq < rk) return 0;
+    last = block_start(g, rk) + (tq - rk) / g.N;
+  }
+  const int lim = last - k0 + 1;
+  return lim < 0 ? 0 : (lim > nk ? nk : lim);
+}
+
+__device__ __forceinline__ uint32_t bit_range(int lo, int hi) {
+  const uint32_t upto = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
+  return upto & ~((1u << lo) - 1u);
+}
+
+// Allowed columns of the tile as two 32-bit masks.
+__device__ __forceinline__ void tile_mask(uint32_t mw[2], const FwdParams& p, int L, bool valid,
+                                          int cls, int rq, int tq, int k0, int nk) {
+  if (!valid) {
+    mw[0] = mw[1] = 0u;
+    return;
+  }
+  if (cls == CLS_FULL) {
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      const int n = min(max(nk - 32 * w, 0), 32);
+      mw[w] = n >= 32 ? 0xffffffffu : ((1u << n) - 1u);
+    }
+    return;
+  }
+  const RingGeom g = make_geom(L, p.n_ring, p.layout, p.causal, p.passes);
+  mw[0] = mw[1] = 0u;
+  const int kend = k0 + nk;
+  int c = k0;
+  for (int rk = block_of(g, k0); c < kend && rk < g.N; ++rk) {
+    const int be = min(block_start(g, rk + 1), kend);
+    if (be <= c) continue;
+    const int a = c - k0, bnd = a + block_limit(g, rq, tq, rk, c, be - c);
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      const int lo = max(a - 32 * w, 0), hi = min(bnd - 32 * w, 32);
+      if (hi > lo) mw[w] |= bit_range(lo, hi);
+    }
+    c = be;
+  }
+}
+
+// D x 64 keys for one query tile: S_i = Q_i K^T (A 128-row panels, B 64-row
+// panels, both K-major, 128-byte swizzle).
+template <int D>
+__device__ __forceinline__ void issue_qk64(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                           uint32_t idesc) {
+  using C = Cfg<D>;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint64_t ao = (uint64_t)((kk >> 2) * (C::kQPanel >> 4) + (kk & 3) * 2);
+    const uint64_t bo = (uint64_t)((kk >> 2) * (C::kKPanel >> 4) + (kk & 3) * 2);
+    umma_ss(d_tmem, adesc + ao, bdesc + bo, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// dQ_i (+)= dS_i K: A = dS (128 x 64, K-major, one panel), B = K tile
+// MN-major (N = D in 64-element panels kKPanel apart; 8-key groups 1024 B
+// apart).  Step kk covers 16 keys.
+__device__ __forceinline__ void issue_dsk(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < BN / 16; ++kk)
+    umma_ss(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 128), idesc,
+            (accumulate || kk > 0) ? 1u : 0u);
+}
+
+template <int D, int kFmt>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dq_kernel(const Params bp, const __grid_constant__ Maps maps, int n_items,
+                     int claim_limit) {
+  using C = Cfg<D>;
+  constexpr int kRows = BM * QT;
+  const FwdParams& p = bp.f;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + C::kCtrlOff);
+  volatile int* abort_flag = &ctrl->abort;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  int* list = reinterpret_cast<int*>(smem + C::kListOff);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&ctrl->q_full, 1);
+    mbar_init(&ctrl->q_free, 2);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&ctrl->kv_full[s], 1);
+      mbar_init(&ctrl->kv_empty[s], 2);
+    }
+    for (int i = 0; i < QT; ++i) {
+      mbar_init(&ctrl->s_full[i], 1);
+      mbar_init(&ctrl->s_free[i], BM);
+      mbar_init(&ctrl->ds_full[i], BM);
+      mbar_init(&ctrl->ds_done[i], 1);
+      mbar_init(&ctrl->dq_full[i], 1);
+      mbar_init(&ctrl->dq_free[i], BM);
+      mbar_init(&ctrl->drain[i], 1);
+    }
+    for (int b = 0; b < kBufs; ++b) {
+      mbar_init(&ctrl->list_full[b], 1);
+      mbar_init(&ctrl->list_empty[b], kConsumers);
+    }
+    ctrl->abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == kMma0) {
+    tmem_alloc(&ctrl->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem_base;
+  ListReader rd;
+  rd.list = list;
+  rd.full = ctrl->list_full;
+  rd.empty = ctrl->list_empty;
+  rd.n = 0;
+
+  if (warp >= 8) {
+    regs_dec<kRegsControl>();
+    if (warp == kBuilder) {
+      // ---------------------------------------------------------- schedule
+      int c = 0, pos = 0;
+      bool ok = true;
+      auto put = [&](int v) -> bool {
+        const int b = c % kBufs;
+        if (pos == 0 && c >= kBufs &&
+            !mbar_wait(&ctrl->list_empty[b], ((c / kBufs) - 1) & 1, abort_flag))
+          return false;
+        list[b * kChunk + pos] = v;
+        if (++pos == kChunk) {
+          mbar_arrive(&ctrl->list_full[b]);
+          ++c;
+          pos = 0;
+        }
+        return true;
+      };
+      auto flush = [&]() -> bool {
+        bool f = true;
+        while (f && pos != 0) f = put(kPad);
+        return f;
+      };
+      int j = 0;
+      while (ok) {
+        if (claim_limit > 0 && j >= claim_limit) {
+          if (lane == 0) ok = put(kAllDone) && flush();
+          break;
+        }
+        if (lane == 0 && j > 0) {
+          ok = flush();
+          if (ok) ok = mbar_wait(&ctrl->q_full, (j - 1) & 1, abort_flag);
+        }
+        int item = 0;
+        if (lane == 0 && ok) item = atomicAdd(p.work_counter, 1);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        item = __shfl_sync(0xffffffffu, item, 0);
+        if (!ok) break;
+        if (item >= n_items) {
+          if (lane == 0) ok = put(kAllDone) && flush();
+          break;
+        }
+        const SeqWork it = find_work_item(p, kRows, item);
+        if (!it.live) continue;
+        if (lane == 0) {
+          const int q0 = it.qr * kRows;
+          const int qm = min(q0 + BM, it.L), q1 = min(q0 + kRows, it.L);
+          const RingGeom g = make_geom(it.L, p.n_ring, p.layout, p.causal, p.passes);
+          ok = put(item_header(item)) && put(it.b) && put(it.qr) && put(it.h) &&
+               put(it.base) && put(it.L);
+          TileWalk walk;
+          walk.init(g, q0, qm, q1, BN);
+          int kt, c0, c1;
+          while (ok && walk.next(&kt, &c0, &c1)) ok = put((kt << 4) | (c1 << 2) | c0);
+          if (ok) ok = put(kItemEnd);
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        ++j;
+      }
+      if (lane == 0 && !ok) {
+        *abort_flag = 1;
+        latch_status(p.status, ST_TIMEOUT);
+      }
+      __syncwarp();
+    } else if (warp == kProducer) {
+      // ---------------------------------------------------------- producer
+      if (lane == 0) {
+        tma_prefetch_desc(&maps.q);
+        tma_prefetch_desc(&maps.dout);
+        tma_prefetch_desc(&maps.k);
+        tma_prefetch_desc(&maps.v);
+      }
+      int n = 0, k = 0, nq = 0;
+      bool ok = true;
+      // one (K, V) pair of kv tile `row` into the next ring slot
+      auto load_kv = [&](int hk, int row) -> bool {
+        const int slot = n % kStages;
+        if (n >= kStages &&
+            !mbar_wait(&ctrl->kv_empty[slot], ((n / kStages) - 1) & 1, abort_flag))
+          return false;
+        uint8_t* dst = smem + C::kKVOff + slot * 2 * C::kKTile;
+        mbar_arrive_expect_tx(&ctrl->kv_full[slot], 2 * C::kKTile);
+        for (int pn = 0; pn < C::kPanels; ++pn) {
+          tma_load_3d(dst + pn * C::kKPanel, &maps.k, &ctrl->kv_full[slot], pn * 64, hk, row);
+          tma_load_3d(dst + C::kKTile + pn * C::kKPanel, &maps.v, &ctrl->kv_full[slot],
+                      pn * 64, hk, row);
+        }
+        ++n;
+        return true;
+      };
+      while (ok) {
+        int h = 0;
+        if (lane == 0) ok = rd.next(&h, abort_flag);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        h = __shfl_sync(0xffffffffu, h, 0);
+        if (!ok || h == kAllDone) break;
+        if (lane == 0) {
+          SeqWork it;
+          ok = read_item<false>(rd, &it, abort_flag);
+          const int hk = it.h / p.kv_group;
+          int e = -1;
+          if (ok) ok = rd.next(&e, abort_flag);
+          if (ok && e >= 0) ok = load_kv(hk, it.base + entry_tile(e) * BN);
+          if (ok && k > 0) ok = mbar_wait(&ctrl->q_free, (k - 1) & 1, abort_flag);
+          if (ok) {
+            const int q0 = it.qr * kRows;
+            mbar_arrive_expect_tx(&ctrl->q_full, 2 * QT * C::kQTile);
+            for (int i = 0; i < QT; ++i)
+              for (int pn = 0; pn < C::kPanels; ++pn) {
+                tma_load_3d(smem + C::kQOff + i * C::kQTile + pn * C::kQPanel, &maps.q,
+                            &ctrl->q_full, pn * 64, it.h, it.base + q0 + i * BM);
+                tma_load_3d(smem + C::kDOOff + i * C::kQTile + pn * C::kQPanel, &maps.dout,
+                            &ctrl->q_full, pn * 64, it.h, it.base + q0 + i * BM);
+              }
+            ++nq;
+          }
+          while (ok && e >= 0) {
+            ok = rd.next(&e, abort_flag);
+            if (ok && e >= 0) ok = load_kv(hk, it.base + entry_tile(e) * BN);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        ++k;
+      }
+      if (lane == 0 && !ok) {
+        *abort_flag = 1;
+        latch_status(p.status, ST_TIMEOUT);
+        for (int u = (n > kStages ? n - kStages : 0); u < n; ++u)
+          mbar_wait(&ctrl->kv_full[u % kStages], (u / kStages) & 1, nullptr);
+        if (nq > 0) mbar_wait(&ctrl->q_full, (nq - 1) & 1, nullptr);
+      }
+      __syncwarp();
+    } else {
+      // ---------------------------------------------------------- MMA issuers
+      // Issuer i, per kv tile t: S_i(t+1), dP_i(t+1) once the gradient warps
+      // have read S_i(t), dP_i(t) (s_free); then dQ_i += dS_i(t) K(t) once
+      // dS_i(t) is in shared memory (ds_full).  The slot of tile t is released
+      // by one commit of each issuer after its dQ MMA.
+      const int i = warp == kMma1 ? 1 : 0;
+      const uint32_t idesc_s = idesc_f16kind_f32(BM, BN, 0, kFmt);
+      constexpr uint32_t idesc_q = idesc_f16kind_f32(BM, D, 1, kFmt);
+      const uint64_t qdesc = smem_desc_sw128(smem_u32(smem + C::kQOff + i * C::kQTile), 16, 1024);
+      const uint64_t dodesc =
+          smem_desc_sw128(smem_u32(smem + C::kDOOff + i * C::kQTile), 16, 1024);
+      const uint64_t dsdesc =
+          smem_desc_sw128(smem_u32(smem + C::kDSOff + i * C::kDSBytes), 16, 1024);
+      const uint64_t kdesc0 = smem_desc_sw128(smem_u32(smem + C::kKVOff), 16, 1024);
+      const uint64_t vdesc0 = smem_desc_sw128(smem_u32(smem + C::kKVOff + C::kKTile), 16, 1024);
+      const uint64_t kmn0 = smem_desc_sw128(smem_u32(smem + C::kKVOff), C::kKPanel, 1024);
+      constexpr uint64_t kSlotStep = (uint64_t)((2 * C::kKTile) >> 4);
+      const uint32_t tS = tmem + C::kColS + i * BN;
+      const uint32_t tDP = tmem + C::kColDP + i * BN;
+      const uint32_t tDQ = tmem + C::kColDQ + i * D;
+      uint32_t ns = 0, nd = 0;
+      int n = 0, k = 0;
+      bool ok = true, issued_any = false;
+      auto take = [&]() -> int {
+        const int slot = n % kStages;
+        ok = mbar_wait(&ctrl->kv_full[slot], (n / kStages) & 1, abort_flag);
+        ++n;
+        if (ok) tc_fence_after();
+        return slot;
+      };
+      while (ok) {
+        int h = 0;
+        if (lane == 0) ok = rd.next(&h, abort_flag);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        h = __shfl_sync(0xffffffffu, h, 0);
+        if (!ok || h == kAllDone) break;
+        if (lane == 0) {
+          SeqWork skip;
+          ok = read_item<false>(rd, &skip, abort_flag);
+          if (ok) ok = mbar_wait(&ctrl->q_full, k & 1, abort_flag);
+          tc_fence_after();
+          bool started = false;
+          // S_i, dP_i of the tile in `slot` if this issuer's query tile sees it
+          auto issue_sdp = [&](int e, int slot) {
+            if (entry_cls(e, i) == CLS_EMPTY) return;
+            if (ns > 0) {
+              ok = mbar_wait(&ctrl->s_free[i], (ns - 1) & 1, abort_flag);
+              if (!ok) return;
+              tc_fence_after();
+            }
+            issue_qk64<D>(tS, qdesc, kdesc0 + slot * kSlotStep, idesc_s);
+            issue_qk64<D>(tDP, dodesc, vdesc0 + slot * kSlotStep, idesc_s);
+            umma_commit(&ctrl->s_full[i]);
+            ++ns;
+            issued_any = true;
+          };
+          int e = -1;
+          if (ok) ok = rd.next(&e, abort_flag);
+          if (ok && e >= 0) {
+            int slot = take();
+            if (ok) issue_sdp(e, slot);
+            while (ok) {
+              int en = -1;
+              ok = rd.next(&en, abort_flag);
+              if (!ok) break;
+              int slot_n = -1;
+              if (en >= 0) {
+                slot_n = take();
+                if (!ok) break;
+                issue_sdp(en, slot_n);
+                if (!ok) break;
+              } else {
+                umma_commit(&ctrl->q_free);  // every S/dP of this item issued
+              }
+              if (entry_cls(e, i) != CLS_EMPTY) {
+                ok = mbar_wait(&ctrl->ds_full[i], nd & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                if (!started && k > 0) {
+                  ok = mbar_wait(&ctrl->dq_free[i], (k - 1) & 1, abort_flag);
+                  if (!ok) break;
+                  tc_fence_after();
+                }
+                issue_dsk(tDQ, dsdesc, kmn0 + slot * kSlotStep, idesc_q, started);
+                umma_commit(&ctrl->ds_done[i]);
+                ++nd;
+                started = true;
+              }
+              umma_commit(&ctrl->kv_empty[slot]);
+              if (en < 0) break;
+              e = en;
+              slot = slot_n;
+            }
+          } else if (ok) {
+            umma_commit(&ctrl->q_free);
+          }
+          if (ok) {
+            if (!started && k > 0) {
+              // no dQ MMA this item: the read-out of the previous one must
+              // still finish before dq_full is signalled again
+              ok = mbar_wait(&ctrl->dq_free[i], (k - 1) & 1, abort_flag);
+              tc_fence_after();
+            }
+            if (ok) umma_commit(&ctrl->dq_full[i]);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        ++k;
+      }
+      if (lane == 0 && !ok) {
+        *abort_flag = 1;
+        latch_status(p.status, ST_TIMEOUT);
+        if (issued_any) {
+          umma_commit(&ctrl->drain[i]);
+          mbar_wait(&ctrl->drain[i], 0, nullptr);
+        }
+      }
+      __syncwarp();
+    }
+  } else {
+    regs_inc<kRegsGrad>();
+    // ---------------------------------------------------------- gradient warps
+    const int tile = warp >> 2;
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::kColS + tile * BN;
+    const uint32_t tDP = tmem + lane_off + C::kColDP + tile * BN;
+    const uint32_t tDQ = tmem + lane_off + C::kColDQ + tile * D;
+    const uint32_t dsrow = smem_u32(smem + C::kDSOff + tile * C::kDSBytes) + (uint32_t)r * 128u;
+    const uint32_t swz = (uint32_t)(r & 7);
+    uint32_t sphase = 0, nd = 0;
+    int k = 0;
+    bool ok = true;
+    while (true) {
+      int h;
+      ok = rd.next_warp(&h, abort_flag);
+      if (!ok || h == kAllDone) break;
+      SeqWork it;
+      ok = read_item<true>(rd, &it, abort_flag);
+      if (!ok) break;
+      const int L = it.L;
+      const int sq = it.qr * kRows + tile * BM + r;
+      const bool valid = sq < L;
+      int rq = 0, tq = 0;
+      if (valid) {
+        const RingGeom g = make_geom(L, p.n_ring, p.layout, p.causal, p.passes);
+        rq = block_of(g, sq);
+        tq = token_of(g, sq, rq);
+      }
+      const int64_t li = (int64_t)it.b * p.lse_seq_stride + (int64_t)it.h * p.lse_head_stride +
+                         (p.cu_seqlens ? it.base : 0) + sq;
+      const int64_t roff = ((int64_t)(it.base + sq) * bp.heads_q + it.h) * D;
+      // D = <dO, O> for this row, fp32 over the 16-bit inputs
+      float dsum = 0.f, lse2 = 0.f;
+      if (valid) {
+        const uint4* dorow = reinterpret_cast<const uint4*>(
+            static_cast<const uint16_t*>(bp.dout) + roff);
+        const uint4* orow =
+            reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(bp.o) + roff);
+#pragma unroll 4
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 a = dorow[c], b = orow[c];
+          const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float a0, a1, b0, b1;
+            if (kFmt == kFmtBF16) {
+              a0 = __uint_as_float(av[j] << 16);
+              a1 = __uint_as_float(av[j] & 0xffff0000u);
+              b0 = __uint_as_float(bv[j] << 16);
+              b1 = __uint_as_float(bv[j] & 0xffff0000u);
+            } else {
+              const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&av[j]));
+              const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&bv[j]));
+              a0 = fa.x; a1 = fa.y; b0 = fb.x; b1 = fb.y;
+            }
+            dsum = fmaf(a0, b0, dsum);
+            dsum = fmaf(a1, b1, dsum);
+          }
+        }
+        lse2 = p.lse[li] * 1.4426950408889634f;
+        if (bp.dsum) bp.dsum[li] = dsum;
+      }
+      bool any = false;
+      while (true) {
+        int e;
+        ok = rd.next_warp(&e, abort_flag);
+        if (!ok || e < 0) break;
+        const int cls = entry_cls(e, tile);
+        if (cls == CLS_EMPTY) continue;
+        ok = warp_wait(&ctrl->s_full[tile], sphase, abort_flag);
+        sphase ^= 1;
+        if (!ok) break;
+        tc_fence_after();
+        float s[BN], dp[BN];
+        {
+          uint32_t* sr = reinterpret_cast<uint32_t*>(s);
+          uint32_t* dr = reinterpret_cast<uint32_t*>(dp);
+          RA_TMEM_LD32(tS, sr);
+          RA_TMEM_LD32(tS + 32, (sr + 32));
+          RA_TMEM_LD32(tDP, dr);
+          RA_TMEM_LD32(tDP + 32, (dr + 32));
+          tmem_wait_ld();
+        }
+        tc_fence_before();
+        mbar_arrive(&ctrl->s_free[tile]);
+        const int k0 = entry_tile(e) * BN;
+        const int nk = min(BN, L - k0);
+        uint32_t mw[2];
+        tile_mask(mw, p, L, valid, cls, rq, tq, k0, nk);
+        uint32_t pk[BN / 2];
+#pragma unroll
+        for (int j = 0; j < BN / 2; ++j) {
+          const int c0 = 2 * j, c1 = 2 * j + 1;
+          const bool a0 = (mw[c0 >> 5] >> (c0 & 31)) & 1u;
+          const bool a1 = (mw[c1 >> 5] >> (c1 & 31)) & 1u;
+          const float p0 = a0 ? ex2_approx(fmaf(s[c0], p.scale_log2, -lse2)) : 0.f;
+          const float p1 = a1 ? ex2_approx(fmaf(s[c1], p.scale_log2, -lse2)) : 0.f;
+          pk[j] = pack_x2<kFmt>(p0 * (dp[c0] - dsum), p1 * (dp[c1] - dsum));
+        }
+        // the previous dQ MMA of this tile has read dS
+        if (nd > 0) {
+          ok = warp_wait(&ctrl->ds_done[tile], (nd - 1) & 1, abort_flag);
+          if (!ok) break;
+        }
+#pragma unroll
+        for (int g8 = 0; g8 < BN / 8; ++g8) {
+          const uint32_t addr = dsrow + ((((uint32_t)g8) ^ swz) << 4);
+          st_shared_v4(addr, pk[4 * g8], pk[4 * g8 + 1], pk[4 * g8 + 2], pk[4 * g8 + 3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&ctrl->ds_full[tile]);
+        ++nd;
+        any = true;
+      }
+      if (!ok) break;
+      // epilogue: dQ out of tensor memory, scaled, in the input format
+      ok = warp_wait(&ctrl->dq_full[tile], k & 1, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t o[32];
+        if (any) {
+          RA_TMEM_LD32(tDQ + c, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = 0u;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          pk[j] = pack_x2<kFmt>(__uint_as_float(o[2 * j]) * p.scale,
+                                __uint_as_float(o[2 * j + 1]) * p.scale);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(bp.dq) + roff + c);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&ctrl->dq_free[tile]);
+      ++k;
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) latch_status(p.status, ST_TIMEOUT);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMma0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) !=
+            cudaSuccess ||
+        qres != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// [rows, heads, D] 16-bit view, box 64 x 1 x box_rows, 128-byte swizzle.
+static bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int heads, int D,
+                     int64_t tok_stride, int fmt, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)tok_stride * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapDataType dt =
+      fmt == kFmtBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  return enc(map, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+template <int D, int kFmt>
+static cudaError_t launch_t(const Params& bp_in, cudaStream_t stream, int num_sms) {
+  using C = Cfg<D>;
+  Params bp = bp_in;
+  FwdParams& p = bp.f;
+  p.n_qranges = (p.seqlen + BM * QT - 1) / (BM * QT);
+  if (!p.cu_seqlens) p.n_qranges = (p.seqlen + BM * QT - 1) / (BM * QT);
+  const int64_t items = work_grid(p, BM * QT);
+  if (items == 0) return cudaSuccess;
+  if (items > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  const bool per_item = p.causal && !p.cu_seqlens;
+  const int64_t grid = per_item ? items : (items < num_sms ? items : num_sms);
+  Maps maps;
+  if (!make_map(&maps.q, p.q, p.total_rows, p.heads, D, p.tok_stride, kFmt, BM) ||
+      !make_map(&maps.dout, bp.dout, p.total_rows, bp.heads_q, D, (int64_t)bp.heads_q * D,
+                kFmt, BM) ||
+      !make_map(&maps.k, p.k, p.total_rows, p.heads_kv, D, p.kv_tok_stride, kFmt, BN) ||
+      !make_map(&maps.v, p.v, p.total_rows, p.heads_kv, D, p.kv_tok_stride, kFmt, BN))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel<D, kFmt>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  bwd_dq_kernel<D, kFmt><<<(unsigned)grid, kThreads, C::kSmemBytes, stream>>>(
+      bp, maps, (int)items, per_item ? 1 : 0);
+  return cudaGetLastError();
+}
+
+
+namespace kv {
+
+constexpr int BK = 128;  // keys per CTA
+constexpr int BQ = 64;   // query rows per step
+constexpr int kMma = 9;
+constexpr int kKvConsumers = 10;  // producer, issuer, 8 gradient warps
+constexpr int kQStages = 2;       // (Q, dO) pairs in the ring
+
+template <int D>
+struct Cfg {
+  static constexpr int kPanels = D / 64;
+  static constexpr int kKPanel = BK * 128;      // 16 KB: 128 rows x 128 B
+  static constexpr int kKTile = kPanels * kKPanel;
+  static constexpr int kQPanel = BQ * 128;      // 8 KB: 64 rows x 128 B
+  static constexpr int kQTile = kPanels * kQPanel;
+  static constexpr int kPBytes = BK * BQ * 2;   // one 128-byte panel of 64 queries
+  static constexpr int kKOff = 0;
+  static constexpr int kVOff = kKOff + kKTile;
+  static constexpr int kRingOff = kVOff + kKTile;  // slot s: Q at +0, dO at +kQTile
+  static constexpr int kPOff = kRingOff + kQStages * 2 * kQTile;
+  static constexpr int kDSOff = kPOff + kPBytes;
+  static constexpr int kVecOff = kDSOff + kPBytes;  // per slot: lse2[64], D[64]
+  static constexpr int kListOff = kVecOff + kQStages * 2 * BQ * 4;
+  static constexpr int kCtrlOff = kListOff + kBufs * kChunk * 4;
+  static constexpr int kSmemBytes = kCtrlOff + 512 + 1024;
+  static constexpr uint32_t kColS = 0, kColDP = 64, kColDV = 128, kColDK = 128 + D;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kColDK + D <= kTmemCols, "tensor memory budget");
+};
+
+struct Ctrl {
+  uint64_t kv_full, kv_free;
+  uint64_t q_full[kQStages], q_empty[kQStages];
+  uint64_t s_full, s_free;
+  uint64_t pds_full, pds_done;
+  uint64_t acc_full, acc_free;
+  uint64_t list_full[kBufs], list_empty[kBufs];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(Ctrl) <= 512, "control block");
+
+struct Maps {
+  CUtensorMap k, v, q, dout;
+};
+
+// entries: (query head within the group << 24) | (query tile << 2) | class
+__device__ __forceinline__ int entry_g(int e) { return e >> 24; }
+__device__ __forceinline__ int entry_qt(int e) { return (e >> 2) & 0x3fffff; }
+__device__ __forceinline__ int entry_cls(int e) { return e & 3; }
+
+// A (128 rows, panels kKPanel apart) x B (64 rows, panels kQPanel apart),
+// both K-major: M = 128, N = 64, K = D.
+template <int D>
+__device__ __forceinline__ void issue_kq(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc) {
+  using C = Cfg<D>;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint64_t ao = (uint64_t)((kk >> 2) * (C::kKPanel >> 4) + (kk & 3) * 2);
+    const uint64_t bo = (uint64_t)((kk >> 2) * (C::kQPanel >> 4) + (kk & 3) * 2);
+    umma_ss(d_tmem, adesc + ao, bdesc + bo, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// acc (+)= A B: A = 128 x 64 K-major (one panel), B = 64-row tile MN-major
+// (N = D in panels kQPanel apart).  Step kk covers 16 queries.
+__device__ __forceinline__ void issue_acc(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < BQ / 16; ++kk)
+    umma_ss(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 128), idesc,
+            (accumulate || kk > 0) ? 1u : 0u);
+}
+
+template <int D, int kFmt>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dkdv_kernel(const Params bp, const __grid_constant__ Maps maps, int n_items) {
+  using C = Cfg<D>;
+  const FwdParams& p = bp.f;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + C::kCtrlOff);
+  volatile int* abort_flag = &ctrl->abort;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  int* list = reinterpret_cast<int*>(smem + C::kListOff);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&ctrl->kv_full, 1);
+    mbar_init(&ctrl->kv_free, 1);
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(&ctrl->q_full[s], 1);
+      mbar_init(&ctrl->q_empty[s], 1);
+    }
+    mbar_init(&ctrl->s_full, 1);
+    mbar_init(&ctrl->s_free, 256);
+    mbar_init(&ctrl->pds_full, 256);
+    mbar_init(&ctrl->pds_done, 1);
+    mbar_init(&ctrl->acc_full, 1);
+    mbar_init(&ctrl->acc_free, 256);
+    mbar_init(&ctrl->drain, 1);
+    for (int b = 0; b < kBufs; ++b) {
+      mbar_init(&ctrl->list_full[b], 1);
+      mbar_init(&ctrl->list_empty[b], kKvConsumers);
+    }
+    ctrl->abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == kMma) {
+    tmem_alloc(&ctrl->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem_base;
+  ListReader rd;
+  rd.list = list;
+  rd.full = ctrl->list_full;
+  rd.empty = ctrl->list_empty;
+  rd.n = 0;
+
+  if (warp >= 8) {
+    regs_dec<kRegsControl>();
+    if (warp == kBuilder) {
+      // ---------------------------------------------------------- schedule
+      // One item per CTA (grid = items): its header, then every query tile
+      // that sees the key tile, with its class.
+      int c = 0, pos = 0;
+      bool ok = true;
+      auto put = [&](int v) -> bool {
+        const int b = c % kBufs;
+        if (pos == 0 && c >= kBufs &&
+            !mbar_wait(&ctrl->list_empty[b], ((c / kBufs) - 1) & 1, abort_flag))
+          return false;
+        list[b * kChunk + pos] = v;
+        if (++pos == kChunk) {
+          mbar_arrive(&ctrl->list_full[b]);
+          ++c;
+          pos = 0;
+        }
+        return true;
+      };
+      const int item = blockIdx.x;
+      const SeqWork it = find_work_item(p, BK, item);
+      if (lane == 0) {
+        if (it.live && item < n_items) {
+          const int k_lo = it.qr * BK, k_hi = min(k_lo + BK, it.L);
+          const RingGeom g = make_geom(it.L, p.n_ring, p.layout, p.causal, p.passes);
+          ok = put(item_header(item)) && put(it.b) && put(it.qr) && put(it.h) &&
+               put(it.base) && put(it.L);
+          const int nqt = (it.L + BQ - 1) / BQ;
+          // every query head of the key/value head's group, in turn
+          for (int gq = 0; ok && gq < p.kv_group; ++gq)
+            for (int qt = 0; ok && qt < nqt; ++qt) {
+              const int q_lo = qt * BQ, q_hi = min(q_lo + BQ, it.L);
+              const int cls = classify(g, q_lo, q_hi, k_lo, k_hi);
+              if (cls != CLS_EMPTY) ok = put((gq << 24) | (qt << 2) | cls);
+            }
+          if (ok) ok = put(kItemEnd);
+        }
+        if (ok) ok = put(kAllDone);
+        while (ok && pos != 0) ok = put(kPad);
+        if (!ok) {
+          *abort_flag = 1;
+          latch_status(p.status, ST_TIMEOUT);
+        }
+      }
+      __syncwarp();
+    } else if (warp == kProducer) {
+      // ---------------------------------------------------------- producer
+      // The whole warp reads the list; per query tile its lanes stage the
+      // tile's lse (log2 units) and D into the slot's vectors, then lane 0
+      // arms the slot's barrier and issues the Q and dO copies.
+      if (lane == 0) {
+        tma_prefetch_desc(&maps.k);
+        tma_prefetch_desc(&maps.v);
+        tma_prefetch_desc(&maps.q);
+        tma_prefetch_desc(&maps.dout);
+      }
+      int n = 0, k = 0, nkv = 0;
+      bool ok = true;
+      while (ok) {
+        int h = 0;
+        ok = rd.next_warp(&h, abort_flag);
+        if (!ok || h == kAllDone) break;
+        SeqWork it;
+        ok = read_item<true>(rd, &it, abort_flag);
+        if (ok && k > 0) ok = warp_wait(&ctrl->kv_free, (k - 1) & 1, abort_flag);
+        if (!ok) break;
+        if (lane == 0) {
+          const int k_row = it.base + it.qr * BK;
+          mbar_arrive_expect_tx(&ctrl->kv_full, 2 * C::kKTile);
+          for (int pn = 0; pn < C::kPanels; ++pn) {
+            tma_load_3d(smem + C::kKOff + pn * C::kKPanel, &maps.k, &ctrl->kv_full, pn * 64,
+                        it.h, k_row);
+            tma_load_3d(smem + C::kVOff + pn * C::kKPanel, &maps.v, &ctrl->kv_full, pn * 64,
+                        it.h, k_row);
+          }
+        }
+        ++nkv;
+        while (ok) {
+          int e = 0;
+          ok = rd.next_warp(&e, abort_flag);
+          if (!ok || e < 0) break;
+          const int slot = n % kQStages;
+          if (n >= kQStages) {
+            ok = warp_wait(&ctrl->q_empty[slot], ((n / kQStages) - 1) & 1, abort_flag);
+            if (!ok) break;
+          }
+          const int q_lo = entry_qt(e) * BQ;
+          const int hq = it.h * p.kv_group + entry_g(e);  // query head
+          float* vec = reinterpret_cast<float*>(smem + C::kVecOff) + slot * 2 * BQ;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int j = lane + 32 * u;
+            const int qi = q_lo + j;
+            float l2 = 0.f, dd = 0.f;
+            if (qi < it.L) {
+              const int64_t li = (int64_t)it.b * p.lse_seq_stride +
+                                 (int64_t)hq * p.lse_head_stride +
+                                 (p.cu_seqlens ? it.base : 0) + qi;
+              l2 = p.lse[li] * 1.4426950408889634f;
+              dd = bp.dsum[li];
+            }
+            vec[j] = l2;
+            vec[BQ + j] = dd;
+          }
+          __syncwarp();
+          if (lane == 0) {
+            uint8_t* dst = smem + C::kRingOff + slot * 2 * C::kQTile;
+            const int q_row = it.base + q_lo;
+            mbar_arrive_expect_tx(&ctrl->q_full[slot], 2 * C::kQTile);
+            for (int pn = 0; pn < C::kPanels; ++pn) {
+              tma_load_3d(dst + pn * C::kQPanel, &maps.q, &ctrl->q_full[slot], pn * 64, hq,
+                          q_row);
+              tma_load_3d(dst + C::kQTile + pn * C::kQPanel, &maps.dout, &ctrl->q_full[slot],
+                          pn * 64, hq, q_row);
+            }
+          }
+          ++n;
+        }
+        ++k;
+      }
+      if (lane == 0 && !ok) {
+        *abort_flag = 1;
+        latch_status(p.status, ST_TIMEOUT);
+        for (int u = (n > kQStages ? n - kQStages : 0); u < n; ++u)
+          mbar_wait(&ctrl->q_full[u % kQStages], (u / kQStages) & 1, nullptr);
+        if (nkv > 0) mbar_wait(&ctrl->kv_full, (nkv - 1) & 1, nullptr);
+      }
+      __syncwarp();
+    } else if (warp == kMma) {
+      // ---------------------------------------------------------- MMA issuer
+      // Per query tile t: S^T(t+1), dP^T(t+1) once the gradient warps have
+      // read S^T(t), dP^T(t) (s_free); then dV += P^T(t) dO(t), dK += dS^T(t)
+      // Q(t) once P^T(t), dS^T(t) are in shared memory (pds_full).
+      const uint32_t idesc_s = idesc_f16kind_f32(BK, BQ, 0, kFmt);
+      constexpr uint32_t idesc_a = idesc_f16kind_f32(BK, D, 1, kFmt);
+      const uint64_t kdesc = smem_desc_sw128(smem_u32(smem + C::kKOff), 16, 1024);
+      const uint64_t vdesc = smem_desc_sw128(smem_u32(smem + C::kVOff), 16, 1024);
+      const uint64_t qk0 = smem_desc_sw128(smem_u32(smem + C::kRingOff), 16, 1024);
+      const uint64_t dok0 = smem_desc_sw128(smem_u32(smem + C::kRingOff + C::kQTile), 16, 1024);
+      const uint64_t qmn0 = smem_desc_sw128(smem_u32(smem + C::kRingOff), C::kQPanel, 1024);
+      const uint64_t domn0 =
+          smem_desc_sw128(smem_u32(smem + C::kRingOff + C::kQTile), C::kQPanel, 1024);
+      const uint64_t pdesc = smem_desc_sw128(smem_u32(smem + C::kPOff), 16, 1024);
+      const uint64_t dsdesc = smem_desc_sw128(smem_u32(smem + C::kDSOff), 16, 1024);
+      constexpr uint64_t kSlotStep = (uint64_t)((2 * C::kQTile) >> 4);
+      const uint32_t tS = tmem + C::kColS, tDP = tmem + C::kColDP;
+      const uint32_t tDV = tmem + C::kColDV, tDK = tmem + C::kColDK;
+      uint32_t ns = 0, npd = 0;
+      int n = 0, k = 0;
+      bool ok = true, issued_any = false;
+      auto take = [&]() -> int {
+        const int slot = n % kQStages;
+        ok = mbar_wait(&ctrl->q_full[slot], (n / kQStages) & 1, abort_flag);
+        ++n;
+        if (ok) tc_fence_after();
+        return slot;
+      };
+      auto issue_sdp = [&](int slot) {
+        if (ns > 0) {
+          ok = mbar_wait(&ctrl->s_free, (ns - 1) & 1, abort_flag);
+          if (!ok) return;
+          tc_fence_after();
+        }
+        issue_kq<D>(tS, kdesc, qk0 + slot * kSlotStep, idesc_s);
+        issue_kq<D>(tDP, vdesc, dok0 + slot * kSlotStep, idesc_s);
+        umma_commit(&ctrl->s_full);
+        ++ns;
+        issued_any = true;
+      };
+      while (ok) {
+        int h = 0;
+        if (lane == 0) ok = rd.next(&h, abort_flag);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        h = __shfl_sync(0xffffffffu, h, 0);
+        if (!ok || h == kAllDone) break;
+        if (lane == 0) {
+          SeqWork skip;
+          ok = read_item<false>(rd, &skip, abort_flag);
+          if (ok) ok = mbar_wait(&ctrl->kv_full, k & 1, abort_flag);
+          tc_fence_after();
+          bool started = false;
+          int e = -1;
+          if (ok) ok = rd.next(&e, abort_flag);
+          if (ok && e >= 0) {
+            int slot = take();
+            if (ok) issue_sdp(slot);
+            while (ok) {
+              int en = -1;
+              ok = rd.next(&en, abort_flag);
+              if (!ok) break;
+              int slot_n = -1;
+              if (en >= 0) {
+                slot_n = take();
+                if (!ok) break;
+                issue_sdp(slot_n);
+                if (!ok) break;
+              } else {
+                umma_commit(&ctrl->kv_free);  // every S^T/dP^T of this item issued
+              }
+              ok = mbar_wait(&ctrl->pds_full, npd & 1, abort_flag);
+              if (!ok) break;
+              tc_fence_after();
+              if (!started && k > 0) {
+                ok = mbar_wait(&ctrl->acc_free, (k - 1) & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+              }
+              issue_acc(tDV, pdesc, domn0 + slot * kSlotStep, idesc_a, started);
+              issue_acc(tDK, dsdesc, qmn0 + slot * kSlotStep, idesc_a, started);
+              umma_commit(&ctrl->pds_done);
+              umma_commit(&ctrl->q_empty[slot]);
+              ++npd;
+              started = true;
+              if (en < 0) break;
+              e = en;
+              slot = slot_n;
+            }
+          } else if (ok) {
+            umma_commit(&ctrl->kv_free);
+          }
+          if (ok) {
+            if (!started && k > 0) {
+              ok = mbar_wait(&ctrl->acc_free, (k - 1) & 1, abort_flag);
+              tc_fence_after();
+            }
+            if (ok) umma_commit(&ctrl->acc_full);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        ++k;
+      }
+      if (lane == 0 && !ok) {
+        *abort_flag = 1;
+        latch_status(p.status, ST_TIMEOUT);
+        if (issued_any) {
+          umma_commit(&ctrl->drain);
+          mbar_wait(&ctrl->drain, 0, nullptr);
+        }
+      }
+      __syncwarp();
+    }
+  } else {
+    regs_inc<kRegsGrad>();
+    // ---------------------------------------------------------- gradient warps
+    const int half = warp >> 2;           // query columns [32 half, 32 half + 32)
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;       // key row of the tile
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::kColS + half * 32;
+    const uint32_t tDP = tmem + lane_off + C::kColDP + half * 32;
+    const uint32_t prow = smem_u32(smem + C::kPOff) + (uint32_t)r * 128u;
+    const uint32_t dsrow = smem_u32(smem + C::kDSOff) + (uint32_t)r * 128u;
+    const uint32_t swz = (uint32_t)(r & 7);
+    uint32_t sphase = 0, npd = 0;
+    int k = 0, nstep = 0;
+    bool ok = true;
+    while (true) {
+      int h;
+      ok = rd.next_warp(&h, abort_flag);
+      if (!ok || h == kAllDone) break;
+      SeqWork it;
+      ok = read_item<true>(rd, &it, abort_flag);
+      if (!ok) break;
+      const int L = it.L;
+      const int sk = it.qr * BK + r;
+      const bool kvalid = sk < L;
+      const RingGeom g = make_geom(L, p.n_ring, p.layout, p.causal, p.passes);
+      bool any = false;
+      while (true) {
+        int e;
+        ok = rd.next_warp(&e, abort_flag);
+        if (!ok || e < 0) break;
+        const int cls = entry_cls(e);
+        const int q_lo = entry_qt(e) * BQ;
+        const int slot = nstep % kQStages;
+        // the slot's lse / D vectors were written before its barrier was armed
+        ok = warp_wait(&ctrl->q_full[slot], (nstep / kQStages) & 1, abort_flag);
+        if (!ok) break;
+        const float* vec = reinterpret_cast<const float*>(smem + C::kVecOff) + slot * 2 * BQ;
+        ++nstep;
+        ok = warp_wait(&ctrl->s_full, sphase, abort_flag);
+        sphase ^= 1;
+        if (!ok) break;
+        tc_fence_after();
+        float s[32], dp[32];
+        {
+          uint32_t* sr = reinterpret_cast<uint32_t*>(s);
+          uint32_t* dr = reinterpret_cast<uint32_t*>(dp);
+          RA_TMEM_LD32(tS, sr);
+          RA_TMEM_LD32(tDP, dr);
+          tmem_wait_ld();
+        }
+        tc_fence_before();
+        mbar_arrive(&ctrl->s_free);
+        uint32_t pp[16], pd[16];
+#pragma unroll
+        for (int j2 = 0; j2 < 16; ++j2) {
+          float pv[2], dv2[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int j = 2 * j2 + u;
+            const int qi = q_lo + half * 32 + j;   // query row in the sequence
+            bool a = kvalid && qi < L;
+            if (a && cls == CLS_PARTIAL) {
+              const int rq = block_of(g, qi);
+              a = allowed(g, qi, rq, token_of(g, qi, rq), sk);
+            }
+            float pj = 0.f, dsj = 0.f;
+            if (a) {
+              const int jj = half * 32 + j;
+              pj = ex2_approx(fmaf(s[j], p.scale_log2, -vec[jj]));
+              dsj = pj * (dp[j] - vec[BQ + jj]);
+            }
+            pv[u] = pj;
+            dv2[u] = dsj;
+          }
+          pp[j2] = pack_x2<kFmt>(pv[0], pv[1]);
+          pd[j2] = pack_x2<kFmt>(dv2[0], dv2[1]);
+        }
+        // the previous dV/dK MMAs have read P^T, dS^T
+        if (npd > 0) {
+          ok = warp_wait(&ctrl->pds_done, (npd - 1) & 1, abort_flag);
+          if (!ok) break;
+        }
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const uint32_t chunk = ((uint32_t)(half * 4 + c4) ^ swz) << 4;
+          st_shared_v4(prow + chunk, pp[4 * c4], pp[4 * c4 + 1], pp[4 * c4 + 2], pp[4 * c4 + 3]);
+          st_shared_v4(dsrow + chunk, pd[4 * c4], pd[4 * c4 + 1], pd[4 * c4 + 2],
+                       pd[4 * c4 + 3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&ctrl->pds_full);
+        ++npd;
+        any = true;
+      }
+      if (!ok) break;
+      // epilogue: warps 0-3 write dV, warps 4-7 dK (scaled), one key row each
+      ok = warp_wait(&ctrl->acc_full, k & 1, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tA = tmem + lane_off + (half == 0 ? C::kColDV : C::kColDK);
+      const float mul = half == 0 ? 1.f : p.scale;
+      const int64_t goff = ((int64_t)(it.base + sk) * p.heads + it.h) * D;
+      uint16_t* dst16 = static_cast<uint16_t*>(half == 0 ? bp.dv : bp.dk);
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t o[32];
+        if (any) {
+          RA_TMEM_LD32(tA + c, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = 0u;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          pk[j] = pack_x2<kFmt>(__uint_as_float(o[2 * j]) * mul,
+                                __uint_as_float(o[2 * j + 1]) * mul);
+        if (kvalid) {
+          uint4* dst = reinterpret_cast<uint4*>(dst16 + goff + c);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&ctrl->acc_free);
+      ++k;
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) latch_status(p.status, ST_TIMEOUT);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+
+template <int D, int kFmt>
+static cudaError_t launch_t(const Params& bp_in, cudaStream_t stream) {
+  using C = Cfg<D>;
+  Params bp = bp_in;
+  FwdParams& p = bp.f;
+  p.order = 0;
+  p.n_qranges = (p.seqlen + BK - 1) / BK;
+  const int64_t items = work_grid(p, BK);
+  if (items == 0) return cudaSuccess;
+  if (items > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  Maps maps;
+  if (!make_map(&maps.k, p.k, p.total_rows, p.heads, D, p.kv_tok_stride, kFmt, BK) ||
+      !make_map(&maps.v, p.v, p.total_rows, p.heads, D, p.kv_tok_stride, kFmt, BK) ||
+      !make_map(&maps.q, p.q, p.total_rows, bp.heads_q, D, p.tok_stride, kFmt, BQ) ||
+      !make_map(&maps.dout, bp.dout, p.total_rows, bp.heads_q, D, (int64_t)bp.heads_q * D,
+                kFmt, BQ))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, kFmt>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  bwd_dkdv_kernel<D, kFmt><<<(unsigned)items, kThreads, C::kSmemBytes, stream>>>(
+      bp, maps, (int)items);
+  return cudaGetLastError();
+}
+
+}  // namespace kv
+
+template <int D, int kFmt>
+static cudaError_t launch_both(const Params& bp, int num_sms, cudaStream_t stream) {
+  cudaError_t e = launch_t<D, kFmt>(bp, stream, num_sms);
+  if (e != cudaSuccess) return e;
+  // dK/dV: the work decode runs over the key/value heads
+  Params kvp = bp;
+  kvp.f.heads = bp.f.heads_kv;
+  return kv::launch_t<D, kFmt>(kvp, stream);
+}
+
+}  // namespace tcb
+
+// dq (and D into dsum), then dk and dv, on `stream`.  f: the forward's
+// parameters (q/k/v, lse, geometry, status word, a zeroed work counter);
+// dsum: float scratch in lse layout.  16-bit inputs, d_head 64 or 128.
+cudaError_t launch_bwd_tc(const FwdParams& f, const void* o, const void* dout, void* dq,
+                          void* dk, void* dv, float* dsum, int fmt, int num_sms,
+                          cudaStream_t stream) {
+  tcb::Params bp;
+  bp.f = f;
+  bp.heads_q = f.heads;
+  bp.o = o;
+  bp.dout = dout;
+  bp.dq = dq;
+  bp.dk = dk;
+  bp.dv = dv;
+  bp.dsum = dsum;
+  if (fmt == kFmtBF16) {
+    if (f.d_head == 128) return tcb::launch_both<128, kFmtBF16>(bp, num_sms, stream);
+    if (f.d_head == 64) return tcb::launch_both<64, kFmtBF16>(bp, num_sms, stream);
+  } else if (fmt == kFmtF16) {
+    if (f.d_head == 128) return tcb::launch_both<128, kFmtF16>(bp, num_sms, stream);
+    if (f.d_head == 64) return tcb::launch_both<64, kFmtF16>(bp, num_sms, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ra

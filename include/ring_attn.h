@@ -210,8 +210,15 @@ ra_status ring_attn_fwd_step(const void* q, const void* k, const void* v,
  * are plain calculus on out_i = sum_j P_ij v_j, P_ij = exp(scale q_i.k_j -
  * lse_i) over the allowed keys: dV = P^T dout, dS = P (dP - D) with dP =
  * dout v^T and D_i = dout_i . out_i, dQ = scale dS K, dK = scale dS^T Q.
- * P is recomputed from the forward's lse.  Computed on CUDA cores in fp32
- * arithmetic (two kernels: query rows for dq, key rows for dk/dv).
+ * P is recomputed from the forward's lse.  Two kernels, so that every
+ * gradient element has one writer: a query-outer one for dq (it also forms
+ * D_i) and a key/value-outer one for dk and dv.  RA_BF16 and RA_F16 with
+ * d_head 64 or 128 run on the tensor cores (16-bit products, fp32
+ * accumulation; P and dS are rounded to the input type before their
+ * products); everything else runs on CUDA cores in fp32 arithmetic.  The
+ * tensor-core path takes batch * heads * seqlen (varlen: heads * seqlen)
+ * floats of stream-ordered scratch per call (cudaMallocAsync / cudaFreeAsync
+ * on `stream`, from the device's default memory pool).
  *
  *  q, k, v, out, lse  as passed to / returned by the forward (k, v with
  *            heads_kv heads; heads_kv == heads for ring_attn_fwd).
@@ -229,6 +236,21 @@ ra_status ring_attn_bwd(const void* q, const void* k, const void* v,
                         int n_ring_blocks, int layout, int causal,
                         float softmax_scale, int max_ring_passes,
                         const int32_t* cu_seqlens, int dtype, void* stream);
+
+/*
+ * ring_attn_bwd_simt -- ring_attn_bwd computed by the CUDA-core kernels
+ * (fp32 arithmetic) for every dtype and d_head; for RA_BF16 / RA_F16 it is
+ * an independent second GPU path used to cross-check the tensor-core
+ * backward.  Arguments and errors as ring_attn_bwd; allocates nothing.
+ */
+ra_status ring_attn_bwd_simt(const void* q, const void* k, const void* v,
+                             const void* out, const float* lse,
+                             const void* dout, void* dq, void* dk, void* dv,
+                             int batch, int heads, int heads_kv, int seqlen,
+                             int d_head, int n_ring_blocks, int layout,
+                             int causal, float softmax_scale,
+                             int max_ring_passes, const int32_t* cu_seqlens,
+                             int dtype, void* stream);
 
 /*
  * ring_attn_qkvpacked_fwd -- same computation, q/k/v packed in one tensor.

@@ -94,3 +94,69 @@ def test_backward_varlen_matches_oracle():
     ref = oracle.attention_backward(p, dout.double().numpy())
     w = gen.Workload("bwdvl", "bf16", 1, H, T, D, True, N, 0, N, seed=0)
     check_grads(w, (dq.cpu(), dk.cpu(), dv.cpu()), ref)
+
+
+# The 16-bit cases with d_head 64 or 128 above run on the tensor cores; the
+# tests below add a larger case, the CUDA-core cross-check and the masked-key
+# invariance of dq.
+
+def test_tensor_core_backward_on_a_multi_tile_case():
+    # 4096 tokens: 32 query tiles of 128 rows and 64 key tiles of 64 keys per
+    # head, 8 ring blocks, causal striped with a pass cap
+    w = gen.Workload("bwd_big", "bf16", 1, 2, 4096, 128, True, 8, 1, 5, seed=930)
+    inp = gen.make_inputs(w)
+    g = torch.Generator().manual_seed(931)
+    dout = torch.randn(1, 4096, 2, 128, generator=g).to(torch.bfloat16)
+    got = run_bwd(w, inp, dout)
+    ref = oracle.attention_backward(problem_for(w, inp),
+                                    dout.reshape(4096, 2, 128).double().numpy())
+    check_grads(w, got, ref)
+
+
+@pytest.mark.parametrize("dt,D,causal,layout,P,Hkv", [
+    ("bf16", 128, True, 0, 8, 2), ("f16", 64, False, 1, 3, 1), ("bf16", 64, True, 1, 8, 4)])
+def test_tensor_core_backward_agrees_with_cuda_core_kernels(dt, D, causal, layout, P, Hkv):
+    w = gen.Workload("bwd_x", dt, 2, 4, 1024, D, causal, 8, layout, P, seed=940 + D,
+                     heads_kv=Hkv)
+    inp = gen.make_inputs(w)
+    q, k, v = (inp[n].to(DEV) for n in ("q", "k", "v"))
+    B, S, H, _ = q.shape
+    out = torch.empty_like(q)
+    lse = torch.empty(B, H, S, device=DEV)
+    ra.ring_attn_gqa_fwd(q, k, v, out, lse, B, H, Hkv, S, D, w.n_ring, w.layout, w.causal,
+                         w.softmax_scale, w.passes)
+    dout = torch.randn(B, S, H, D, generator=torch.Generator().manual_seed(941)).to(q.dtype)
+    dout = dout.to(DEV)
+    res = []
+    for fn in (ra.ring_attn_bwd, ra.ring_attn_bwd_simt):
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        fn(q, k, v, out, lse, dout, dq, dk, dv, B, H, Hkv, S, D, w.n_ring, w.layout, w.causal,
+           w.softmax_scale, w.passes)
+        torch.cuda.synchronize()
+        assert ra.ring_attn_status() == ra.RA_OK
+        res.append((dq.float(), dk.float(), dv.float()))
+    tol = BWD_TOL[dt]
+    for a, b in zip(*res):
+        assert float((a - b).abs().max()) <= tol * (1.0 + float(b.abs().max()))
+
+
+def test_dq_of_rows_that_never_see_a_key_block_is_bitwise_unchanged():
+    # causal contiguous: rows before the last ring block never see its keys,
+    # so overwriting that block's k and v (large finite values) must leave
+    # their dq bitwise as it was
+    B, H, S, D, N = 1, 2, 2048, 128, 4
+    w = gen.Workload("bwd_mask", "bf16", B, H, S, D, True, N, 0, N, seed=950)
+    inp = gen.make_inputs(w)
+    dout = torch.randn(B, S, H, D, generator=torch.Generator().manual_seed(951))
+    dout = dout.to(torch.bfloat16)
+    dqs = []
+    for poison in (False, True):
+        k, v = inp["k"].clone(), inp["v"].clone()
+        if poison:
+            k[:, 3 * S // 4:] = 1e4
+            v[:, 3 * S // 4:] = -1e4
+        w_inp = dict(q=inp["q"], k=k, v=v)
+        dq, _, _ = run_bwd(w, w_inp, dout)
+        dqs.append(dq)
+    rows = 3 * S // 4
+    assert torch.equal(dqs[0][:rows], dqs[1][:rows])

@@ -1208,6 +1208,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         mbar_arrive(&ctrl->s_free);
+        // this half's 32 query columns: lse (log2 units) and D, read as
+        // vectors from shared memory before any arithmetic
+        float l2[32], dd[32];
+        {
+          const uint32_t va = smem_u32(vec + half * 32), vb = smem_u32(vec + BQ + half * 32);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            ld_shared_f4(va + 16u * u, l2[4 * u], l2[4 * u + 1], l2[4 * u + 2], l2[4 * u + 3]);
+            ld_shared_f4(vb + 16u * u, dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
+          }
+        }
+        // allowed query columns of this key row as a bit word
+        const int qc = q_lo + half * 32;  // first query column of this half
+        uint32_t am = 0u;
+        if (kvalid) {
+          const int nq = min(max(L - qc, 0), 32);
+          am = nq >= 32 ? 0xffffffffu : ((1u << nq) - 1u);
+          if (cls == CLS_PARTIAL) {
+            uint32_t bits = 0u;
+            for (int j = 0; j < nq; ++j) {
+              const int qi = qc + j;
+              const int rq = block_of(g, qi);
+              if (allowed(g, qi, rq, token_of(g, qi, rq), sk)) bits |= 1u << j;
+            }
+            am &= bits;
+          }
+        }
         uint32_t pp[16], pd[16];
 #pragma unroll
         for (int j2 = 0; j2 < 16; ++j2) {
@@ -1215,20 +1242,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int j = 2 * j2 + u;
-            const int qi = q_lo + half * 32 + j;   // query row in the sequence
-            bool a = kvalid && qi < L;
-            if (a && cls == CLS_PARTIAL) {
-              const int rq = block_of(g, qi);
-              a = allowed(g, qi, rq, token_of(g, qi, rq), sk);
-            }
-            float pj = 0.f, dsj = 0.f;
-            if (a) {
-              const int jj = half * 32 + j;
-              pj = ex2_approx(fmaf(s[j], p.scale_log2, -vec[jj]));
-              dsj = pj * (dp[j] - vec[BQ + jj]);
-            }
-            pv[u] = pj;
-            dv2[u] = dsj;
+            const float pj = ex2_approx(fmaf(s[j], p.scale_log2, -l2[j]));
+            const bool a = (am >> j) & 1u;
+            pv[u] = a ? pj : 0.f;
+            dv2[u] = a ? pj * (dp[j] - dd[j]) : 0.f;
           }
           pp[j2] = pack_x2<kFmt>(pv[0], pv[1]);
           pd[j2] = pack_x2<kFmt>(dv2[0], dv2[1]);

@@ -793,7 +793,7 @@ constexpr int BK = 128;  // keys per CTA
 constexpr int BQ = 64;   // query rows per step
 constexpr int kMma = 9;
 constexpr int kKvConsumers = 10;  // producer, issuer, 8 gradient warps
-constexpr int kQStages = 2;       // (Q, dO) pairs in the ring
+constexpr int kQStages = 3;       // (Q, dO) pairs in the ring
 
 template <int D>
 struct Cfg {
@@ -881,7 +881,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&ctrl->kv_full, 1);
     mbar_init(&ctrl->kv_free, 1);
     for (int s = 0; s < kQStages; ++s) {
-      mbar_init(&ctrl->q_full[s], 1);
+      // two arrivals: the copies' expect_tx and the producer once the
+      // slot's lse / D vectors are written
+      mbar_init(&ctrl->q_full[s], 2);
       mbar_init(&ctrl->q_empty[s], 1);
     }
     mbar_init(&ctrl->s_full, 1);
@@ -1002,6 +1004,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const int q_lo = entry_qt(e) * BQ;
           const int hq = it.h * p.kv_group + entry_g(e);  // query head
+          // the copies first, so their latency overlaps the vector loads
+          if (lane == 0) {
+            uint8_t* dst = smem + C::kRingOff + slot * 2 * C::kQTile;
+            const int q_row = it.base + q_lo;
+            mbar_arrive_expect_tx(&ctrl->q_full[slot], 2 * C::kQTile);
+            for (int pn = 0; pn < C::kPanels; ++pn) {
+              tma_load_3d(dst + pn * C::kQPanel, &maps.q, &ctrl->q_full[slot], pn * 64, hq,
+                          q_row);
+              tma_load_3d(dst + C::kQTile + pn * C::kQPanel, &maps.dout, &ctrl->q_full[slot],
+                          pn * 64, hq, q_row);
+            }
+          }
           float* vec = reinterpret_cast<float*>(smem + C::kVecOff) + slot * 2 * BQ;
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
@@ -1019,17 +1033,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             vec[BQ + j] = dd;
           }
           __syncwarp();
-          if (lane == 0) {
-            uint8_t* dst = smem + C::kRingOff + slot * 2 * C::kQTile;
-            const int q_row = it.base + q_lo;
-            mbar_arrive_expect_tx(&ctrl->q_full[slot], 2 * C::kQTile);
-            for (int pn = 0; pn < C::kPanels; ++pn) {
-              tma_load_3d(dst + pn * C::kQPanel, &maps.q, &ctrl->q_full[slot], pn * 64, hq,
-                          q_row);
-              tma_load_3d(dst + C::kQTile + pn * C::kQPanel, &maps.dout, &ctrl->q_full[slot],
-                          pn * 64, hq, q_row);
-            }
-          }
+          if (lane == 0) mbar_arrive(&ctrl->q_full[slot]);
           ++n;
         }
         ++k;

@@ -271,10 +271,13 @@ def time_steps(step, steps, warmup, dist, dev, graph=False):
     return dist.max(ms)
 
 
-def measure_workload(name, steps, warmup, dist, dev, peaks):
+def measure_workload(name, steps, warmup, dist, dev, peaks, heads=0):
+    import dataclasses
     from blockwise_exact_attention_attn_b200 import inputs as gen
     import blockwise_exact_attention_attn_b200 as ra
     w = gen.WORKLOADS[name]
+    if heads:
+        w = dataclasses.replace(w, heads=heads, heads_kv=0)
     step, lens, in_bytes, out_bytes, keep = make_step(w, dev, dist.rank)
     flops = workload_flops(w, lens)
     ms = time_steps(step, steps, warmup, dist, dev, graph=True)
@@ -601,12 +604,28 @@ def main():
     ap.add_argument("--workload", default=HEADLINE)
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time only the backward (ring_attn_bwd) workload and print its "
+                         "object (for profiling captures)")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run the workload with this many heads (a reduced copy for "
+                         "profiling captures); 0 keeps the workload's own")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     dist = Dist()
     try:
         if args.impl == "reference":
             run_reference(args, dist)
+            return
+        if args.backward:
+            import blockwise_exact_attention_attn_b200 as ra
+            dev = torch.device("cuda", dist.local)
+            torch.cuda.set_device(dev)
+            ra.load_library()
+            peaks, _ = load_peaks()
+            r = measure_backward(args.steps, args.warmup, dist, dev, peaks)
+            if dist.rank == 0:
+                print(json.dumps({"backward": r}), flush=True)
             return
         run_ours(args, dist)
     finally:
@@ -624,7 +643,7 @@ def run_ours(args, dist):
     while True:
         with ClockSampler(dist.local) as clocks:
             head, w, in_bytes, out_bytes, flops = measure_workload(
-                args.workload, args.steps, args.warmup, dist, dev, peaks)
+                args.workload, args.steps, args.warmup, dist, dev, peaks, args.heads)
         if not clocks.rejected() or attempt >= 1:
             break
         attempt += 1
@@ -639,7 +658,7 @@ def run_ours(args, dist):
     peak_desc = (f"{peak_kind} sustained bf16 (cuBLAS back to back under the power cap; "
                  f"the timed region runs {timed_s:.1f} s)" if sustained
                  else f"{peak_kind} burst bf16 (cuBLAS)")
-    traffic = profiled_traffic(w.name) if w.dtype == "bf16" else None
+    traffic = profiled_traffic(w.name) if w.dtype == "bf16" and not args.heads else None
 
     # The extra workloads, ring steps and backward are per-GPU figures: they
     # run at N = 1 only, so a multi-rank run stays short and its line carries

@@ -37,6 +37,7 @@ from ._binding import (  # noqa: F401
     ring_attn_schedule,
     ring_attn_status,
     ring_attn_test_withhold_q,
+    ring_attn_test_dump_schedule,
     ring_attn_status_string,
     ring_attn_varlen_qkvpacked_func,
 )

@@ -40,6 +40,7 @@ EXPORTS = (
     "ring_attn_status_string",
     "ring_attn_schedule",
     "ring_attn_test_withhold_q",
+    "ring_attn_test_dump_schedule",
 )
 
 
@@ -111,6 +112,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.ring_attn_schedule.restype = _c_i64
         lib.ring_attn_test_withhold_q.argtypes = [_c_int]
         lib.ring_attn_test_withhold_q.restype = _c_int
+        lib.ring_attn_test_dump_schedule.argtypes = [_c_vp, _c_i64]
+        lib.ring_attn_test_dump_schedule.restype = _c_int
         _lib = lib
         return lib
 
@@ -398,6 +401,21 @@ def ring_attn_test_withhold_q(on: bool) -> bool:
     no query tile, so their bounded wait expires and RA_ERR_TIMEOUT is latched.
     Returns the previous setting."""
     return bool(load_library().ring_attn_test_withhold_q(1 if on else 0))
+
+
+def ring_attn_test_dump_schedule(buf) -> None:
+    """Schedule-dump test hook: a CUDA int32 tensor of 4 + 4 * capacity
+    elements receives one record per visited kv tile of every tensor-core
+    forward launch while set; None turns it off (see ring_attn.h)."""
+    lib = load_library()
+    if buf is None:
+        st = lib.ring_attn_test_dump_schedule(None, 0)
+    else:
+        n = buf.numel()
+        if n < 4 or (n - 4) % 4:
+            raise ValueError("buf must hold 4 + 4 * capacity int32 elements")
+        st = lib.ring_attn_test_dump_schedule(_ptr(buf, "buf"), (n - 4) // 4)
+    _check("ring_attn_test_dump_schedule", st)
 
 
 def ring_attn_schedule(seqlen: int, n_ring_blocks: int, layout=CONTIGUOUS,

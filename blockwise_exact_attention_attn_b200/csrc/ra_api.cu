@@ -39,6 +39,10 @@ int g_num_sms[kMaxDevices] = {0};
 unsigned g_next_slot[kMaxDevices] = {0};
 // Failure-detection test hook, read by every forward call (ring_attn_test_withhold_q).
 std::atomic<int> g_withhold_q{0};
+// Schedule-dump test hook (ring_attn_test_dump_schedule): device buffer and
+// record capacity, read by every forward call.
+std::atomic<int*> g_sched_dump{nullptr};
+std::atomic<int64_t> g_sched_dump_cap{0};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -147,6 +151,8 @@ ra::FwdParams make_params(const void* q, const void* k, const void* v, int64_t t
   p.q_block = p.kv_block = p.step_rows = 0;
   p.accumulate = 0;
   p.withhold_q = g_withhold_q.load(std::memory_order_relaxed);
+  p.sched_dump = g_sched_dump.load(std::memory_order_relaxed);
+  p.sched_dump_cap = g_sched_dump_cap.load(std::memory_order_relaxed);
   return p;
 }
 
@@ -420,6 +426,13 @@ ra_status ring_attn_status(void* stream) {
 
 int ring_attn_test_withhold_q(int on) {
   return g_withhold_q.exchange(on ? 1 : 0);
+}
+
+ra_status ring_attn_test_dump_schedule(int32_t* buf, int64_t capacity) {
+  if (capacity < 0 || (buf == nullptr && capacity != 0)) return RA_ERR_INVALID;
+  g_sched_dump_cap.store(buf ? capacity : 0, std::memory_order_relaxed);
+  g_sched_dump.store(buf, std::memory_order_relaxed);
+  return RA_OK;
 }
 
 const char* ring_attn_status_string(int status) {

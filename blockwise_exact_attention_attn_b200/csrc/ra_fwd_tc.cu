@@ -414,10 +414,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ok = put(item_header(item)) && put(it.b) && put(it.qr) && put(it.h) && put(it.base) &&
              put(it.L);
         int kt, c0, c1;
+        // test hook: a record of each visited kv tile
+        auto dump = [&](int entry) {
+          if (!p.sched_dump) return;
+          const int i = atomicAdd(p.sched_dump, 1);
+          if (i < p.sched_dump_cap) {
+            int* r = p.sched_dump + 4 + 4 * (int64_t)i;
+            r[0] = it.b;
+            r[1] = it.h;
+            r[2] = it.qr;
+            r[3] = entry;
+          }
+        };
         if (!p.step) {
           TileWalk walk;
           walk.init(g, q0, qm, q1, kTcBN);
-          while (ok && walk.next(&kt, &c0, &c1)) ok = put((kt << 4) | (c1 << 2) | c0);
+          while (ok && walk.next(&kt, &c0, &c1)) {
+            dump((kt << 4) | (c1 << 2) | c0);
+            ok = put((kt << 4) | (c1 << 2) | c0);
+          }
         } else {
           // one ring step: the tiles of key/value block kv_block (tile-aligned
           // blocks; kt counts tiles inside the block)
@@ -426,7 +441,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int k0 = ko + kt * kTcBN;
             c0 = classify(g, qo + q0, qo + qm, k0, k0 + kTcBN);
             c1 = classify(g, qo + qm, qo + q1, k0, k0 + kTcBN);
-            if (c0 != CLS_EMPTY || c1 != CLS_EMPTY) ok = put((kt << 4) | (c1 << 2) | c0);
+            if (c0 != CLS_EMPTY || c1 != CLS_EMPTY) {
+              dump((kt << 4) | (c1 << 2) | c0);
+              ok = put((kt << 4) | (c1 << 2) | c0);
+            }
           }
         }
         if (ok) ok = put(kItemEnd);

@@ -49,6 +49,13 @@ struct FwdParams {
   // producer issues no query-tile load, so the MMA issuers' bounded wait for
   // Q expires and the launch unwinds with ST_TIMEOUT.
   int withhold_q;
+  // Schedule-dump test hook (NULL in normal use): the tensor-core kernel's
+  // schedule builder appends one record {b, h, qr, entry} per visited kv
+  // tile to sched_dump + 4, counting records in sched_dump[0] (atomically;
+  // only the first sched_dump_cap are stored).  entry = (kv tile << 4) |
+  // (class of query tile 1 << 2) | class of query tile 0.
+  int* sched_dump;
+  int64_t sched_dump_cap;
 };
 
 // Query rows per dense sequence held by q/out: the whole sequence, or one

@@ -432,6 +432,31 @@ ra_status ring_attn_status(void* stream);
  */
 int ring_attn_test_withhold_q(int on);
 
+/*
+ * ring_attn_test_dump_schedule -- test hook that makes the tensor-core
+ * forward's own schedule visible; leave it off (buf = NULL) in normal use.
+ * While set, every tensor-core forward launch made by this process
+ * (ring_attn_fwd, _gqa_fwd, _fwd_step, _qkvpacked_fwd, _fwd_noalloc, bf16 or
+ * fp16) appends, from the kernel's schedule-builder warp, one record of four
+ * int32 per visited key/value tile of 128 keys:
+ *     {sequence b, head h, query range qr, entry}
+ * where the work item (b, h, qr) is query rows [256 qr, 256 qr + 256) of
+ * sequence b (in a ring step: of the query block), and entry = (kv tile << 4)
+ * | (class of the item's second 128-row query tile << 2) | (class of its
+ * first), class 0 = EMPTY, 1 = FULL, 2 = PARTIAL; kv tile counts 128-key
+ * tiles from the sequence start (in a ring step: from the key block's
+ * start).  The records of one item appear in visit order.
+ *  buf       DEVICE int32 array of 4 + 4 * capacity elements; buf[0] counts
+ *            the records (atomically, also past capacity; only the first
+ *            capacity are stored from buf[4] on).  The caller zeroes buf[0]
+ *            before the launch and keeps buf alive while the hook is set.
+ *  capacity  records buf holds (>= 0).
+ * Host-only setting, read when a call builds its launch parameters.
+ * Returns RA_ERR_INVALID for a negative capacity or a NULL buf with
+ * capacity > 0 (the setting is unchanged then), RA_OK otherwise.
+ */
+ra_status ring_attn_test_dump_schedule(int32_t* buf, int64_t capacity);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* ring_attn_status_string(int status);
 

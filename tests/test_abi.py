@@ -223,3 +223,9 @@ def test_host_call_rejects_invalid_arguments_before_cuda(lib):
 
 def test_noalloc_status_is_exported_with_a_stream_argument(lib):
     assert lib.ring_attn_noalloc_status.argtypes == [ctypes.c_void_p]
+
+
+def test_schedule_dump_hook_validates_on_the_host(lib):
+    assert lib.ring_attn_test_dump_schedule(None, 5) == ra.RA_ERR_INVALID
+    assert lib.ring_attn_test_dump_schedule(FAKE, -1) == ra.RA_ERR_INVALID
+    assert lib.ring_attn_test_dump_schedule(None, 0) == ra.RA_OK   # off

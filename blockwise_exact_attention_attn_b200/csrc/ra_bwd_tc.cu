@@ -38,6 +38,7 @@
 #include <cuda_runtime.h>
 
 #include "ra_common.cuh"
+#include "ra_list.cuh"
 #include "ra_params.h"
 #include "ra_sched.h"
 #include "ra_work.cuh"
@@ -50,7 +51,6 @@ constexpr int QT = 2;     // query tiles per CTA
 constexpr int BN = 64;    // keys per kv tile
 constexpr int kThreads = 384;
 constexpr int kProducer = 8, kMma0 = 9, kBuilder = 10, kMma1 = 11;
-constexpr int kChunk = 16, kBufs = 16;
 constexpr int kConsumers = 11;  // producer, 2 issuers, 8 gradient warps
 constexpr int kStages = 2;      // (K, V) pairs in the ring
 constexpr int kRegsGrad = 184, kRegsControl = 136;  // 256*184 + 128*136 = 384*168
@@ -69,7 +69,7 @@ struct Cfg {
   static constexpr int kKVOff = kDOOff + QT * kQTile;  // slot s: K at +0, V at +kKTile
   static constexpr int kDSOff = kKVOff + kStages * 2 * kKTile;
   static constexpr int kListOff = kDSOff + QT * kDSBytes;
-  static constexpr int kCtrlOff = kListOff + kBufs * kChunk * 4;
+  static constexpr int kCtrlOff = kListOff + kListBufs * kListChunk * 4;
   static constexpr int kSmemBytes = kCtrlOff + 512 + 1024;
   static constexpr uint32_t kColS = 0;      // S_i at i * 64
   static constexpr uint32_t kColDP = 128;   // dP_i at 128 + i * 64
@@ -84,7 +84,7 @@ struct Ctrl {
   uint64_t s_full[QT], s_free[QT];
   uint64_t ds_full[QT], ds_done[QT];
   uint64_t dq_full[QT], dq_free[QT];
-  uint64_t list_full[kBufs], list_empty[kBufs];
+  uint64_t list_full[kListBufs], list_empty[kListBufs];
   uint64_t drain[QT];
   uint32_t tmem_base;
   int abort;
@@ -109,68 +109,8 @@ struct Params {
   float* dsum;      // D = <dO, O> per query row, lse layout (written by bwd_dq_kernel)
 };
 
-constexpr int kItemEnd = -1, kAllDone = -2, kPad = -3, kItemInfo = 5;
-__device__ __forceinline__ int item_header(int item) { return -(item + 8); }
 __device__ __forceinline__ int entry_tile(int e) { return e >> 4; }
 __device__ __forceinline__ int entry_cls(int e, int i) { return (e >> (2 * i)) & 3; }
-
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  const bool ok = mbar_wait(bar, parity, abort);
-  return __all_sync(0xffffffffu, ok);
-}
-
-struct ListReader {
-  const int* list;
-  uint64_t* full;
-  uint64_t* empty;
-  int n;
-  __device__ __forceinline__ bool next_raw(int* e, volatile int* abort) {
-    const int pos = n % kChunk, c = n / kChunk, b = c % kBufs;
-    if (pos == 0 && !mbar_wait(&full[b], (c / kBufs) & 1, abort)) return false;
-    *e = list[b * kChunk + pos];
-    ++n;
-    if (pos == kChunk - 1) mbar_arrive(&empty[b]);
-    return true;
-  }
-  __device__ __forceinline__ bool next_warp_raw(int* e, volatile int* abort) {
-    const int pos = n % kChunk, c = n / kChunk, b = c % kBufs;
-    if (pos == 0 && !warp_wait(&full[b], (c / kBufs) & 1, abort)) return false;
-    *e = list[b * kChunk + pos];
-    ++n;
-    if (pos == kChunk - 1) {
-      __syncwarp();
-      if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[b]);
-    }
-    return true;
-  }
-  __device__ __forceinline__ bool next(int* e, volatile int* abort) {
-    do {
-      if (!next_raw(e, abort)) return false;
-    } while (*e == kPad);
-    return true;
-  }
-  __device__ __forceinline__ bool next_warp(int* e, volatile int* abort) {
-    do {
-      if (!next_warp_raw(e, abort)) return false;
-    } while (*e == kPad);
-    return true;
-  }
-};
-
-template <bool kWarp>
-__device__ __forceinline__ bool read_item(ListReader& rd, SeqWork* it, volatile int* abort) {
-  int v[kItemInfo];
-#pragma unroll
-  for (int i = 0; i < kItemInfo; ++i)
-    if (!(kWarp ? rd.next_warp_raw(&v[i], abort) : rd.next_raw(&v[i], abort))) return false;
-  it->b = v[0];
-  it->qr = v[1];
-  it->h = v[2];
-  it->base = v[3];
-  it->L = v[4];
-  it->live = true;
-  return true;
-}
 
 // Leading allowed columns of kv tile [k0, k0 + nk) for query (rq, tq) when the
 // tile lies in ring block rk (allowed keys of one block form a prefix).
@@ -283,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ctrl->dq_free[i], BM);
       mbar_init(&ctrl->drain[i], 1);
     }
-    for (int b = 0; b < kBufs; ++b) {
+    for (int b = 0; b < kListBufs; ++b) {
       mbar_init(&ctrl->list_full[b], 1);
       mbar_init(&ctrl->list_empty[b], kConsumers);
     }
@@ -299,35 +239,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = ctrl->tmem_base;
   ListReader rd;
-  rd.list = list;
+  rd.list = smem_u32(list);
   rd.full = ctrl->list_full;
   rd.empty = ctrl->list_empty;
-  rd.n = 0;
 
   if (warp >= 8) {
     regs_dec<kRegsControl>();
     if (warp == kBuilder) {
       // ---------------------------------------------------------- schedule
-      int c = 0, pos = 0;
+      ListWriter wr;
+      wr.list = smem_u32(list);
+      wr.full = ctrl->list_full;
+      wr.empty = ctrl->list_empty;
+      wr.abort = abort_flag;
       bool ok = true;
-      auto put = [&](int v) -> bool {
-        const int b = c % kBufs;
-        if (pos == 0 && c >= kBufs &&
-            !mbar_wait(&ctrl->list_empty[b], ((c / kBufs) - 1) & 1, abort_flag))
-          return false;
-        list[b * kChunk + pos] = v;
-        if (++pos == kChunk) {
-          mbar_arrive(&ctrl->list_full[b]);
-          ++c;
-          pos = 0;
-        }
-        return true;
-      };
-      auto flush = [&]() -> bool {
-        bool f = true;
-        while (f && pos != 0) f = put(kPad);
-        return f;
-      };
+      auto put = [&](int v) -> bool { return wr.put(v); };
+      auto flush = [&]() -> bool { return wr.flush(); };
       int j = 0;
       while (ok) {
         if (claim_limit > 0 && j >= claim_limit) {
@@ -353,8 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int q0 = it.qr * kRows;
           const int qm = min(q0 + BM, it.L), q1 = min(q0 + kRows, it.L);
           const RingGeom g = make_geom(it.L, p.n_ring, p.layout, p.causal, p.passes);
-          ok = put(item_header(item)) && put(it.b) && put(it.qr) && put(it.h) &&
-               put(it.base) && put(it.L);
+          ok = put_item(wr, item, it);
           TileWalk walk;
           walk.init(g, q0, qm, q1, BN);
           int kt, c0, c1;
@@ -810,7 +736,7 @@ struct Cfg {
   static constexpr int kDSOff = kPOff + kPBytes;
   static constexpr int kVecOff = kDSOff + kPBytes;  // per slot: lse2[64], D[64]
   static constexpr int kListOff = kVecOff + kQStages * 2 * BQ * 4;
-  static constexpr int kCtrlOff = kListOff + kBufs * kChunk * 4;
+  static constexpr int kCtrlOff = kListOff + kListBufs * kListChunk * 4;
   static constexpr int kSmemBytes = kCtrlOff + 512 + 1024;
   static constexpr uint32_t kColS = 0, kColDP = 64, kColDV = 128, kColDK = 128 + D;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -823,7 +749,7 @@ struct Ctrl {
   uint64_t s_full, s_free;
   uint64_t pds_full, pds_done;
   uint64_t acc_full, acc_free;
-  uint64_t list_full[kBufs], list_empty[kBufs];
+  uint64_t list_full[kListBufs], list_empty[kListBufs];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -893,7 +819,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&ctrl->acc_full, 1);
     mbar_init(&ctrl->acc_free, 256);
     mbar_init(&ctrl->drain, 1);
-    for (int b = 0; b < kBufs; ++b) {
+    for (int b = 0; b < kListBufs; ++b) {
       mbar_init(&ctrl->list_full[b], 1);
       mbar_init(&ctrl->list_empty[b], kKvConsumers);
     }
@@ -909,10 +835,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = ctrl->tmem_base;
   ListReader rd;
-  rd.list = list;
+  rd.list = smem_u32(list);
   rd.full = ctrl->list_full;
   rd.empty = ctrl->list_empty;
-  rd.n = 0;
 
   if (warp >= 8) {
     regs_dec<kRegsControl>();
@@ -920,29 +845,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------- schedule
       // One item per CTA (grid = items): its header, then every query tile
       // that sees the key tile, with its class.
-      int c = 0, pos = 0;
+      ListWriter wr;
+      wr.list = smem_u32(list);
+      wr.full = ctrl->list_full;
+      wr.empty = ctrl->list_empty;
+      wr.abort = abort_flag;
       bool ok = true;
-      auto put = [&](int v) -> bool {
-        const int b = c % kBufs;
-        if (pos == 0 && c >= kBufs &&
-            !mbar_wait(&ctrl->list_empty[b], ((c / kBufs) - 1) & 1, abort_flag))
-          return false;
-        list[b * kChunk + pos] = v;
-        if (++pos == kChunk) {
-          mbar_arrive(&ctrl->list_full[b]);
-          ++c;
-          pos = 0;
-        }
-        return true;
-      };
+      auto put = [&](int v) -> bool { return wr.put(v); };
       const int item = blockIdx.x;
       const SeqWork it = find_work_item(p, BK, item);
       if (lane == 0) {
         if (it.live && item < n_items) {
           const int k_lo = it.qr * BK, k_hi = min(k_lo + BK, it.L);
           const RingGeom g = make_geom(it.L, p.n_ring, p.layout, p.causal, p.passes);
-          ok = put(item_header(item)) && put(it.b) && put(it.qr) && put(it.h) &&
-               put(it.base) && put(it.L);
+          ok = put_item(wr, item, it);
           const int nqt = (it.L + BQ - 1) / BQ;
           // every query head of the key/value head's group, in turn
           for (int gq = 0; ok && gq < p.kv_group; ++gq)
@@ -954,7 +870,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok) ok = put(kItemEnd);
         }
         if (ok) ok = put(kAllDone);
-        while (ok && pos != 0) ok = put(kPad);
+        if (ok) ok = wr.flush();
         if (!ok) {
           *abort_flag = 1;
           latch_status(p.status, ST_TIMEOUT);

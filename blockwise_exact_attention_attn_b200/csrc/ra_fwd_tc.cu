@@ -58,6 +58,7 @@
 #include <cuda_runtime.h>
 
 #include "ra_common.cuh"
+#include "ra_list.cuh"
 #include "ra_params.h"
 #include "ra_sched.h"
 #include "ra_work.cuh"
@@ -74,8 +75,6 @@ constexpr int kTcMmaWarp1 = 11;    // second MMA issuer when kTcIssuers == 2
 constexpr int kTcListWarp = 10;
 // MMA issuer warps: 2 = one per query tile, 1 = warp 9 issues for both tiles
 constexpr int kTcIssuers = 1;
-constexpr int kListChunk = 16;      // entries per schedule-list chunk (published at once)
-constexpr int kListBufs = 16;       // chunks in the shared-memory ring
 constexpr int kListConsumers = 9 + kTcIssuers;  // producer, issuers, 8 softmax warps
 // Register split.  Launch: 384 threads x 168 = 64512 registers.  After the
 // split: 256 softmax threads x 176 + 128 control threads x 152 = 64512.
@@ -140,14 +139,6 @@ __device__ __forceinline__ int single_block_limit(const RingGeom& g, int rq, int
   }
   const int lim = last - k0 + 1;
   return lim < 0 ? 0 : (lim > nk ? nk : lim);
-}
-
-// Warp-uniform bounded wait: every lane polls (one shared-memory request for
-// the warp) and the verdict is a vote -- measured 4-5 % faster than one lane
-// polling and broadcasting with a shuffle.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  const bool ok = mbar_wait(bar, parity, abort);
-  return __all_sync(0xffffffffu, ok);
 }
 
 // S = Q K^T for one query tile: M = 128 rows, N = 128 keys, K = D in steps of
@@ -222,84 +213,10 @@ __device__ __forceinline__ void apply_mask(float* x, const FwdParams& p, int L, 
   for (int c = 0; c < kTcBN; ++c) x[c] = ((mw[c >> 5] >> (c & 31)) & 1u) ? x[c] : -INFINITY;
 }
 
-// Schedule-list entries: (kt << 4) | (class of query tile 1 << 2) | class of
-// query tile 0 for a visited kv tile; kItemEnd ends a work item, kAllDone ends
-// the stream, kPad fills a chunk published early, and -(item + 8) starts work
-// item `item`.  A header is followed by kItemInfo entries describing the item
-// (sequence, query range, head, first row, length), decoded once by the
-// builder.  Chunks are released by every consumer after it read their last
-// entry.
-constexpr int kItemEnd = -1;
-constexpr int kAllDone = -2;
-constexpr int kPad = -3;
-constexpr int kItemInfo = 5;
-__device__ __forceinline__ int item_header(int item) { return -(item + 8); }
+// Schedule-list entries of an item (ra_list.cuh): (kt << 4) | (class of
+// query tile 1 << 2) | class of query tile 0 for a visited kv tile.
 __device__ __forceinline__ int entry_tile(int e) { return e >> 4; }
 __device__ __forceinline__ int entry_cls(int e, int i) { return (e >> (2 * i)) & 3; }
-
-// Sequential reader of the schedule list for a single thread (producer, MMA).
-struct ListReader {
-  const int* list;
-  uint64_t* full;
-  uint64_t* empty;
-  int n;
-  // Next entry other than padding into *e; false when a wait gave up.
-  __device__ __forceinline__ bool next(int* e, volatile int* abort) {
-    do {
-      if (!next_raw(e, abort)) return false;
-    } while (*e == kPad);
-    return true;
-  }
-  __device__ __forceinline__ bool next_warp(int* e, volatile int* abort) {
-    do {
-      if (!next_warp_raw(e, abort)) return false;
-    } while (*e == kPad);
-    return true;
-  }
-  __device__ __forceinline__ bool next_raw(int* e, volatile int* abort) {
-    const int pos = n % kListChunk;
-    const int c = n / kListChunk;
-    const int b = c % kListBufs;
-    if (pos == 0 && !mbar_wait(&full[b], (c / kListBufs) & 1, abort)) return false;
-    *e = list[b * kListChunk + pos];
-    ++n;
-    if (pos == kListChunk - 1) mbar_arrive(&empty[b]);
-    return true;
-  }
-  // Same for a whole warp: lane 0 waits and releases, every lane reads.
-  __device__ __forceinline__ bool next_warp_raw(int* e, volatile int* abort) {
-    const int pos = n % kListChunk;
-    const int c = n / kListChunk;
-    const int b = c % kListBufs;
-    if (pos == 0 && !warp_wait(&full[b], (c / kListBufs) & 1, abort)) return false;
-    *e = list[b * kListChunk + pos];
-    ++n;
-    if (pos == kListChunk - 1) {
-      __syncwarp();
-      if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[b]);
-    }
-    return true;
-  }
-};
-
-// The kItemInfo entries after a header, for one thread (kWarp false) or a
-// whole warp.
-template <bool kWarp>
-__device__ __forceinline__ bool read_item(ListReader& rd, SeqWork* it, volatile int* abort) {
-  int v[kItemInfo];
-#pragma unroll
-  for (int i = 0; i < kItemInfo; ++i) {
-    if (!(kWarp ? rd.next_warp_raw(&v[i], abort) : rd.next_raw(&v[i], abort)))
-      return false;
-  }
-  it->b = v[0];
-  it->qr = v[1];
-  it->h = v[2];
-  it->base = v[3];
-  it->L = v[4];
-  it->live = true;
-  return true;
-}
 
 template <int D, int kFmt>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -349,10 +266,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_after();
   const uint32_t tmem = ctrl->tmem_base;
   ListReader rd;
-  rd.list = list;
+  rd.list = smem_u32(list);
   rd.full = ctrl->list_full;
   rd.empty = ctrl->list_empty;
-  rd.n = 0;
 
   if (warp >= 8) {
    regs_dec<kRegsControl>();
@@ -362,27 +278,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // items come first in the item order), at most one item ahead of the
     // producer, and streams each item's header, ring-order visit list and
     // end marker, in chunks of kListChunk entries.
-    int c = 0, pos = 0;
+    ListWriter wr;
+    wr.list = smem_u32(list);
+    wr.full = ctrl->list_full;
+    wr.empty = ctrl->list_empty;
+    wr.abort = abort_flag;
     bool ok = true;
-    auto put = [&](int v) -> bool {
-      const int b = c % kListBufs;
-      if (pos == 0 && c >= kListBufs &&
-          !mbar_wait(&ctrl->list_empty[b], ((c / kListBufs) - 1) & 1, abort_flag))
-        return false;
-      list[b * kListChunk + pos] = v;
-      if (++pos == kListChunk) {
-        mbar_arrive(&ctrl->list_full[b]);
-        ++c;
-        pos = 0;
-      }
-      return true;
-    };
-    // publish the current chunk now (padded), so a waiting consumer sees it
-    auto flush = [&]() -> bool {
-      bool f = true;
-      while (f && pos != 0) f = put(kPad);
-      return f;
-    };
+    auto put = [&](int v) -> bool { return wr.put(v); };
+    auto flush = [&]() -> bool { return wr.flush(); };
     int j = 0;  // items emitted
     while (ok) {
       if (claim_limit > 0 && j >= claim_limit) {
@@ -411,8 +314,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int q0 = it.qr * kRows;
         const int qm = min(q0 + kTcBM, nrows), q1 = min(q0 + kRows, nrows);
         const RingGeom g = make_geom(it.L, p.n_ring, p.layout, p.causal, p.passes);
-        ok = put(item_header(item)) && put(it.b) && put(it.qr) && put(it.h) && put(it.base) &&
-             put(it.L);
+        ok = put_item(wr, item, it);
         int kt, c0, c1;
         // test hook: a record of each visited kv tile
         auto dump = [&](int entry) {

@@ -24,6 +24,7 @@ from ._binding import (  # noqa: F401
     ring_attn_func,
     ring_attn_func_host,
     ring_attn_fwd,
+    ring_attn_fwd_fp8,
     ring_attn_fwd_host,
     ring_attn_fwd_host_workspace,
     ring_attn_fwd_noalloc,

@@ -26,6 +26,7 @@ F32, BF16, F16 = 0, 1, 2
 EXPORTS = (
     "ring_attn_fwd",
     "ring_attn_gqa_fwd",
+    "ring_attn_fwd_fp8",
     "ring_attn_fwd_step",
     "ring_attn_bwd",
     "ring_attn_bwd_simt",
@@ -87,6 +88,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.ring_attn_bwd_simt.restype = _c_int
         lib.ring_attn_gqa_fwd.argtypes = _GQA_ARGS
         lib.ring_attn_gqa_fwd.restype = _c_int
+        lib.ring_attn_fwd_fp8.argtypes = _GQA_ARGS[:16] + [_c_float] * 3 + [_c_vp]
+        lib.ring_attn_fwd_fp8.restype = _c_int
         lib.ring_attn_fwd_simt.argtypes = _FWD_ARGS
         lib.ring_attn_fwd_simt.restype = _c_int
         lib.ring_attn_fwd_noalloc.argtypes = _FWD_ARGS
@@ -212,6 +215,28 @@ def ring_attn_gqa_fwd(q, k, v, out, lse, batch: int, heads: int, heads_kv: int, 
         _ptr(cu_seqlens, "cu_seqlens"), _dtype_code(q) if dtype is None else int(dtype),
         _stream(stream))
     _check("ring_attn_gqa_fwd", st)
+
+
+def ring_attn_fwd_fp8(q, k, v, out, lse, batch: int, heads: int, heads_kv: int, seqlen: int,
+                      d_head: int, n_ring_blocks: int, layout=CONTIGUOUS, causal: bool = False,
+                      softmax_scale: Optional[float] = None,
+                      max_ring_passes: Optional[int] = None, cu_seqlens=None,
+                      descale_q: float = 1.0, descale_k: float = 1.0, descale_v: float = 1.0,
+                      stream=None) -> None:
+    """Forward on e4m3 q/k/v (torch.float8_e4m3fn or uint8 tensors) with
+    per-tensor descale factors; out is bf16 (see ring_attn.h)."""
+    lib = load_library()
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d_head)
+    if max_ring_passes is None:
+        max_ring_passes = n_ring_blocks
+    st = lib.ring_attn_fwd_fp8(
+        _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _ptr(out, "out"), _ptr(lse, "lse"),
+        int(batch), int(heads), int(heads_kv), int(seqlen), int(d_head), int(n_ring_blocks),
+        _layout_code(layout), int(bool(causal)), float(softmax_scale), int(max_ring_passes),
+        _ptr(cu_seqlens, "cu_seqlens"), float(descale_q), float(descale_k), float(descale_v),
+        _stream(stream))
+    _check("ring_attn_fwd_fp8", st)
 
 
 def ring_attn_fwd_step(q, k, v, out, lse, batch: int, heads: int, seqlen: int, d_head: int,

@@ -131,6 +131,7 @@ ra::FwdParams make_params(const void* q, const void* k, const void* v, int64_t t
   p.passes = passes < n_ring ? passes : n_ring;
   p.scale = scale;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  p.out_scale = 1.f;
   p.n_qranges = 0;
   // heaviest query ranges first (the kernel launchers refine this per tile size)
   p.order = (causal && layout == RA_LAYOUT_CONTIGUOUS) ? 1 : 0;
@@ -350,6 +351,41 @@ ra_status ring_attn_gqa_fwd(const void* q, const void* k, const void* v, void* o
                              n_ring_blocks, layout, causal, softmax_scale, max_ring_passes,
                              cu_seqlens),
                  dtype, stream, false);
+}
+
+ra_status ring_attn_fwd_fp8(const void* q, const void* k, const void* v, void* out, float* lse,
+                            int batch, int heads, int heads_kv, int seqlen, int d_head,
+                            int n_ring_blocks, int layout, int causal, float softmax_scale,
+                            int max_ring_passes, const int32_t* cu_seqlens, float descale_q,
+                            float descale_k, float descale_v, void* stream) {
+  if (!q || !k || !v || !out || !lse) return RA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return RA_ERR_INVALID;
+  // the shape and mask checks of the 16-bit call
+  ra_status st = validate_fwd(batch, heads, heads_kv, seqlen, d_head, n_ring_blocks, layout,
+                              causal, softmax_scale, max_ring_passes, cu_seqlens, RA_BF16);
+  if (st != RA_OK) return st;
+  if (!std::isfinite(descale_q) || !std::isfinite(descale_k) || !std::isfinite(descale_v))
+    return RA_ERR_INVALID;
+  // the q and k descales fold into the score scale, v's into the output
+  const double sc = (double)softmax_scale * descale_q * descale_k;
+  if (!std::isfinite((float)sc)) return RA_ERR_INVALID;
+  if (d_head != 128 || (float)sc == 0.f) return RA_ERR_UNSUPPORTED;
+  ra::FwdParams p = make_params(q, k, v, (int64_t)heads * d_head, heads_kv,
+                                (int64_t)heads_kv * d_head, out, lse, batch, heads, seqlen,
+                                d_head, n_ring_blocks, layout, causal, (float)sc,
+                                max_ring_passes, cu_seqlens);
+  p.out_scale = descale_v;
+  int* status = nullptr;
+  st = device_state(&status, nullptr);
+  if (st != RA_OK) return st;
+  p.status = status;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  p.work_counter = next_counter(status);
+  if (cudaMemsetAsync(p.work_counter, 0, sizeof(int), s) != cudaSuccess) return RA_ERR_CUDA;
+  const cudaError_t e = ra::launch_fwd_tc(p, ra::kFmtE4M3, s);
+  if (e == cudaErrorInvalidValue) return RA_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
 ra_status ring_attn_fwd_simt(const void* q, const void* k, const void* v, void* out,

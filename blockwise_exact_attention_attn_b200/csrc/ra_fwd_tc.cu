@@ -83,12 +83,24 @@ constexpr int kRegsControl = 152;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 
-template <int D>
+// Element format traits: 16-bit (f16 / bf16, kind::f16 MMAs, K = 16 per
+// instruction) or 8-bit e4m3 (kind::f8f6f4, K = 32).
+template <int kFmt>
+struct TcFmt {
+  static constexpr bool kF8 = kFmt == kFmtE4M3;
+  static constexpr int kBytes = kF8 ? 1 : 2;       // bytes per element
+  static constexpr int kK = kF8 ? 32 : 16;         // K per MMA instruction
+  static constexpr int kPanelElems = 128 / kBytes; // elements per 128-byte row panel
+  // MMA format field: e4m3 is 0 under kind::f8f6f4; f16 0 and bf16 1 under kind::f16
+  static constexpr int kMmaFmt = kF8 ? 0 : kFmt;
+};
+
+template <int D, int kFmt = kFmtBF16>
 struct TcCfg {
-  static constexpr int kPanels = D / 64;                    // 128-byte swizzle panels
+  static constexpr int kPanels = D * TcFmt<kFmt>::kBytes / 128;  // 128-byte swizzle panels
   static constexpr int kPanelBytes = kTcBM * 128;           // 128 rows x 128 B
   static constexpr int kTileBytes = kPanels * kPanelBytes;  // one Q/K/V tile
-  static constexpr int kStages = D == 128 ? 5 : 10;         // K/V ring slots
+  static constexpr int kStages = kTileBytes >= 32768 ? 5 : 10;  // K/V ring slots
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = kTcQT * kTileBytes;
   static constexpr int kListOff = kKVOff + kStages * kTileBytes;
@@ -142,31 +154,43 @@ __device__ __forceinline__ int single_block_limit(const RingGeom& g, int rq, int
 }
 
 // S = Q K^T for one query tile: M = 128 rows, N = 128 keys, K = D in steps of
-// 16.  Both operands K-major in 128-byte-swizzled panels of 64 elements; the
-// descriptors of step kk are the tile's base descriptors plus a constant
-// (start address field, in 16-byte units: panel * 1024 + 2 * (kk % 4)).
-template <int D>
+// 32 bytes (16 16-bit or 32 8-bit elements).  Both operands K-major in
+// 128-byte-swizzled panels; the descriptors of step kk are the tile's base
+// descriptors plus a constant (start address field, in 16-byte units: panel
+// * 1024 + 2 * (kk % 4)).
+template <int D, int kFmt>
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t qdesc, uint64_t kdesc,
                                          uint32_t idesc) {
-  using C = TcCfg<D>;
+  using C = TcCfg<D, kFmt>;
+  using F = TcFmt<kFmt>;
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
+  for (int kk = 0; kk < D / F::kK; ++kk) {
     const uint64_t off = (uint64_t)((kk >> 2) * (C::kPanelBytes >> 4) + (kk & 3) * 2);
-    umma_ss(d_tmem, qdesc + off, kdesc + off, idesc, kk > 0 ? 1u : 0u);
+    if (F::kF8)
+      umma_ss_f8(d_tmem, qdesc + off, kdesc + off, idesc, kk > 0 ? 1u : 0u);
+    else
+      umma_ss(d_tmem, qdesc + off, kdesc + off, idesc, kk > 0 ? 1u : 0u);
   }
 }
 
-// O (+)= P V for one query tile: A = P from tensor memory (128 lanes x 64
-// columns, two 16-bit keys per column; 16 keys = 8 columns per step), B = V
-// tile MN-major (N = D split in 64-element panels, LBO = panel stride; 8-key
-// groups 1024 bytes apart).  Step kk covers 16 keys.
-template <int D>
+// O (+)= P V for one query tile: A = P from tensor memory (128 lanes, two
+// 16-bit or four 8-bit keys per column; one step's K keys are 8 columns), B
+// = V tile MN-major (N = D split in 128-byte panels, LBO = panel stride;
+// 8-key groups 1024 bytes apart).  Step kk covers K keys (16 or 32).
+template <int D, int kFmt>
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t vdesc,
                                          uint32_t idesc, bool accumulate) {
+  using F = TcFmt<kFmt>;
 #pragma unroll
-  for (int kk = 0; kk < kTcBN / 16; ++kk)
-    umma_ts(d_tmem, p_tmem + (uint32_t)(kk * 8), vdesc + (uint64_t)(kk * 128), idesc,
-            (accumulate || kk > 0) ? 1u : 0u);
+  for (int kk = 0; kk < kTcBN / F::kK; ++kk) {
+    const uint64_t voff = (uint64_t)(kk * F::kK * 8);  // K rows of 128 B, 16-byte units
+    if (F::kF8)
+      umma_ts_f8(d_tmem, p_tmem + (uint32_t)(kk * 8), vdesc + voff, idesc,
+                 (accumulate || kk > 0) ? 1u : 0u);
+    else
+      umma_ts(d_tmem, p_tmem + (uint32_t)(kk * 8), vdesc + voff, idesc,
+              (accumulate || kk > 0) ? 1u : 0u);
+  }
 }
 
 // Bits [lo, hi) of a 32-bit word, 0 <= lo < hi <= 32.
@@ -222,7 +246,8 @@ template <int D, int kFmt>
 __global__ void __launch_bounds__(kTcThreads, 1)
     fwd_tc_kernel(const FwdParams p, const __grid_constant__ TcMaps maps, int n_items,
                   int claim_limit) {
-  using C = TcCfg<D>;
+  using C = TcCfg<D, kFmt>;
+  using F = TcFmt<kFmt>;
   constexpr int kRows = kTcBM * kTcQT;  // query rows per work item
   constexpr int KVS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -377,7 +402,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint8_t* dst = smem + C::kKVOff + slot * C::kTileBytes;
       mbar_arrive_expect_tx(&ctrl->kv_full[slot], C::kTileBytes);
       for (int pn = 0; pn < C::kPanels; ++pn)
-        tma_load_3d(dst + pn * C::kPanelBytes, map, &ctrl->kv_full[slot], pn * 64, h, row);
+        tma_load_3d(dst + pn * C::kPanelBytes, map, &ctrl->kv_full[slot], pn * F::kPanelElems,
+                    h, row);
       ++n;
       return true;
     };
@@ -404,7 +430,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int i = 0; i < kTcQT; ++i)
             for (int pn = 0; pn < C::kPanels; ++pn)
               tma_load_3d(qs + i * C::kTileBytes + pn * C::kPanelBytes, &maps.q,
-                          &ctrl->q_full, pn * 64, it.h, it.base + q0 + i * kTcBM);
+                          &ctrl->q_full, pn * F::kPanelElems, it.h, it.base + q0 + i * kTcBM);
           ++nq;
         }
         if (ok && e >= 0) ok = load(&maps.v, hk, it.base + entry_tile(e) * kTcBN);
@@ -439,8 +465,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int i1 = kTcIssuers == 2 ? i0 + 1 : kTcQT;
     // a negative softmax scale is applied as S = (-Q) K^T times |scale|
     const uint32_t idesc_s =
-        idesc_f16kind_f32(kTcBM, kTcBN, 0, kFmt) | (p.scale_log2 < 0.f ? (1u << 13) : 0u);
-    constexpr uint32_t idesc_o = idesc_f16kind_f32(kTcBM, D, 1, kFmt);
+        idesc_f16kind_f32(kTcBM, kTcBN, 0, F::kMmaFmt) | (p.scale_log2 < 0.f ? (1u << 13) : 0u);
+    constexpr uint32_t idesc_o = idesc_f16kind_f32(kTcBM, D, 1, F::kMmaFmt);
     // base descriptors: K-major tiles (Q, K) and MN-major tiles (V)
     const uint64_t qdesc0 = smem_desc_sw128(smem_u32(smem + C::kQOff), 16, 1024);
     const uint64_t kdesc0 = smem_desc_sw128(smem_u32(smem + C::kKVOff), 16, 1024);
@@ -460,7 +486,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     };
     auto issue_s_tile = [&](int e, int i, int slot) {
       if (entry_cls(e, i) == CLS_EMPTY) return;
-      issue_qk<D>(tmem + C::kColS + i * kTcBN, qdesc0 + i * kQStep, kdesc0 + slot * kSlotStep,
+      issue_qk<D, kFmt>(tmem + C::kColS + i * kTcBN, qdesc0 + i * kQStep, kdesc0 + slot * kSlotStep,
                   idesc_s);
       umma_commit(&ctrl->s_full[i]);
       issued_any = true;
@@ -517,7 +543,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (!started[i]) wait_ofree(i);
                 if (!ok) break;
                 // an accumulating ring step adds to the O loaded from the state
-                issue_pv<D>(tmem + C::kColO + i * D, tmem + C::kColS + i * kTcBN,
+                issue_pv<D, kFmt>(tmem + C::kColO + i * D, tmem + C::kColS + i * kTcBN,
                             vdesc0 + slot_v * kSlotStep, idesc_o, started[i] || p.accumulate);
                 started[i] = true;
               }
@@ -667,7 +693,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // sums in paired fp32 instructions
         const uint64_t sc2 = f32x2_pack(sl2, sl2), ms2 = f32x2_pack(-msub, -msub);
         uint64_t sum2[2] = {0ull, 0ull};  // two independent (even, odd) partial sums
-        uint32_t pk[kTcBN / 2];
+        // P packed 2 (16-bit) or 4 (e4m3) keys per 32-bit column
+        constexpr int kPCols = kTcBN * F::kBytes / 4;
+        uint32_t pk[kPCols];
+        float pa = 0.f, pb = 0.f;  // e4m3: the even pair, packed with the odd one
 #pragma unroll
         for (int j = 0; j < kTcBN / 2; ++j) {
           float ya, yb;
@@ -675,12 +704,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const float a = ex2_approx(ya);
           const float b = ex2_approx(yb);
           sum2[j & 1] = fadd2(sum2[j & 1], a, b);
-          pk[j] = pack_x2<kFmt>(a, b);
+          if (F::kF8) {
+            if (j & 1)
+              pk[j >> 1] = pack_e4m3x4(pa, pb, a, b);
+            else
+              pa = a, pb = b;
+          } else {
+            pk[j] = pack_x2<kFmt>(a, b);
+          }
         }
         // P into tensor memory, over the scores just read (the previous PV of
         // this tile finished before this S was announced)
 #pragma unroll
-        for (int c = 0; c < kTcBN / 2; c += 32) RA_TMEM_ST32(tP + c, (pk + c));
+        for (int c = 0; c < kPCols; c += 32) RA_TMEM_ST32(tP + c, (pk + c));
         l = l * alpha + ((f32x2_lo(sum2[0]) + f32x2_hi(sum2[0])) +
                          (f32x2_lo(sum2[1]) + f32x2_hi(sum2[1])));
         if ((!first || from_state) && __any_sync(0xffffffffu, need)) {
@@ -708,7 +744,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_after();
       const int64_t orow_off = ((int64_t)(it.base + sq) * p.heads + it.h) * D;
       if (!first) {
-        const float inv_l = valid ? 1.f / l : 0.f;
+        const float inv_l = valid ? p.out_scale / l : 0.f;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
           uint32_t o[32];
@@ -728,8 +764,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             uint32_t pk[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              pk[j] = pack_x2<kFmt>(__uint_as_float(o[2 * j]) * inv_l,
-                                    __uint_as_float(o[2 * j + 1]) * inv_l);
+              pk[j] = pack_x2<F::kF8 ? kFmtBF16 : kFmt>(__uint_as_float(o[2 * j]) * inv_l,
+                                                       __uint_as_float(o[2 * j + 1]) * inv_l);
             if (valid) {
               uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + orow_off + c);
 #pragma unroll
@@ -798,12 +834,14 @@ static bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int heads,
                      int64_t tok_stride, int fmt) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
+  const int esz = fmt == kFmtE4M3 ? 1 : 2;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)tok_stride * 2};
-  cuuint32_t box[3] = {64, 1, (cuuint32_t)kTcBM};
+  cuuint64_t strides[2] = {(cuuint64_t)D * esz, (cuuint64_t)tok_stride * esz};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / esz), 1, (cuuint32_t)kTcBM};  // one 128-byte panel
   cuuint32_t estr[3] = {1, 1, 1};
-  const CUtensorMapDataType dt =
-      fmt == kFmtBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const CUtensorMapDataType dt = fmt == kFmtE4M3   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : fmt == kFmtBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                   : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUresult r = enc(map, dt, 3, const_cast<void*>(ptr), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -813,7 +851,7 @@ static bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int heads,
 
 template <int D, int kFmt>
 static cudaError_t launch_tc_t(const FwdParams& p, cudaStream_t stream) {
-  using C = TcCfg<D>;
+  using C = TcCfg<D, kFmt>;
   FwdParams pp = p;
   pp.n_qranges = (q_rows_per_seq(p) + kTcBM * kTcQT - 1) / (kTcBM * kTcQT);
   set_striped_order(pp, kTcBM * kTcQT);
@@ -854,7 +892,8 @@ static cudaError_t launch_tc_t(const FwdParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-// 16-bit inputs (fmt kFmtBF16 or kFmtF16), d_head 64 or 128.
+// 16-bit inputs (fmt kFmtBF16 or kFmtF16), d_head 64 or 128; e4m3 inputs
+// (kFmtE4M3) with d_head 128, not in ring-step mode.
 cudaError_t launch_fwd_tc(const FwdParams& p, int fmt, cudaStream_t stream) {
   if (fmt == kFmtBF16) {
     switch (p.d_head) {
@@ -866,6 +905,8 @@ cudaError_t launch_fwd_tc(const FwdParams& p, int fmt, cudaStream_t stream) {
       case 64: return launch_tc_t<64, kFmtF16>(p, stream);
       case 128: return launch_tc_t<128, kFmtF16>(p, stream);
     }
+  } else if (fmt == kFmtE4M3 && p.d_head == 128 && !p.step) {
+    return launch_tc_t<128, kFmtE4M3>(p, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -9,6 +9,8 @@ namespace ra {
 // (A and B always share one).
 constexpr int kFmtF16 = 0;
 constexpr int kFmtBF16 = 1;
+// 8-bit e4m3 inputs on kind::f8f6f4 MMAs (the output is bf16)
+constexpr int kFmtE4M3 = 2;
 
 // One forward call, in the form every forward kernel consumes.  Rows of all
 // sequences are addressed as one token axis: token row r of sequence b is
@@ -36,6 +38,7 @@ struct FwdParams {
   int qr_per_block;         // order 2: query ranges per ring block
   float scale;              // softmax scale
   float scale_log2;         // scale * log2(e)
+  float out_scale;          // multiplies O / l in the epilogue (1, or fp8's v descale)
   int* status;              // device status word (never NULL at launch)
   int* work_counter;        // persistent kernels: next work item (zeroed per launch)
   // Key/value-outer ring step (ring_attn_fwd_step): q, out and lse hold the

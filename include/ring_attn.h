@@ -71,6 +71,8 @@ typedef enum { RA_LAYOUT_CONTIGUOUS = 0, RA_LAYOUT_STRIPED = 1 } ra_layout;
  * lists fp16 and bf16 as the flash-attention input types; fp32 is the gist's
  * (and the fp32 workload's) type. */
 typedef enum { RA_F32 = 0, RA_BF16 = 1, RA_F16 = 2 } ra_dtype;
+/* (8-bit e4m3 inputs have their own entry point, ring_attn_fwd_fp8, because
+ * they come with scale factors.) */
 
 /*
  * ring_attn_fwd -- exact attention forward, ring-ordered blockwise.
@@ -156,6 +158,40 @@ ra_status ring_attn_gqa_fwd(const void* q, const void* k, const void* v,
                             float softmax_scale, int max_ring_passes,
                             const int32_t* cu_seqlens, int dtype,
                             void* stream);
+
+/*
+ * ring_attn_fwd_fp8 -- ring_attn_gqa_fwd for 8-bit e4m3 (fp8, "E4M3FN":
+ * 1 sign, 4 exponent, 3 mantissa bits, no infinities) q, k, v with one
+ * scale factor per tensor: the values are q = descale_q * q8, k = descale_k
+ * * k8, v = descale_v * v8.  The output is bf16.
+ *
+ * Source: "Tensorflow flash attention" page, which lists the input types
+ * flash attention takes (fp8 with bf16/fp16); the method is ring_attn_fwd's.
+ * The products run on the tensor cores in e4m3 (kind::f8f6f4, fp32
+ * accumulation): scores from q8 and k8 scaled by softmax_scale * descale_q
+ * * descale_k, and P = exp(s - m) rounded to e4m3 (round to nearest even;
+ * relative error at most 2^-4 for P >= 2^-6 relative to the running
+ * reference, absolute error at most 2^-10 below) before P V; l and lse use
+ * the unrounded P in fp32.
+ *
+ *  q         uint8 holding e4m3, dense [batch, seqlen, heads, 128], varlen
+ *            [seqlen, heads, 128].
+ *  k, v      e4m3 with heads_kv heads (a divisor of heads).
+ *  out       bf16, q's shape: descale_v * sum_j P_ij v8_j / l_i.
+ *  lse       float32, as ring_attn_fwd (of the scaled scores).
+ *  descale_q, descale_k, descale_v  finite per-tensor scale factors.
+ * Other arguments as ring_attn_gqa_fwd.  Errors as ring_attn_gqa_fwd, plus
+ * RA_ERR_INVALID for a non-finite descale (or a non-finite product with
+ * softmax_scale) and RA_ERR_UNSUPPORTED for d_head != 128 or a zero
+ * combined scale.
+ */
+ra_status ring_attn_fwd_fp8(const void* q, const void* k, const void* v,
+                            void* out, float* lse, int batch, int heads,
+                            int heads_kv, int seqlen, int d_head,
+                            int n_ring_blocks, int layout, int causal,
+                            float softmax_scale, int max_ring_passes,
+                            const int32_t* cu_seqlens, float descale_q,
+                            float descale_k, float descale_v, void* stream);
 
 /*
  * ring_attn_fwd_step -- one key/value-outer ring step: the queries of ring

@@ -715,30 +715,43 @@ static cudaError_t launch_t(const Params& bp_in, cudaStream_t stream, int num_sm
 
 namespace kv {
 
+// Key/value-outer kernel: one CTA per 128 keys of a (sequence, key/value
+// head), 128-query steps.  Per step t the tensor core computes
+//   S^T(t) = K Q(t)^T and dP^T(t) = V dO(t)^T     (M = 128 keys, N = 128)
+// into tensor memory; the gradient warps turn them into P^T and dS^T, which
+// they write as 16-bit over the scores they have read (two queries per
+// column); then
+//   dV += P^T(t) dO(t) and dK += dS^T(t) Q(t)     (A from tensor memory)
+// and S^T(t+1), dP^T(t+1) follow from the same issuing thread.  The tensor
+// core runs one thread's MMAs in issue order, so S^T(t+1) and dP^T(t+1)
+// overwrite the P^T(t), dS^T(t) columns only after dV and dK have read
+// them; the commit announcing S^T(t+1) also covers dV(t) and dK(t).
+// Gradient warp w works on key rows 32 (w % 4) .. + 31 (its TMEM lane
+// quadrant) and query columns 64 (w / 4) .. + 63; it writes P^T of its 64
+// queries into the first 32 columns of its own 64-column range, so the two
+// halves never overwrite scores the other has not read yet (each MMA step
+// takes its 16 queries' 8 columns from the half that holds them).
 constexpr int BK = 128;  // keys per CTA
-constexpr int BQ = 64;   // query rows per step
+constexpr int BQ = 128;  // query rows per step
 constexpr int kMma = 9;
 constexpr int kKvConsumers = 10;  // producer, issuer, 8 gradient warps
-constexpr int kQStages = 3;       // (Q, dO) pairs in the ring
+constexpr int kQStages = 2;       // (Q, dO) pairs in the ring
 
 template <int D>
 struct Cfg {
   static constexpr int kPanels = D / 64;
   static constexpr int kKPanel = BK * 128;      // 16 KB: 128 rows x 128 B
   static constexpr int kKTile = kPanels * kKPanel;
-  static constexpr int kQPanel = BQ * 128;      // 8 KB: 64 rows x 128 B
+  static constexpr int kQPanel = BQ * 128;      // 16 KB: 128 rows x 128 B
   static constexpr int kQTile = kPanels * kQPanel;
-  static constexpr int kPBytes = BK * BQ * 2;   // one 128-byte panel of 64 queries
   static constexpr int kKOff = 0;
   static constexpr int kVOff = kKOff + kKTile;
   static constexpr int kRingOff = kVOff + kKTile;  // slot s: Q at +0, dO at +kQTile
-  static constexpr int kPOff = kRingOff + kQStages * 2 * kQTile;
-  static constexpr int kDSOff = kPOff + kPBytes;
-  static constexpr int kVecOff = kDSOff + kPBytes;  // per slot: lse2[64], D[64]
+  static constexpr int kVecOff = kRingOff + kQStages * 2 * kQTile;  // per slot: lse2, D
   static constexpr int kListOff = kVecOff + kQStages * 2 * BQ * 4;
   static constexpr int kCtrlOff = kListOff + kListBufs * kListChunk * 4;
   static constexpr int kSmemBytes = kCtrlOff + 512 + 1024;
-  static constexpr uint32_t kColS = 0, kColDP = 64, kColDV = 128, kColDK = 128 + D;
+  static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(kColDK + D <= kTmemCols, "tensor memory budget");
 };
@@ -746,8 +759,7 @@ struct Cfg {
 struct Ctrl {
   uint64_t kv_full, kv_free;
   uint64_t q_full[kQStages], q_empty[kQStages];
-  uint64_t s_full, s_free;
-  uint64_t pds_full, pds_done;
+  uint64_t s_full, pds_full;
   uint64_t acc_full, acc_free;
   uint64_t list_full[kListBufs], list_empty[kListBufs];
   uint64_t drain;
@@ -765,8 +777,8 @@ __device__ __forceinline__ int entry_g(int e) { return e >> 24; }
 __device__ __forceinline__ int entry_qt(int e) { return (e >> 2) & 0x3fffff; }
 __device__ __forceinline__ int entry_cls(int e) { return e & 3; }
 
-// A (128 rows, panels kKPanel apart) x B (64 rows, panels kQPanel apart),
-// both K-major: M = 128, N = 64, K = D.
+// S^T-like product: A (128 key rows, K-major, panels kKPanel apart) x B
+// (128 query rows, K-major, panels kQPanel apart): M = N = 128, K = D.
 template <int D>
 __device__ __forceinline__ void issue_kq(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                          uint32_t idesc) {
@@ -779,14 +791,16 @@ __device__ __forceinline__ void issue_kq(uint32_t d_tmem, uint64_t adesc, uint64
   }
 }
 
-// acc (+)= A B: A = 128 x 64 K-major (one panel), B = 64-row tile MN-major
-// (N = D in panels kQPanel apart).  Step kk covers 16 queries.
-__device__ __forceinline__ void issue_acc(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+// acc (+)= A B with A (128 keys x 128 queries, 16-bit) in tensor memory --
+// queries 0-63 in columns [a, a + 32), 64-127 in [a + 64, a + 96) -- and B a
+// 128-query tile MN-major (N = D in panels kQPanel apart).  Step kk covers
+// 16 queries.
+__device__ __forceinline__ void issue_acc(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
                                           uint32_t idesc, bool accumulate) {
 #pragma unroll
   for (int kk = 0; kk < BQ / 16; ++kk)
-    umma_ss(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 128), idesc,
-            (accumulate || kk > 0) ? 1u : 0u);
+    umma_ts(d_tmem, a_tmem + (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8),
+            bdesc + (uint64_t)(kk * 128), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 template <int D, int kFmt>
@@ -813,9 +827,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ctrl->q_empty[s], 1);
     }
     mbar_init(&ctrl->s_full, 1);
-    mbar_init(&ctrl->s_free, 256);
     mbar_init(&ctrl->pds_full, 256);
-    mbar_init(&ctrl->pds_done, 1);
     mbar_init(&ctrl->acc_full, 1);
     mbar_init(&ctrl->acc_free, 256);
     mbar_init(&ctrl->drain, 1);
@@ -843,15 +855,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_dec<kRegsControl>();
     if (warp == kBuilder) {
       // ---------------------------------------------------------- schedule
-      // One item per CTA (grid = items): its header, then every query tile
-      // that sees the key tile, with its class.
+      // One item per CTA (grid = items): its header, then for every query
+      // head of the key/value head's group every query tile that sees the
+      // key tile, with its class.
       ListWriter wr;
       wr.list = smem_u32(list);
       wr.full = ctrl->list_full;
       wr.empty = ctrl->list_empty;
       wr.abort = abort_flag;
       bool ok = true;
-      auto put = [&](int v) -> bool { return wr.put(v); };
       const int item = blockIdx.x;
       const SeqWork it = find_work_item(p, BK, item);
       if (lane == 0) {
@@ -860,16 +872,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const RingGeom g = make_geom(it.L, p.n_ring, p.layout, p.causal, p.passes);
           ok = put_item(wr, item, it);
           const int nqt = (it.L + BQ - 1) / BQ;
-          // every query head of the key/value head's group, in turn
           for (int gq = 0; ok && gq < p.kv_group; ++gq)
             for (int qt = 0; ok && qt < nqt; ++qt) {
               const int q_lo = qt * BQ, q_hi = min(q_lo + BQ, it.L);
               const int cls = classify(g, q_lo, q_hi, k_lo, k_hi);
-              if (cls != CLS_EMPTY) ok = put((gq << 24) | (qt << 2) | cls);
+              if (cls != CLS_EMPTY) ok = wr.put((gq << 24) | (qt << 2) | cls);
             }
-          if (ok) ok = put(kItemEnd);
+          if (ok) ok = wr.put(kItemEnd);
         }
-        if (ok) ok = put(kAllDone);
+        if (ok) ok = wr.put(kAllDone);
         if (ok) ok = wr.flush();
         if (!ok) {
           *abort_flag = 1;
@@ -879,9 +890,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     } else if (warp == kProducer) {
       // ---------------------------------------------------------- producer
-      // The whole warp reads the list; per query tile its lanes stage the
-      // tile's lse (log2 units) and D into the slot's vectors, then lane 0
-      // arms the slot's barrier and issues the Q and dO copies.
+      // The whole warp reads the list.  Per query tile lane 0 issues the Q
+      // and dO copies, then the lanes stage the tile's lse (log2 units) and
+      // D into the slot's vectors and lane 0 arrives once more.
       if (lane == 0) {
         tma_prefetch_desc(&maps.k);
         tma_prefetch_desc(&maps.v);
@@ -934,7 +945,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           float* vec = reinterpret_cast<float*>(smem + C::kVecOff) + slot * 2 * BQ;
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
+          for (int u = 0; u < BQ / 32; ++u) {
             const int j = lane + 32 * u;
             const int qi = q_lo + j;
             float l2 = 0.f, dd = 0.f;
@@ -964,9 +975,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     } else if (warp == kMma) {
       // ---------------------------------------------------------- MMA issuer
-      // Per query tile t: S^T(t+1), dP^T(t+1) once the gradient warps have
-      // read S^T(t), dP^T(t) (s_free); then dV += P^T(t) dO(t), dK += dS^T(t)
-      // Q(t) once P^T(t), dS^T(t) are in shared memory (pds_full).
       const uint32_t idesc_s = idesc_f16kind_f32(BK, BQ, 0, kFmt);
       constexpr uint32_t idesc_a = idesc_f16kind_f32(BK, D, 1, kFmt);
       const uint64_t kdesc = smem_desc_sw128(smem_u32(smem + C::kKOff), 16, 1024);
@@ -976,12 +984,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t qmn0 = smem_desc_sw128(smem_u32(smem + C::kRingOff), C::kQPanel, 1024);
       const uint64_t domn0 =
           smem_desc_sw128(smem_u32(smem + C::kRingOff + C::kQTile), C::kQPanel, 1024);
-      const uint64_t pdesc = smem_desc_sw128(smem_u32(smem + C::kPOff), 16, 1024);
-      const uint64_t dsdesc = smem_desc_sw128(smem_u32(smem + C::kDSOff), 16, 1024);
       constexpr uint64_t kSlotStep = (uint64_t)((2 * C::kQTile) >> 4);
       const uint32_t tS = tmem + C::kColS, tDP = tmem + C::kColDP;
       const uint32_t tDV = tmem + C::kColDV, tDK = tmem + C::kColDK;
-      uint32_t ns = 0, npd = 0;
+      uint32_t npd = 0;
       int n = 0, k = 0;
       bool ok = true, issued_any = false;
       auto take = [&]() -> int {
@@ -992,15 +998,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         return slot;
       };
       auto issue_sdp = [&](int slot) {
-        if (ns > 0) {
-          ok = mbar_wait(&ctrl->s_free, (ns - 1) & 1, abort_flag);
-          if (!ok) return;
-          tc_fence_after();
-        }
         issue_kq<D>(tS, kdesc, qk0 + slot * kSlotStep, idesc_s);
         issue_kq<D>(tDP, vdesc, dok0 + slot * kSlotStep, idesc_s);
         umma_commit(&ctrl->s_full);
-        ++ns;
         issued_any = true;
       };
       while (ok) {
@@ -1024,15 +1024,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               int en = -1;
               ok = rd.next(&en, abort_flag);
               if (!ok) break;
-              int slot_n = -1;
-              if (en >= 0) {
-                slot_n = take();
-                if (!ok) break;
-                issue_sdp(slot_n);
-                if (!ok) break;
-              } else {
-                umma_commit(&ctrl->kv_free);  // every S^T/dP^T of this item issued
-              }
+              const int slot_n = en >= 0 ? take() : -1;
+              if (!ok) break;
+              if (en < 0) umma_commit(&ctrl->kv_free);  // every use of K, V is issued
               ok = mbar_wait(&ctrl->pds_full, npd & 1, abort_flag);
               if (!ok) break;
               tc_fence_after();
@@ -1041,14 +1035,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 tc_fence_after();
               }
-              issue_acc(tDV, pdesc, domn0 + slot * kSlotStep, idesc_a, started);
-              issue_acc(tDK, dsdesc, qmn0 + slot * kSlotStep, idesc_a, started);
-              umma_commit(&ctrl->pds_done);
+              issue_acc(tDV, tS, domn0 + slot * kSlotStep, idesc_a, started);
+              issue_acc(tDK, tDP, qmn0 + slot * kSlotStep, idesc_a, started);
               umma_commit(&ctrl->q_empty[slot]);
               ++npd;
               started = true;
               if (en < 0) break;
-              e = en;
+              // in issue order after dV and dK, which read P^T and dS^T
+              issue_sdp(slot_n);
               slot = slot_n;
             }
           } else if (ok) {
@@ -1078,16 +1072,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     regs_inc<kRegsGrad>();
     // ---------------------------------------------------------- gradient warps
-    const int half = warp >> 2;           // query columns [32 half, 32 half + 32)
+    const int half = warp >> 2;           // query columns [64 half, 64 half + 64)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;       // key row of the tile
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::kColS + half * 32;
-    const uint32_t tDP = tmem + lane_off + C::kColDP + half * 32;
-    const uint32_t prow = smem_u32(smem + C::kPOff) + (uint32_t)r * 128u;
-    const uint32_t dsrow = smem_u32(smem + C::kDSOff) + (uint32_t)r * 128u;
-    const uint32_t swz = (uint32_t)(r & 7);
-    uint32_t sphase = 0, npd = 0;
+    const uint32_t tS = tmem + lane_off + C::kColS + half * 64;
+    const uint32_t tDP = tmem + lane_off + C::kColDP + half * 64;
+    uint32_t sphase = 0;
     int k = 0, nstep = 0;
     bool ok = true;
     while (true) {
@@ -1109,83 +1100,72 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int cls = entry_cls(e);
         const int q_lo = entry_qt(e) * BQ;
         const int slot = nstep % kQStages;
-        // the slot's lse / D vectors were written before its barrier was armed
+        // the slot's lse / D vectors were written before its second arrival
         ok = warp_wait(&ctrl->q_full[slot], (nstep / kQStages) & 1, abort_flag);
         if (!ok) break;
         const float* vec = reinterpret_cast<const float*>(smem + C::kVecOff) + slot * 2 * BQ;
         ++nstep;
+        // S^T(t), dP^T(t) computed; dV and dK of the previous step done
         ok = warp_wait(&ctrl->s_full, sphase, abort_flag);
         sphase ^= 1;
         if (!ok) break;
         tc_fence_after();
-        float s[32], dp[32];
-        {
-          uint32_t* sr = reinterpret_cast<uint32_t*>(s);
-          uint32_t* dr = reinterpret_cast<uint32_t*>(dp);
-          RA_TMEM_LD32(tS, sr);
-          RA_TMEM_LD32(tDP, dr);
-          tmem_wait_ld();
-        }
-        tc_fence_before();
-        mbar_arrive(&ctrl->s_free);
-        // this half's 32 query columns: lse (log2 units) and D, read as
-        // vectors from shared memory before any arithmetic
-        float l2[32], dd[32];
-        {
-          const uint32_t va = smem_u32(vec + half * 32), vb = smem_u32(vec + BQ + half * 32);
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            ld_shared_f4(va + 16u * u, l2[4 * u], l2[4 * u + 1], l2[4 * u + 2], l2[4 * u + 3]);
-            ld_shared_f4(vb + 16u * u, dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
-          }
-        }
-        // allowed query columns of this key row as a bit word
-        const int qc = q_lo + half * 32;  // first query column of this half
-        uint32_t am = 0u;
-        if (kvalid) {
-          const int nq = min(max(L - qc, 0), 32);
-          am = nq >= 32 ? 0xffffffffu : ((1u << nq) - 1u);
-          if (cls == CLS_PARTIAL) {
-            uint32_t bits = 0u;
-            for (int j = 0; j < nq; ++j) {
-              const int qi = qc + j;
-              const int rq = block_of(g, qi);
-              if (allowed(g, qi, rq, token_of(g, qi, rq), sk)) bits |= 1u << j;
+        for (int c = 0; c < 2; ++c) {
+          // 32 query columns: scores and dP^T, then lse (log2 units) and D
+          float s[32], dp[32], l2[32], dd[32];
+          {
+            uint32_t* sr = reinterpret_cast<uint32_t*>(s);
+            uint32_t* dr = reinterpret_cast<uint32_t*>(dp);
+            RA_TMEM_LD32(tS + c * 32, sr);
+            RA_TMEM_LD32(tDP + c * 32, dr);
+            const int q0 = half * 64 + c * 32;
+            const uint32_t va = smem_u32(vec + q0), vb = smem_u32(vec + BQ + q0);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              ld_shared_f4(va + 16u * u, l2[4 * u], l2[4 * u + 1], l2[4 * u + 2], l2[4 * u + 3]);
+              ld_shared_f4(vb + 16u * u, dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
             }
-            am &= bits;
+            tmem_wait_ld();
           }
-        }
-        uint32_t pp[16], pd[16];
-#pragma unroll
-        for (int j2 = 0; j2 < 16; ++j2) {
-          float pv[2], dv2[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int j = 2 * j2 + u;
-            const float pj = ex2_approx(fmaf(s[j], p.scale_log2, -l2[j]));
-            const bool a = (am >> j) & 1u;
-            pv[u] = a ? pj : 0.f;
-            dv2[u] = a ? pj * (dp[j] - dd[j]) : 0.f;
+          // allowed query columns of this key row as a bit word
+          const int qc = q_lo + half * 64 + c * 32;
+          uint32_t am = 0u;
+          if (kvalid) {
+            const int nq = min(max(L - qc, 0), 32);
+            am = nq >= 32 ? 0xffffffffu : ((1u << nq) - 1u);
+            if (cls == CLS_PARTIAL) {
+              uint32_t bits = 0u;
+              for (int j = 0; j < nq; ++j) {
+                const int qi = qc + j;
+                const int rq = block_of(g, qi);
+                if (allowed(g, qi, rq, token_of(g, qi, rq), sk)) bits |= 1u << j;
+              }
+              am &= bits;
+            }
           }
-          pp[j2] = pack_x2<kFmt>(pv[0], pv[1]);
-          pd[j2] = pack_x2<kFmt>(dv2[0], dv2[1]);
-        }
-        // the previous dV/dK MMAs have read P^T, dS^T
-        if (npd > 0) {
-          ok = warp_wait(&ctrl->pds_done, (npd - 1) & 1, abort_flag);
-          if (!ok) break;
-        }
+          uint32_t pp[16], pd[16];
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const uint32_t chunk = ((uint32_t)(half * 4 + c4) ^ swz) << 4;
-          st_shared_v4(prow + chunk, pp[4 * c4], pp[4 * c4 + 1], pp[4 * c4 + 2], pp[4 * c4 + 3]);
-          st_shared_v4(dsrow + chunk, pd[4 * c4], pd[4 * c4 + 1], pd[4 * c4 + 2],
-                       pd[4 * c4 + 3]);
+          for (int j2 = 0; j2 < 16; ++j2) {
+            float pv[2], dv2[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int j = 2 * j2 + u;
+              const float pj = ex2_approx(fmaf(s[j], p.scale_log2, -l2[j]));
+              const bool a = (am >> j) & 1u;
+              pv[u] = a ? pj : 0.f;
+              dv2[u] = a ? pj * (dp[j] - dd[j]) : 0.f;
+            }
+            pp[j2] = pack_x2<kFmt>(pv[0], pv[1]);
+            pd[j2] = pack_x2<kFmt>(dv2[0], dv2[1]);
+          }
+          // over the columns this warp has already read
+          RA_TMEM_ST16(tS + c * 16, pp);
+          RA_TMEM_ST16(tDP + c * 16, pd);
         }
-        fence_proxy_async_smem();
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&ctrl->pds_full);
-        ++npd;
         any = true;
       }
       if (!ok) break;
@@ -1236,7 +1216,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem, kTmemCols);
   }
 }
-
 
 template <int D, int kFmt>
 static cudaError_t launch_t(const Params& bp_in, cudaStream_t stream) {

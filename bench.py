@@ -51,7 +51,8 @@ L2_BYTES = 126 * 1024 * 1024
 DATASHEET_BF16_TFLOPS = 2250.0
 DATASHEET_HBM_GBS = 8000.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-TC_SOURCES = ["ra_fwd_tc.cu", "ra_common.cuh", "ra_sched.h", "ra_work.cuh", "ra_params.h"]
+TC_SOURCES = ["ra_fwd_tc.cu", "ra_common.cuh", "ra_list.cuh", "ra_sched.h", "ra_work.cuh",
+              "ra_params.h"]
 
 
 # ----------------------------------------------------------------------------- infra

@@ -872,8 +872,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const RingGeom g = make_geom(it.L, p.n_ring, p.layout, p.causal, p.passes);
           ok = put_item(wr, item, it);
           const int nqt = (it.L + BQ - 1) / BQ;
+          // contiguous causal: the query tiles that end before the first key
+          // see none of it (query and key positions are the stored rows), so
+          // the walk starts at the tile that holds row k_lo; every other
+          // tile is classified exactly (a few divisions per call, which the
+          // leading empty tiles would otherwise spend before the first entry)
+          const int qt0 = (g.causal && g.layout == LAYOUT_CONTIGUOUS) ? k_lo / BQ : 0;
           for (int gq = 0; ok && gq < p.kv_group; ++gq)
-            for (int qt = 0; ok && qt < nqt; ++qt) {
+            for (int qt = qt0; ok && qt < nqt; ++qt) {
               const int q_lo = qt * BQ, q_hi = min(q_lo + BQ, it.L);
               const int cls = classify(g, q_lo, q_hi, k_lo, k_hi);
               if (cls != CLS_EMPTY) ok = wr.put((gq << 24) | (qt << 2) | cls);

@@ -289,6 +289,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // Ring steps are launched as programmatic dependents of the previous
+  // launch on the stream: the next step's CTAs may be placed on SMs this
+  // launch has finished with and run their set-up (barriers, tensor memory)
+  // while its last CTAs finish.  The launch before may have written any of
+  // the inputs (q, k, v, cu_seqlens, the running out and lse), so no thread
+  // reads global memory before griddepcontrol.wait has returned, which is
+  // after that launch has completed and its writes are visible.
+  if (p.step) {
+    if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+  }
   const uint32_t tmem = ctrl->tmem_base;
   ListReader rd;
   rd.list = smem_u32(list);
@@ -311,7 +322,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool ok = true;
     auto put = [&](int v) -> bool { return wr.put(v); };
     auto flush = [&]() -> bool { return wr.flush(); };
-    int j = 0;  // items emitted
+    int j = 0;       // items emitted
+    int claims = 0;  // items claimed (emitted or skipped)
     while (ok) {
       if (claim_limit > 0 && j >= claim_limit) {
         if (lane == 0) ok = put(kAllDone) && flush();
@@ -322,8 +334,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // item j-1 has started (its Q landed) before another item is claimed
         if (ok) ok = mbar_wait(&ctrl->q_full, (j - 1) & 1, abort_flag);
       }
-      int item = 0;
-      if (lane == 0 && ok) item = atomicAdd(p.work_counter, 1);
+      // the launch's counter hands out items; without one (ring steps,
+      // whose items are all alike) CTA c takes items c, c + grid, ...
+      int item = blockIdx.x + claims * (int)gridDim.x;
+      ++claims;
+      if (lane == 0 && ok && p.work_counter) item = atomicAdd(p.work_counter, 1);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       item = __shfl_sync(0xffffffffu, item, 0);
       if (!ok) break;
@@ -362,12 +377,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         } else {
           // one ring step: the tiles of key/value block kv_block (tile-aligned
-          // blocks; kt counts tiles inside the block)
+          // blocks; kt counts tiles inside the block).  The item's query rows
+          // all lie in ring block q_block and every key tile in kv_block, so
+          // a tile's class is that of one segment pair: no block lookups (the
+          // general classify() divides by the block geometry several times
+          // per call, which at one thread paced the whole step).
           const int qo = p.q_block * p.step_rows, ko = p.kv_block * p.step_rows;
+          auto seg_class = [&](int a, int b, int c) -> int {
+            if (a >= b) return CLS_EMPTY;
+            bool any = false, all = true;
+            classify_segment(g, p.q_block, a, b, p.kv_block, c, c + kTcBN, &any, &all);
+            return any ? (all ? CLS_FULL : CLS_PARTIAL) : CLS_EMPTY;
+          };
           for (kt = 0; ok && kt < p.step_rows / kTcBN; ++kt) {
             const int k0 = ko + kt * kTcBN;
-            c0 = classify(g, qo + q0, qo + qm, k0, k0 + kTcBN);
-            c1 = classify(g, qo + qm, qo + q1, k0, k0 + kTcBN);
+            c0 = seg_class(qo + q0, qo + qm, k0);
+            c1 = seg_class(qo + qm, qo + q1, k0);
             if (c0 != CLS_EMPTY || c1 != CLS_EMPTY) {
               dump((kt << 4) | (c1 << 2) | c0);
               ok = put((kt << 4) | (c1 << 2) | c0);
@@ -630,22 +655,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           m_ref = lp * 1.4426950408889634f;
           l = 1.f;
         }
-        const float* orow = static_cast<const float*>(p.out) +
-                            ((int64_t)(it.base + sq) * p.heads + it.h) * D;
+        const float4* orow = reinterpret_cast<const float4*>(
+            static_cast<const float*>(p.out) + ((int64_t)(it.base + sq) * p.heads + it.h) * D);
+        // every load of the row is issued before the first tensor-memory
+        // store (a store orders the loads after it)
+        uint32_t o[D];
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t o[32];
-#pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            const float4 f = has ? *reinterpret_cast<const float4*>(orow + c + j)
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-            o[j] = __float_as_uint(f.x);
-            o[j + 1] = __float_as_uint(f.y);
-            o[j + 2] = __float_as_uint(f.z);
-            o[j + 3] = __float_as_uint(f.w);
-          }
-          RA_TMEM_ST32(tO + c, o);
+        for (int j = 0; j < D / 4; ++j) {
+          const float4 f = has ? orow[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+          o[4 * j] = __float_as_uint(f.x);
+          o[4 * j + 1] = __float_as_uint(f.y);
+          o[4 * j + 2] = __float_as_uint(f.z);
+          o[4 * j + 3] = __float_as_uint(f.w);
         }
+#pragma unroll
+        for (int c = 0; c < D; c += 32) RA_TMEM_ST32(tO + c, (o + c));
         tmem_wait_st();
       }
 
@@ -873,8 +897,10 @@ static cudaError_t launch_tc_t(const FwdParams& p, cudaStream_t stream) {
   }
   // Dense causal work varies per item: one CTA per item, balanced by the
   // hardware block scheduler, measured faster than persistent CTAs there.
-  // Otherwise (and for ring steps, whose items are short) persistent CTAs
-  // (one per SM) claim items until none is left.
+  // Otherwise persistent CTAs (one per SM) claim items until none is left:
+  // from the launch's counter, or for ring steps (launched as programmatic
+  // dependents of the previous launch, with no counter reset between) by a
+  // static stride over the CTAs.
   const bool per_item = p.causal && !p.cu_seqlens && !p.step;
   const int64_t grid = per_item ? items : (items < num_sms ? items : num_sms);
   const int claim_limit = per_item ? 1 : 0;
@@ -887,6 +913,19 @@ static cudaError_t launch_tc_t(const FwdParams& p, cudaStream_t stream) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;
+  if (p.step) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, fwd_tc_kernel<D, kFmt>, pp, maps, (int)items, claim_limit);
+  }
   fwd_tc_kernel<D, kFmt><<<(unsigned)grid, kTcThreads, C::kSmemBytes, stream>>>(
       pp, maps, (int)items, claim_limit);
   return cudaGetLastError();

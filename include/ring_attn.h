@@ -228,6 +228,10 @@ ra_status ring_attn_fwd_fp8(const void* q, const void* k, const void* v,
  * range or accumulate not in {0,1}; RA_ERR_UNSUPPORTED for RA_F32, a zero
  * scale, or a block size seqlen / n_ring_blocks that is not a multiple of
  * 128 (the step runs on the tensor cores with whole tiles per block).
+ * Launch: one persistent thread block per SM, as a programmatic dependent of
+ * the launch before it on the stream, so that its set-up overlaps that
+ * launch's last blocks; it reads no input before that launch has completed,
+ * so ordering on the stream is the same as for any kernel.
  */
 ra_status ring_attn_fwd_step(const void* q, const void* k, const void* v,
                              float* out, float* lse, int batch, int heads,

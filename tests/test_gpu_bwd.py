@@ -160,3 +160,20 @@ def test_dq_of_rows_that_never_see_a_key_block_is_bitwise_unchanged():
         dqs.append(dq)
     rows = 3 * S // 4
     assert torch.equal(dqs[0][:rows], dqs[1][:rows])
+
+
+def test_backward_at_the_benchmark_size_on_two_heads():
+    # the benchmark's backward workload (bf16 1x8x8192x128 causal, 8 ring
+    # blocks) in the launch configuration bench.py times; the oracle's
+    # gradients of the first and last head (a whole head: dk and dv need
+    # every query row that sees a key)
+    B, H, S, D, N = 1, 8, 8192, 128, 8
+    w = gen.Workload("bwd_bench", "bf16", B, H, S, D, True, N, 0, N, seed=960)
+    inp = gen.make_inputs(w)
+    dout = torch.randn(B, S, H, D, generator=torch.Generator().manual_seed(961))
+    dout = dout.to(torch.bfloat16)
+    got = run_bwd(w, inp, dout)
+    heads = [0, H - 1]
+    ref = oracle.attention_backward(problem_for(w, inp, heads=heads),
+                                    dout.reshape(S, H, D)[:, heads].double().numpy())
+    check_grads(w, tuple(g[:, heads] for g in got), ref)

@@ -141,10 +141,15 @@ __device__ __forceinline__ void tile_mask(uint32_t mw[2], const FwdParams& p, in
     mw[0] = mw[1] = 0u;
     return;
   }
-  if (cls == CLS_FULL) {
+  // causal rows of the contiguous layout without a pass limit see every
+  // stored key up to their own position tq: one interval, no block lookups
+  const bool prefix =
+      cls == CLS_FULL || (p.causal && p.layout == LAYOUT_CONTIGUOUS && p.passes >= p.n_ring);
+  if (prefix) {
+    const int lim = cls == CLS_FULL ? nk : min(nk, tq - k0 + 1);
 #pragma unroll
     for (int w = 0; w < 2; ++w) {
-      const int n = min(max(nk - 32 * w, 0), 32);
+      const int n = min(max(lim - 32 * w, 0), 32);
       mw[w] = n >= 32 ? 0xffffffffu : ((1u << n) - 1u);
     }
     return;
@@ -1142,10 +1147,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             am = nq >= 32 ? 0xffffffffu : ((1u << nq) - 1u);
             if (cls == CLS_PARTIAL) {
               uint32_t bits = 0u;
-              for (int j = 0; j < nq; ++j) {
-                const int qi = qc + j;
-                const int rq = block_of(g, qi);
-                if (allowed(g, qi, rq, token_of(g, qi, rq), sk)) bits |= 1u << j;
+              if (p.causal && p.layout == LAYOUT_CONTIGUOUS && p.passes >= p.n_ring) {
+                // contiguous causal, no pass limit: the queries at or after
+                // the key's own position
+                const int lo = sk - qc;
+                bits = lo <= 0 ? 0xffffffffu : (lo >= 32 ? 0u : ~((1u << lo) - 1u));
+              } else {
+                for (int j = 0; j < nq; ++j) {
+                  const int qi = qc + j;
+                  const int rq = block_of(g, qi);
+                  if (allowed(g, qi, rq, token_of(g, qi, rq), sk)) bits |= 1u << j;
+                }
               }
               am &= bits;
             }

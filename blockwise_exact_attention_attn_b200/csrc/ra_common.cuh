@@ -270,6 +270,39 @@ __host__ __device__ constexpr uint32_t idesc_f16kind_f32(int M, int N, int b_mn_
       "r"(r[14]), "r"(r[15])                                                            \
       : "memory")
 
+// 16 lanes x 256 bit, repeated over 8 column groups (64 columns): the
+// shape of the m16n8 accumulator fragment.  Thread t holds, for group g,
+// r[4g], r[4g+1] = lane t/4, columns 8g + 2(t%4) + {0, 1}, and r[4g+2],
+// r[4g+3] = lane t/4 + 8, same columns (lanes relative to the address's
+// lane field, a multiple of 16 inside the warp's quadrant).  Four threads
+// then cover 32 contiguous bytes of a row, which makes row-major global
+// loads and stores of fp32 rows whole 32-byte sectors.
+#define RA_TMEM_LD256X8(taddr, r)                                                       \
+  asm volatile(                                                                         \
+      "tcgen05.ld.sync.aligned.16x256b.x8.b32 "                                         \
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"                         \
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"        \
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),         \
+        "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),       \
+        "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]),   \
+        "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),   \
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),   \
+        "=r"(r[30]), "=r"(r[31])                                                        \
+      : "r"(taddr)                                                                      \
+      : "memory")
+
+#define RA_TMEM_ST256X8(taddr, r)                                                       \
+  asm volatile(                                                                         \
+      "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], "                                   \
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"                        \
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr), \
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),     \
+      "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),  \
+      "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]),           \
+      "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]),           \
+      "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])            \
+      : "memory")
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }

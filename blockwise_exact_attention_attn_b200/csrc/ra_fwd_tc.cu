@@ -655,21 +655,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           m_ref = lp * 1.4426950408889634f;
           l = 1.f;
         }
-        const float4* orow = reinterpret_cast<const float4*>(
-            static_cast<const float*>(p.out) + ((int64_t)(it.base + sq) * p.heads + it.h) * D);
-        // every load of the row is issued before the first tensor-memory
-        // store (a store orders the loads after it)
-        uint32_t o[D];
+        // The warp's 32 rows are loaded together in the 16x256b fragment
+        // shape: four threads read 32 contiguous bytes of one row (whole
+        // sectors), where a thread per row would touch a line per thread.
+        // Every load is issued before the first tensor-memory store.
+        const float* obase = static_cast<const float*>(p.out) +
+                             ((int64_t)(it.base + sq - lane) * p.heads + it.h) * D;
+        const int64_t rstride = (int64_t)p.heads * D;
+        uint32_t o[2][D / 2];
 #pragma unroll
-        for (int j = 0; j < D / 4; ++j) {
-          const float4 f = has ? orow[j] : make_float4(0.f, 0.f, 0.f, 0.f);
-          o[4 * j] = __float_as_uint(f.x);
-          o[4 * j + 1] = __float_as_uint(f.y);
-          o[4 * j + 2] = __float_as_uint(f.z);
-          o[4 * j + 3] = __float_as_uint(f.w);
+        for (int hf = 0; hf < 2; ++hf) {
+          const int ra = 16 * hf + (lane >> 2), rb = ra + 8;  // rows of the warp
+          const bool ha = __shfl_sync(0xffffffffu, has ? 1 : 0, ra) != 0;
+          const bool hb = __shfl_sync(0xffffffffu, has ? 1 : 0, rb) != 0;
+#pragma unroll
+          for (int g = 0; g < D / 8; ++g) {
+            const int col = 8 * g + 2 * (lane & 3);
+            const float2 fa = ha ? *reinterpret_cast<const float2*>(obase + ra * rstride + col)
+                                 : make_float2(0.f, 0.f);
+            const float2 fb = hb ? *reinterpret_cast<const float2*>(obase + rb * rstride + col)
+                                 : make_float2(0.f, 0.f);
+            o[hf][4 * g] = __float_as_uint(fa.x);
+            o[hf][4 * g + 1] = __float_as_uint(fa.y);
+            o[hf][4 * g + 2] = __float_as_uint(fb.x);
+            o[hf][4 * g + 3] = __float_as_uint(fb.y);
+          }
         }
 #pragma unroll
-        for (int c = 0; c < D; c += 32) RA_TMEM_ST32(tO + c, (o + c));
+        for (int hf = 0; hf < 2; ++hf) {
+          const uint32_t th = tO + ((uint32_t)(16 * hf) << 16);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) RA_TMEM_ST256X8(th + 64 * c, (o[hf] + 32 * c));
+        }
         tmem_wait_st();
       }
 
@@ -767,35 +784,55 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const int64_t orow_off = ((int64_t)(it.base + sq) * p.heads + it.h) * D;
-      if (!first) {
+      if (!first && p.step) {
+        // ring step: the running output stays fp32, written by the warp's
+        // threads together in the 16x256b fragment shape (32 contiguous
+        // bytes of a row per four threads, as the state was loaded)
+        const float inv_l = valid ? p.out_scale / l : 0.f;
+        float* obase = static_cast<float*>(p.out) + orow_off - (int64_t)lane * p.heads * D;
+        const int64_t rstride = (int64_t)p.heads * D;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int ra = 16 * hf + (lane >> 2), rb = ra + 8;  // rows of the warp
+          const float ia = __shfl_sync(0xffffffffu, inv_l, ra);
+          const float ib = __shfl_sync(0xffffffffu, inv_l, rb);
+          const bool va = __shfl_sync(0xffffffffu, valid ? 1 : 0, ra) != 0;
+          const bool vb = __shfl_sync(0xffffffffu, valid ? 1 : 0, rb) != 0;
+          const uint32_t th = tO + ((uint32_t)(16 * hf) << 16);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t o[32];
+            RA_TMEM_LD256X8(th + 64 * c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+              const int col = 64 * c + 8 * g + 2 * (lane & 3);
+              if (va)
+                *reinterpret_cast<float2*>(obase + ra * rstride + col) = make_float2(
+                    __uint_as_float(o[4 * g]) * ia, __uint_as_float(o[4 * g + 1]) * ia);
+              if (vb)
+                *reinterpret_cast<float2*>(obase + rb * rstride + col) = make_float2(
+                    __uint_as_float(o[4 * g + 2]) * ib, __uint_as_float(o[4 * g + 3]) * ib);
+            }
+          }
+        }
+      } else if (!first) {
         const float inv_l = valid ? p.out_scale / l : 0.f;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
           uint32_t o[32];
           RA_TMEM_LD32(tO + c, o);
           tmem_wait_ld();
-          if (p.step) {
-            // ring step: the running output stays fp32
-            if (valid) {
-              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow_off + c);
+          uint32_t pk[16];
 #pragma unroll
-              for (int j = 0; j < 8; ++j)
-                dst[j] = make_float4(
-                    __uint_as_float(o[4 * j]) * inv_l, __uint_as_float(o[4 * j + 1]) * inv_l,
-                    __uint_as_float(o[4 * j + 2]) * inv_l, __uint_as_float(o[4 * j + 3]) * inv_l);
-            }
-          } else {
-            uint32_t pk[16];
+          for (int j = 0; j < 16; ++j)
+            pk[j] = pack_x2<F::kF8 ? kFmtBF16 : kFmt>(__uint_as_float(o[2 * j]) * inv_l,
+                                                     __uint_as_float(o[2 * j + 1]) * inv_l);
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + orow_off + c);
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              pk[j] = pack_x2<F::kF8 ? kFmtBF16 : kFmt>(__uint_as_float(o[2 * j]) * inv_l,
-                                                       __uint_as_float(o[2 * j + 1]) * inv_l);
-            if (valid) {
-              uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + orow_off + c);
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-            }
+            for (int j = 0; j < 4; ++j)
+              dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
           }
         }
       } else if (p.step && !p.accumulate && valid) {

@@ -11,26 +11,30 @@
 // wrong in an implementation).  Two kernels, so every gradient element has
 // one writer and no atomics are needed:
 //
-//  bwd_dq_kernel (query-outer, the forward's ring walk over 64-key tiles):
-//   per kv tile S = Q K^T and dP = dO V^T into tensor memory, the gradient
-//   warps form dS = P (dP - D) and store it as 16-bit to shared memory, then
-//   dQ += dS K.  It also writes D per query row for the second kernel.
-//   warps 0-3 / 4-7  gradient warps of query tile 0 / 1 (one TMEM lane each)
-//   warp  8          TMA producer: Q, dO per item; (K, V) pairs into a ring
-//   warps 9, 11      MMA issuers, one per query tile
-//   warp  10         schedule builder (the ring walk with 64-key tiles)
-//   TMEM: S_0 | S_1 | dP_0 | dP_1 | dQ_0 | dQ_1 (64, 64, 64, 64, D, D).
+//  bwd_dq_kernel (query-outer, the forward's ring walk over 128-key tiles,
+//   one 128-row query tile per item): per kv tile S = Q K^T and dP = dO V^T
+//   into tensor memory; the gradient warps read both, form dS = P (dP - D)
+//   and write it as 16-bit over the dP columns they have read; then
+//   dQ += dS K takes dS from tensor memory.  dP alternates between two
+//   buffers, so S and dP of the next kv tile are computed while the
+//   gradient warps work on this one.  It also writes D per query row for
+//   the second kernel.
+//   warps 0-7   gradient warps: warp w owns query rows 32 (w % 4) .. + 31
+//               (its TMEM lane quadrant) and keys 64 (w / 4) .. + 63
+//   warp  8     TMA producer: Q, dO per item; (K, V) pairs into a ring
+//   warp  9     MMA issuer;  warp 10 schedule builder;  warp 11 idle
+//   TMEM: S 128 | dP_A 128 | dP_B 128 | dQ D.
 //
 //  bwd_dkdv_kernel (key/value-outer): a CTA owns 128 keys of one (sequence,
 //   key/value head), one TMEM lane each, and walks the 64-row query tiles
-//   of every query head of its group that see them:
-//   S^T = K Q^T and dP^T = V dO^T into tensor memory, the gradient warps form
-//   P^T and dS^T = P^T (dP^T - D) into shared memory, then dV += P^T dO and
-//   dK += dS^T Q.
-//   warps 0-3 / 4-7  gradient warps for query columns 0-31 / 32-63
+//   of every query head of its group that see them, 128 queries a step:
+//   S^T = K Q^T and dP^T = V dO^T into tensor memory, the gradient warps
+//   write P^T and dS^T = P^T (dP^T - D) as 16-bit over the columns they have
+//   read, then dV += P^T dO and dK += dS^T Q take them from tensor memory.
+//   warps 0-3 / 4-7  gradient warps for query columns 0-63 / 64-127
 //   warp  8          TMA producer (and the per-tile lse / D vectors)
 //   warp  9          MMA issuer;  warp 10 schedule builder;  warp 11 idle
-//   TMEM: S^T 64 | dP^T 64 | dV D | dK D.
+//   TMEM: S^T 128 | dP^T 128 | dV D | dK D.
 // Every wait is bounded like the forward's: an expired wait latches
 // ST_TIMEOUT, the CTA drains what it issued and frees its tensor memory.
 #include <cuda.h>
@@ -46,12 +50,11 @@
 namespace ra {
 namespace tcb {
 
-constexpr int BM = 128;   // query rows per tile
-constexpr int QT = 2;     // query tiles per CTA
-constexpr int BN = 64;    // keys per kv tile
+constexpr int BM = 128;   // query rows per item (one TMEM lane each)
+constexpr int BN = 128;   // keys per kv tile
 constexpr int kThreads = 384;
-constexpr int kProducer = 8, kMma0 = 9, kBuilder = 10, kMma1 = 11;
-constexpr int kConsumers = 11;  // producer, 2 issuers, 8 gradient warps
+constexpr int kProducer = 8, kMma = 9, kBuilder = 10;  // warp 11 idle
+constexpr int kConsumers = 10;  // producer, issuer, 8 gradient warps
 constexpr int kStages = 2;      // (K, V) pairs in the ring
 constexpr int kRegsGrad = 184, kRegsControl = 136;  // 256*184 + 128*136 = 384*168
 constexpr uint32_t kTmemCols = 512;
@@ -59,33 +62,28 @@ constexpr uint32_t kTmemCols = 512;
 template <int D>
 struct Cfg {
   static constexpr int kPanels = D / 64;
-  static constexpr int kQPanel = BM * 128;
-  static constexpr int kQTile = kPanels * kQPanel;
-  static constexpr int kKPanel = BN * 128;
-  static constexpr int kKTile = kPanels * kKPanel;
-  static constexpr int kDSBytes = BM * BN * 2;  // one 128-byte panel of 64 keys
+  static constexpr int kPanel = 128 * 128;          // 128 rows x 128 B
+  static constexpr int kTile = kPanels * kPanel;    // a Q, dO, K or V tile
   static constexpr int kQOff = 0;
-  static constexpr int kDOOff = kQOff + QT * kQTile;
-  static constexpr int kKVOff = kDOOff + QT * kQTile;  // slot s: K at +0, V at +kKTile
-  static constexpr int kDSOff = kKVOff + kStages * 2 * kKTile;
-  static constexpr int kListOff = kDSOff + QT * kDSBytes;
+  static constexpr int kDOOff = kTile;
+  static constexpr int kKVOff = 2 * kTile;          // slot s: K at +0, V at +kTile
+  static constexpr int kListOff = kKVOff + kStages * 2 * kTile;
   static constexpr int kCtrlOff = kListOff + kListBufs * kListChunk * 4;
   static constexpr int kSmemBytes = kCtrlOff + 512 + 1024;
-  static constexpr uint32_t kColS = 0;      // S_i at i * 64
-  static constexpr uint32_t kColDP = 128;   // dP_i at 128 + i * 64
-  static constexpr uint32_t kColDQ = 256;   // dQ_i at 256 + i * D
+  static constexpr uint32_t kColS = 0;      // S
+  static constexpr uint32_t kColDP = 128;   // dP buffer b at 128 + 128 b (dS over it)
+  static constexpr uint32_t kColDQ = 384;   // dQ
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(kColDQ + QT * D <= kTmemCols, "tensor memory budget");
+  static_assert(kColDQ + D <= kTmemCols, "tensor memory budget");
 };
 
 struct Ctrl {
   uint64_t q_full, q_free;
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[QT], s_free[QT];
-  uint64_t ds_full[QT], ds_done[QT];
-  uint64_t dq_full[QT], dq_free[QT];
+  uint64_t s_full, s_free, ds_full;
+  uint64_t dq_full, dq_free;
   uint64_t list_full[kListBufs], list_empty[kListBufs];
-  uint64_t drain[QT];
+  uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -171,37 +169,38 @@ __device__ __forceinline__ void tile_mask(uint32_t mw[2], const FwdParams& p, in
   }
 }
 
-// D x 64 keys for one query tile: S_i = Q_i K^T (A 128-row panels, B 64-row
-// panels, both K-major, 128-byte swizzle).
+// S = A B^T for the query tile: A (128 query rows) and B (128 key rows),
+// both K-major in 128-byte-swizzled panels kPanel apart; M = N = 128,
+// K = D in steps of 16 (start address field + panel * kPanel / 16 +
+// 2 * (kk % 4)).
 template <int D>
-__device__ __forceinline__ void issue_qk64(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+__device__ __forceinline__ void issue_rows(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                            uint32_t idesc) {
   using C = Cfg<D>;
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint64_t ao = (uint64_t)((kk >> 2) * (C::kQPanel >> 4) + (kk & 3) * 2);
-    const uint64_t bo = (uint64_t)((kk >> 2) * (C::kKPanel >> 4) + (kk & 3) * 2);
-    umma_ss(d_tmem, adesc + ao, bdesc + bo, idesc, kk > 0 ? 1u : 0u);
+    const uint64_t off = (uint64_t)((kk >> 2) * (C::kPanel >> 4) + (kk & 3) * 2);
+    umma_ss(d_tmem, adesc + off, bdesc + off, idesc, kk > 0 ? 1u : 0u);
   }
 }
 
-// dQ_i (+)= dS_i K: A = dS (128 x 64, K-major, one panel), B = K tile
-// MN-major (N = D in 64-element panels kKPanel apart; 8-key groups 1024 B
-// apart).  Step kk covers 16 keys.
-__device__ __forceinline__ void issue_dsk(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                          uint32_t idesc, bool accumulate) {
+// dQ (+)= dS K: A = dS in tensor memory, 16-bit pairs (keys 0-63 in columns
+// [a, a + 32), keys 64-127 in [a + 64, a + 96)), B = the K tile MN-major
+// (N = D in panels kPanel apart; 8-key groups 1024 bytes apart).  Step kk
+// covers 16 keys.
+__device__ __forceinline__ void issue_dq(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                         uint32_t idesc, bool accumulate) {
 #pragma unroll
   for (int kk = 0; kk < BN / 16; ++kk)
-    umma_ss(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 128), idesc,
-            (accumulate || kk > 0) ? 1u : 0u);
+    umma_ts(d_tmem, a_tmem + (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8),
+            bdesc + (uint64_t)(kk * 128), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 template <int D, int kFmt>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_kernel(const Params bp, const __grid_constant__ Maps maps, int n_items,
-                     int claim_limit) {
+                  int claim_limit) {
   using C = Cfg<D>;
-  constexpr int kRows = BM * QT;
   const FwdParams& p = bp.f;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -214,20 +213,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&ctrl->q_full, 1);
-    mbar_init(&ctrl->q_free, 2);
+    mbar_init(&ctrl->q_free, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&ctrl->kv_full[s], 1);
-      mbar_init(&ctrl->kv_empty[s], 2);
+      mbar_init(&ctrl->kv_empty[s], 1);
     }
-    for (int i = 0; i < QT; ++i) {
-      mbar_init(&ctrl->s_full[i], 1);
-      mbar_init(&ctrl->s_free[i], BM);
-      mbar_init(&ctrl->ds_full[i], BM);
-      mbar_init(&ctrl->ds_done[i], 1);
-      mbar_init(&ctrl->dq_full[i], 1);
-      mbar_init(&ctrl->dq_free[i], BM);
-      mbar_init(&ctrl->drain[i], 1);
-    }
+    mbar_init(&ctrl->s_full, 1);
+    mbar_init(&ctrl->s_free, 256);
+    mbar_init(&ctrl->ds_full, 256);
+    mbar_init(&ctrl->dq_full, 1);
+    mbar_init(&ctrl->dq_free, 256);
+    mbar_init(&ctrl->drain, 1);
     for (int b = 0; b < kListBufs; ++b) {
       mbar_init(&ctrl->list_full[b], 1);
       mbar_init(&ctrl->list_empty[b], kConsumers);
@@ -235,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ctrl->abort = 0;
     mbar_fence_init();
   }
-  if (warp == kMma0) {
+  if (warp == kMma) {
     tmem_alloc(&ctrl->tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -279,17 +275,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) ok = put(kAllDone) && flush();
           break;
         }
-        const SeqWork it = find_work_item(p, kRows, item);
+        const SeqWork it = find_work_item(p, BM, item);
         if (!it.live) continue;
         if (lane == 0) {
-          const int q0 = it.qr * kRows;
-          const int qm = min(q0 + BM, it.L), q1 = min(q0 + kRows, it.L);
+          const int q0 = it.qr * BM, q1 = min(q0 + BM, it.L);
           const RingGeom g = make_geom(it.L, p.n_ring, p.layout, p.causal, p.passes);
           ok = put_item(wr, item, it);
+          // one query range: the walk's second sub-range is empty
           TileWalk walk;
-          walk.init(g, q0, qm, q1, BN);
+          walk.init(g, q0, q1, q1, BN);
           int kt, c0, c1;
-          while (ok && walk.next(&kt, &c0, &c1)) ok = put((kt << 4) | (c1 << 2) | c0);
+          while (ok && walk.next(&kt, &c0, &c1)) ok = put((kt << 4) | c0);
           if (ok) ok = put(kItemEnd);
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -316,12 +312,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (n >= kStages &&
             !mbar_wait(&ctrl->kv_empty[slot], ((n / kStages) - 1) & 1, abort_flag))
           return false;
-        uint8_t* dst = smem + C::kKVOff + slot * 2 * C::kKTile;
-        mbar_arrive_expect_tx(&ctrl->kv_full[slot], 2 * C::kKTile);
+        uint8_t* dst = smem + C::kKVOff + slot * 2 * C::kTile;
+        mbar_arrive_expect_tx(&ctrl->kv_full[slot], 2 * C::kTile);
         for (int pn = 0; pn < C::kPanels; ++pn) {
-          tma_load_3d(dst + pn * C::kKPanel, &maps.k, &ctrl->kv_full[slot], pn * 64, hk, row);
-          tma_load_3d(dst + C::kKTile + pn * C::kKPanel, &maps.v, &ctrl->kv_full[slot],
-                      pn * 64, hk, row);
+          tma_load_3d(dst + pn * C::kPanel, &maps.k, &ctrl->kv_full[slot], pn * 64, hk, row);
+          tma_load_3d(dst + C::kTile + pn * C::kPanel, &maps.v, &ctrl->kv_full[slot], pn * 64,
+                      hk, row);
         }
         ++n;
         return true;
@@ -338,18 +334,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int hk = it.h / p.kv_group;
           int e = -1;
           if (ok) ok = rd.next(&e, abort_flag);
+          // the item's first (K, V) enters the ring before Q and dO wait for
+          // the previous item's last S and dP MMAs (q_free)
           if (ok && e >= 0) ok = load_kv(hk, it.base + entry_tile(e) * BN);
           if (ok && k > 0) ok = mbar_wait(&ctrl->q_free, (k - 1) & 1, abort_flag);
           if (ok) {
-            const int q0 = it.qr * kRows;
-            mbar_arrive_expect_tx(&ctrl->q_full, 2 * QT * C::kQTile);
-            for (int i = 0; i < QT; ++i)
-              for (int pn = 0; pn < C::kPanels; ++pn) {
-                tma_load_3d(smem + C::kQOff + i * C::kQTile + pn * C::kQPanel, &maps.q,
-                            &ctrl->q_full, pn * 64, it.h, it.base + q0 + i * BM);
-                tma_load_3d(smem + C::kDOOff + i * C::kQTile + pn * C::kQPanel, &maps.dout,
-                            &ctrl->q_full, pn * 64, it.h, it.base + q0 + i * BM);
-              }
+            const int q_row = it.base + it.qr * BM;
+            mbar_arrive_expect_tx(&ctrl->q_full, 2 * C::kTile);
+            for (int pn = 0; pn < C::kPanels; ++pn) {
+              tma_load_3d(smem + C::kQOff + pn * C::kPanel, &maps.q, &ctrl->q_full, pn * 64,
+                          it.h, q_row);
+              tma_load_3d(smem + C::kDOOff + pn * C::kPanel, &maps.dout, &ctrl->q_full, pn * 64,
+                          it.h, q_row);
+            }
             ++nq;
           }
           while (ok && e >= 0) {
@@ -368,27 +365,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (nq > 0) mbar_wait(&ctrl->q_full, (nq - 1) & 1, nullptr);
       }
       __syncwarp();
-    } else {
-      // ---------------------------------------------------------- MMA issuers
-      // Issuer i, per kv tile t: S_i(t+1), dP_i(t+1) once the gradient warps
-      // have read S_i(t), dP_i(t) (s_free); then dQ_i += dS_i(t) K(t) once
-      // dS_i(t) is in shared memory (ds_full).  The slot of tile t is released
-      // by one commit of each issuer after its dQ MMA.
-      const int i = warp == kMma1 ? 1 : 0;
+    } else if (warp == kMma) {
+      // ---------------------------------------------------------- MMA issuer
+      // Per kv tile t: S(t+1) and dP(t+1) as soon as the gradient warps have
+      // read S(t) and dP(t) (s_free), dP into the buffer dP(t) does not use;
+      // then dQ += dS(t) K(t) once dS(t) is in tensor memory (ds_full).  One
+      // thread issues everything, so dP(t+2) overwrites dS(t) only after the
+      // dQ MMA of tile t has read it.  The slot of tile t is released after
+      // that MMA.  S/dP number n and dQ number n share buffer n % 2.
       const uint32_t idesc_s = idesc_f16kind_f32(BM, BN, 0, kFmt);
       constexpr uint32_t idesc_q = idesc_f16kind_f32(BM, D, 1, kFmt);
-      const uint64_t qdesc = smem_desc_sw128(smem_u32(smem + C::kQOff + i * C::kQTile), 16, 1024);
-      const uint64_t dodesc =
-          smem_desc_sw128(smem_u32(smem + C::kDOOff + i * C::kQTile), 16, 1024);
-      const uint64_t dsdesc =
-          smem_desc_sw128(smem_u32(smem + C::kDSOff + i * C::kDSBytes), 16, 1024);
+      const uint64_t qdesc = smem_desc_sw128(smem_u32(smem + C::kQOff), 16, 1024);
+      const uint64_t dodesc = smem_desc_sw128(smem_u32(smem + C::kDOOff), 16, 1024);
       const uint64_t kdesc0 = smem_desc_sw128(smem_u32(smem + C::kKVOff), 16, 1024);
-      const uint64_t vdesc0 = smem_desc_sw128(smem_u32(smem + C::kKVOff + C::kKTile), 16, 1024);
-      const uint64_t kmn0 = smem_desc_sw128(smem_u32(smem + C::kKVOff), C::kKPanel, 1024);
-      constexpr uint64_t kSlotStep = (uint64_t)((2 * C::kKTile) >> 4);
-      const uint32_t tS = tmem + C::kColS + i * BN;
-      const uint32_t tDP = tmem + C::kColDP + i * BN;
-      const uint32_t tDQ = tmem + C::kColDQ + i * D;
+      const uint64_t vdesc0 = smem_desc_sw128(smem_u32(smem + C::kKVOff + C::kTile), 16, 1024);
+      const uint64_t kmn0 = smem_desc_sw128(smem_u32(smem + C::kKVOff), C::kPanel, 1024);
+      constexpr uint64_t kSlotStep = (uint64_t)((2 * C::kTile) >> 4);
+      const uint32_t tS = tmem + C::kColS;
+      const uint32_t tDQ = tmem + C::kColDQ;
       uint32_t ns = 0, nd = 0;
       int n = 0, k = 0;
       bool ok = true, issued_any = false;
@@ -398,6 +392,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++n;
         if (ok) tc_fence_after();
         return slot;
+      };
+      // S and dP of the tile in `slot`; S(n) overwrites S(n-1), which the
+      // gradient warps must have read
+      auto issue_sdp = [&](int slot) {
+        if (ns > 0) {
+          ok = mbar_wait(&ctrl->s_free, (ns - 1) & 1, abort_flag);
+          if (!ok) return;
+          tc_fence_after();
+        }
+        issue_rows<D>(tS, qdesc, kdesc0 + slot * kSlotStep, idesc_s);
+        issue_rows<D>(tmem + C::kColDP + 128u * (ns & 1), dodesc, vdesc0 + slot * kSlotStep,
+                      idesc_s);
+        umma_commit(&ctrl->s_full);
+        ++ns;
+        issued_any = true;
       };
       while (ok) {
         int h = 0;
@@ -411,25 +420,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok) ok = mbar_wait(&ctrl->q_full, k & 1, abort_flag);
           tc_fence_after();
           bool started = false;
-          // S_i, dP_i of the tile in `slot` if this issuer's query tile sees it
-          auto issue_sdp = [&](int e, int slot) {
-            if (entry_cls(e, i) == CLS_EMPTY) return;
-            if (ns > 0) {
-              ok = mbar_wait(&ctrl->s_free[i], (ns - 1) & 1, abort_flag);
-              if (!ok) return;
-              tc_fence_after();
-            }
-            issue_qk64<D>(tS, qdesc, kdesc0 + slot * kSlotStep, idesc_s);
-            issue_qk64<D>(tDP, dodesc, vdesc0 + slot * kSlotStep, idesc_s);
-            umma_commit(&ctrl->s_full[i]);
-            ++ns;
-            issued_any = true;
-          };
           int e = -1;
           if (ok) ok = rd.next(&e, abort_flag);
           if (ok && e >= 0) {
             int slot = take();
-            if (ok) issue_sdp(e, slot);
+            if (ok) issue_sdp(slot);
             while (ok) {
               int en = -1;
               ok = rd.next(&en, abort_flag);
@@ -438,28 +433,26 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (en >= 0) {
                 slot_n = take();
                 if (!ok) break;
-                issue_sdp(en, slot_n);
+                issue_sdp(slot_n);
                 if (!ok) break;
               } else {
                 umma_commit(&ctrl->q_free);  // every S/dP of this item issued
               }
-              if (entry_cls(e, i) != CLS_EMPTY) {
-                ok = mbar_wait(&ctrl->ds_full[i], nd & 1, abort_flag);
+              ok = mbar_wait(&ctrl->ds_full, nd & 1, abort_flag);
+              if (!ok) break;
+              tc_fence_after();
+              if (!started && k > 0) {
+                // the previous item's dQ has been read out
+                ok = mbar_wait(&ctrl->dq_free, (k - 1) & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                if (!started && k > 0) {
-                  ok = mbar_wait(&ctrl->dq_free[i], (k - 1) & 1, abort_flag);
-                  if (!ok) break;
-                  tc_fence_after();
-                }
-                issue_dsk(tDQ, dsdesc, kmn0 + slot * kSlotStep, idesc_q, started);
-                umma_commit(&ctrl->ds_done[i]);
-                ++nd;
-                started = true;
               }
+              issue_dq(tDQ, tmem + C::kColDP + 128u * (nd & 1), kmn0 + slot * kSlotStep,
+                       idesc_q, started);
               umma_commit(&ctrl->kv_empty[slot]);
+              ++nd;
+              started = true;
               if (en < 0) break;
-              e = en;
               slot = slot_n;
             }
           } else if (ok) {
@@ -469,10 +462,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!started && k > 0) {
               // no dQ MMA this item: the read-out of the previous one must
               // still finish before dq_full is signalled again
-              ok = mbar_wait(&ctrl->dq_free[i], (k - 1) & 1, abort_flag);
+              ok = mbar_wait(&ctrl->dq_free, (k - 1) & 1, abort_flag);
               tc_fence_after();
             }
-            if (ok) umma_commit(&ctrl->dq_full[i]);
+            if (ok) umma_commit(&ctrl->dq_full);
           }
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -482,8 +475,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 1;
         latch_status(p.status, ST_TIMEOUT);
         if (issued_any) {
-          umma_commit(&ctrl->drain[i]);
-          mbar_wait(&ctrl->drain[i], 0, nullptr);
+          umma_commit(&ctrl->drain);
+          mbar_wait(&ctrl->drain, 0, nullptr);
         }
       }
       __syncwarp();
@@ -491,16 +484,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     regs_inc<kRegsGrad>();
     // ---------------------------------------------------------- gradient warps
-    const int tile = warp >> 2;
+    const int half = warp >> 2;   // keys [64 half, 64 half + 64) of each kv tile
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::kColS + tile * BN;
-    const uint32_t tDP = tmem + lane_off + C::kColDP + tile * BN;
-    const uint32_t tDQ = tmem + lane_off + C::kColDQ + tile * D;
-    const uint32_t dsrow = smem_u32(smem + C::kDSOff + tile * C::kDSBytes) + (uint32_t)r * 128u;
-    const uint32_t swz = (uint32_t)(r & 7);
-    uint32_t sphase = 0, nd = 0;
+    const uint32_t tS = tmem + lane_off + C::kColS + 64 * half;
+    constexpr int kOutCols = D / 2;  // dQ columns this warp writes out
+    const uint32_t tDQ = tmem + lane_off + C::kColDQ + kOutCols * half;
+    uint32_t sphase = 0, nstep = 0;
     int k = 0;
     bool ok = true;
     while (true) {
@@ -511,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = read_item<true>(rd, &it, abort_flag);
       if (!ok) break;
       const int L = it.L;
-      const int sq = it.qr * kRows + tile * BM + r;
+      const int sq = it.qr * BM + r;
       const bool valid = sq < L;
       int rq = 0, tq = 0;
       if (valid) {
@@ -522,7 +513,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t li = (int64_t)it.b * p.lse_seq_stride + (int64_t)it.h * p.lse_head_stride +
                          (p.cu_seqlens ? it.base : 0) + sq;
       const int64_t roff = ((int64_t)(it.base + sq) * bp.heads_q + it.h) * D;
-      // D = <dO, O> for this row, fp32 over the 16-bit inputs
+      // D = <dO, O> for this row, fp32 over the 16-bit inputs (both warps of
+      // the row form it; the first writes it for the dK/dV kernel)
       float dsum = 0.f, lse2 = 0.f;
       if (valid) {
         const uint4* dorow = reinterpret_cast<const uint4*>(
@@ -551,20 +543,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         lse2 = p.lse[li] * 1.4426950408889634f;
-        if (bp.dsum) bp.dsum[li] = dsum;
+        if (bp.dsum && half == 0) bp.dsum[li] = dsum;
       }
       bool any = false;
       while (true) {
         int e;
         ok = rd.next_warp(&e, abort_flag);
         if (!ok || e < 0) break;
-        const int cls = entry_cls(e, tile);
-        if (cls == CLS_EMPTY) continue;
-        ok = warp_wait(&ctrl->s_full[tile], sphase, abort_flag);
+        const int cls = entry_cls(e, 0);
+        ok = warp_wait(&ctrl->s_full, sphase, abort_flag);
         sphase ^= 1;
         if (!ok) break;
         tc_fence_after();
-        float s[BN], dp[BN];
+        // this warp's 64 keys of S and of dP (buffer nstep % 2)
+        const uint32_t tDP = tmem + lane_off + C::kColDP + 128u * (nstep & 1) + 64 * half;
+        float s[64], dp[64];
         {
           uint32_t* sr = reinterpret_cast<uint32_t*>(s);
           uint32_t* dr = reinterpret_cast<uint32_t*>(dp);
@@ -575,14 +568,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
         }
         tc_fence_before();
-        mbar_arrive(&ctrl->s_free[tile]);
-        const int k0 = entry_tile(e) * BN;
-        const int nk = min(BN, L - k0);
+        mbar_arrive(&ctrl->s_free);
+        const int k0 = entry_tile(e) * BN + 64 * half;
+        const int nk = min(64, L - k0);
         uint32_t mw[2];
         tile_mask(mw, p, L, valid, cls, rq, tq, k0, nk);
-        uint32_t pk[BN / 2];
+        uint32_t pk[32];
 #pragma unroll
-        for (int j = 0; j < BN / 2; ++j) {
+        for (int j = 0; j < 32; ++j) {
           const int c0 = 2 * j, c1 = 2 * j + 1;
           const bool a0 = (mw[c0 >> 5] >> (c0 & 31)) & 1u;
           const bool a1 = (mw[c1 >> 5] >> (c1 & 31)) & 1u;
@@ -590,29 +583,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float p1 = a1 ? ex2_approx(fmaf(s[c1], p.scale_log2, -lse2)) : 0.f;
           pk[j] = pack_x2<kFmt>(p0 * (dp[c0] - dsum), p1 * (dp[c1] - dsum));
         }
-        // the previous dQ MMA of this tile has read dS
-        if (nd > 0) {
-          ok = warp_wait(&ctrl->ds_done[tile], (nd - 1) & 1, abort_flag);
-          if (!ok) break;
-        }
-#pragma unroll
-        for (int g8 = 0; g8 < BN / 8; ++g8) {
-          const uint32_t addr = dsrow + ((((uint32_t)g8) ^ swz) << 4);
-          st_shared_v4(addr, pk[4 * g8], pk[4 * g8 + 1], pk[4 * g8 + 2], pk[4 * g8 + 3]);
-        }
-        fence_proxy_async_smem();
+        // dS over the first 32 of this warp's dP columns (already read)
+        RA_TMEM_ST32(tDP, pk);
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&ctrl->ds_full[tile]);
-        ++nd;
+        mbar_arrive(&ctrl->ds_full);
+        ++nstep;
         any = true;
       }
       if (!ok) break;
-      // epilogue: dQ out of tensor memory, scaled, in the input format
-      ok = warp_wait(&ctrl->dq_full[tile], k & 1, abort_flag);
+      // epilogue: this warp's half of the row's dQ, scaled, in the input format
+      ok = warp_wait(&ctrl->dq_full, k & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < D; c += 32) {
+      for (int c = 0; c < kOutCols; c += 32) {
         uint32_t o[32];
         if (any) {
           RA_TMEM_LD32(tDQ + c, o);
@@ -627,14 +612,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[j] = pack_x2<kFmt>(__uint_as_float(o[2 * j]) * p.scale,
                                 __uint_as_float(o[2 * j + 1]) * p.scale);
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(bp.dq) + roff + c);
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(bp.dq) + roff +
+                                                kOutCols * half + c);
 #pragma unroll
           for (int j = 0; j < 4; ++j)
             dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
         }
       }
       tc_fence_before();
-      mbar_arrive(&ctrl->dq_free[tile]);
+      mbar_arrive(&ctrl->dq_free);
       ++k;
     }
     if (!ok) {
@@ -645,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kMma0) {
+  if (warp == kMma) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -694,9 +680,8 @@ static cudaError_t launch_t(const Params& bp_in, cudaStream_t stream, int num_sm
   using C = Cfg<D>;
   Params bp = bp_in;
   FwdParams& p = bp.f;
-  p.n_qranges = (p.seqlen + BM * QT - 1) / (BM * QT);
-  if (!p.cu_seqlens) p.n_qranges = (p.seqlen + BM * QT - 1) / (BM * QT);
-  const int64_t items = work_grid(p, BM * QT);
+  p.n_qranges = (p.seqlen + BM - 1) / BM;
+  const int64_t items = work_grid(p, BM);
   if (items == 0) return cudaSuccess;
   if (items > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const bool per_item = p.causal && !p.cu_seqlens;

@@ -55,7 +55,9 @@ constexpr int BN = 128;   // keys per kv tile
 constexpr int kThreads = 384;
 constexpr int kProducer = 8, kMma = 9, kBuilder = 10;  // warp 11 idle
 constexpr int kConsumers = 10;  // producer, issuer, 8 gradient warps
-constexpr int kStages = 2;      // (K, V) pairs in the ring
+// K and V tiles in two rings: V(t) is free once dP(t) has run, K(t) only
+// after dQ(t), so K gets one slot more and both are loaded a step ahead.
+constexpr int kKSlots = 3, kVSlots = 2;
 constexpr int kRegsGrad = 184, kRegsControl = 136;  // 256*184 + 128*136 = 384*168
 constexpr uint32_t kTmemCols = 512;
 
@@ -66,8 +68,9 @@ struct Cfg {
   static constexpr int kTile = kPanels * kPanel;    // a Q, dO, K or V tile
   static constexpr int kQOff = 0;
   static constexpr int kDOOff = kTile;
-  static constexpr int kKVOff = 2 * kTile;          // slot s: K at +0, V at +kTile
-  static constexpr int kListOff = kKVOff + kStages * 2 * kTile;
+  static constexpr int kKOff = 2 * kTile;           // K ring
+  static constexpr int kVOff = kKOff + kKSlots * kTile;  // V ring
+  static constexpr int kListOff = kVOff + kVSlots * kTile;
   static constexpr int kCtrlOff = kListOff + kListBufs * kListChunk * 4;
   static constexpr int kSmemBytes = kCtrlOff + 512 + 1024;
   static constexpr uint32_t kColS = 0;      // S
@@ -79,7 +82,8 @@ struct Cfg {
 
 struct Ctrl {
   uint64_t q_full, q_free;
-  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t k_full[kKSlots], k_empty[kKSlots];
+  uint64_t v_full[kVSlots], v_empty[kVSlots];
   uint64_t s_full, s_free, ds_full;
   uint64_t dq_full, dq_free;
   uint64_t list_full[kListBufs], list_empty[kListBufs];
@@ -214,9 +218,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(&ctrl->q_full, 1);
     mbar_init(&ctrl->q_free, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&ctrl->kv_full[s], 1);
-      mbar_init(&ctrl->kv_empty[s], 1);
+    for (int s = 0; s < kKSlots; ++s) {
+      mbar_init(&ctrl->k_full[s], 1);
+      mbar_init(&ctrl->k_empty[s], 1);
+    }
+    for (int s = 0; s < kVSlots; ++s) {
+      mbar_init(&ctrl->v_full[s], 1);
+      mbar_init(&ctrl->v_empty[s], 1);
     }
     mbar_init(&ctrl->s_full, 1);
     mbar_init(&ctrl->s_free, 256);
@@ -306,20 +314,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int n = 0, k = 0, nq = 0;
       bool ok = true;
-      // one (K, V) pair of kv tile `row` into the next ring slot
+      int nv = 0;  // V tiles issued (n counts K tiles)
+      // K and V of kv tile `row`, each into the next slot of its ring
       auto load_kv = [&](int hk, int row) -> bool {
-        const int slot = n % kStages;
-        if (n >= kStages &&
-            !mbar_wait(&ctrl->kv_empty[slot], ((n / kStages) - 1) & 1, abort_flag))
+        const int ks = n % kKSlots, vs = nv % kVSlots;
+        if (n >= kKSlots &&
+            !mbar_wait(&ctrl->k_empty[ks], ((n / kKSlots) - 1) & 1, abort_flag))
           return false;
-        uint8_t* dst = smem + C::kKVOff + slot * 2 * C::kTile;
-        mbar_arrive_expect_tx(&ctrl->kv_full[slot], 2 * C::kTile);
-        for (int pn = 0; pn < C::kPanels; ++pn) {
-          tma_load_3d(dst + pn * C::kPanel, &maps.k, &ctrl->kv_full[slot], pn * 64, hk, row);
-          tma_load_3d(dst + C::kTile + pn * C::kPanel, &maps.v, &ctrl->kv_full[slot], pn * 64,
-                      hk, row);
-        }
+        mbar_arrive_expect_tx(&ctrl->k_full[ks], C::kTile);
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_3d(smem + C::kKOff + ks * C::kTile + pn * C::kPanel, &maps.k,
+                      &ctrl->k_full[ks], pn * 64, hk, row);
         ++n;
+        if (nv >= kVSlots &&
+            !mbar_wait(&ctrl->v_empty[vs], ((nv / kVSlots) - 1) & 1, abort_flag))
+          return false;
+        mbar_arrive_expect_tx(&ctrl->v_full[vs], C::kTile);
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_3d(smem + C::kVOff + vs * C::kTile + pn * C::kPanel, &maps.v,
+                      &ctrl->v_full[vs], pn * 64, hk, row);
+        ++nv;
         return true;
       };
       while (ok) {
@@ -360,8 +374,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0 && !ok) {
         *abort_flag = 1;
         latch_status(p.status, ST_TIMEOUT);
-        for (int u = (n > kStages ? n - kStages : 0); u < n; ++u)
-          mbar_wait(&ctrl->kv_full[u % kStages], (u / kStages) & 1, nullptr);
+        // let the copies already issued land before the CTA can exit
+        for (int u = (n > kKSlots ? n - kKSlots : 0); u < n; ++u)
+          mbar_wait(&ctrl->k_full[u % kKSlots], (u / kKSlots) & 1, nullptr);
+        for (int u = (nv > kVSlots ? nv - kVSlots : 0); u < nv; ++u)
+          mbar_wait(&ctrl->v_full[u % kVSlots], (u / kVSlots) & 1, nullptr);
         if (nq > 0) mbar_wait(&ctrl->q_full, (nq - 1) & 1, nullptr);
       }
       __syncwarp();
@@ -371,39 +388,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       // read S(t) and dP(t) (s_free), dP into the buffer dP(t) does not use;
       // then dQ += dS(t) K(t) once dS(t) is in tensor memory (ds_full).  One
       // thread issues everything, so dP(t+2) overwrites dS(t) only after the
-      // dQ MMA of tile t has read it.  The slot of tile t is released after
-      // that MMA.  S/dP number n and dQ number n share buffer n % 2.
+      // dQ MMA of tile t has read it.  V(t)'s slot is released after dP(t),
+      // K(t)'s after dQ(t).  S/dP number n and dQ number n share buffer n % 2
+      // and are kv tile n of the rings.
       const uint32_t idesc_s = idesc_f16kind_f32(BM, BN, 0, kFmt);
       constexpr uint32_t idesc_q = idesc_f16kind_f32(BM, D, 1, kFmt);
       const uint64_t qdesc = smem_desc_sw128(smem_u32(smem + C::kQOff), 16, 1024);
       const uint64_t dodesc = smem_desc_sw128(smem_u32(smem + C::kDOOff), 16, 1024);
-      const uint64_t kdesc0 = smem_desc_sw128(smem_u32(smem + C::kKVOff), 16, 1024);
-      const uint64_t vdesc0 = smem_desc_sw128(smem_u32(smem + C::kKVOff + C::kTile), 16, 1024);
-      const uint64_t kmn0 = smem_desc_sw128(smem_u32(smem + C::kKVOff), C::kPanel, 1024);
-      constexpr uint64_t kSlotStep = (uint64_t)((2 * C::kTile) >> 4);
+      const uint64_t kdesc0 = smem_desc_sw128(smem_u32(smem + C::kKOff), 16, 1024);
+      const uint64_t vdesc0 = smem_desc_sw128(smem_u32(smem + C::kVOff), 16, 1024);
+      const uint64_t kmn0 = smem_desc_sw128(smem_u32(smem + C::kKOff), C::kPanel, 1024);
+      constexpr uint64_t kSlotStep = (uint64_t)(C::kTile >> 4);
       const uint32_t tS = tmem + C::kColS;
       const uint32_t tDQ = tmem + C::kColDQ;
       uint32_t ns = 0, nd = 0;
-      int n = 0, k = 0;
+      int k = 0;
       bool ok = true, issued_any = false;
-      auto take = [&]() -> int {
-        const int slot = n % kStages;
-        ok = mbar_wait(&ctrl->kv_full[slot], (n / kStages) & 1, abort_flag);
-        ++n;
-        if (ok) tc_fence_after();
-        return slot;
-      };
-      // S and dP of the tile in `slot`; S(n) overwrites S(n-1), which the
+      // S and dP of kv tile ns; S overwrites the previous tile's, which the
       // gradient warps must have read
-      auto issue_sdp = [&](int slot) {
+      auto issue_sdp = [&]() {
         if (ns > 0) {
           ok = mbar_wait(&ctrl->s_free, (ns - 1) & 1, abort_flag);
           if (!ok) return;
-          tc_fence_after();
         }
-        issue_rows<D>(tS, qdesc, kdesc0 + slot * kSlotStep, idesc_s);
-        issue_rows<D>(tmem + C::kColDP + 128u * (ns & 1), dodesc, vdesc0 + slot * kSlotStep,
+        const int ks = (int)(ns % kKSlots), vs = (int)(ns % kVSlots);
+        ok = mbar_wait(&ctrl->k_full[ks], (ns / kKSlots) & 1, abort_flag);
+        if (!ok) return;
+        tc_fence_after();
+        issue_rows<D>(tS, qdesc, kdesc0 + ks * kSlotStep, idesc_s);
+        ok = mbar_wait(&ctrl->v_full[vs], (ns / kVSlots) & 1, abort_flag);
+        if (!ok) return;
+        tc_fence_after();
+        issue_rows<D>(tmem + C::kColDP + 128u * (ns & 1), dodesc, vdesc0 + vs * kSlotStep,
                       idesc_s);
+        umma_commit(&ctrl->v_empty[vs]);
         umma_commit(&ctrl->s_full);
         ++ns;
         issued_any = true;
@@ -423,17 +441,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           int e = -1;
           if (ok) ok = rd.next(&e, abort_flag);
           if (ok && e >= 0) {
-            int slot = take();
-            if (ok) issue_sdp(slot);
+            issue_sdp();
             while (ok) {
               int en = -1;
               ok = rd.next(&en, abort_flag);
               if (!ok) break;
-              int slot_n = -1;
               if (en >= 0) {
-                slot_n = take();
-                if (!ok) break;
-                issue_sdp(slot_n);
+                issue_sdp();
                 if (!ok) break;
               } else {
                 umma_commit(&ctrl->q_free);  // every S/dP of this item issued
@@ -447,13 +461,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 tc_fence_after();
               }
-              issue_dq(tDQ, tmem + C::kColDP + 128u * (nd & 1), kmn0 + slot * kSlotStep,
-                       idesc_q, started);
-              umma_commit(&ctrl->kv_empty[slot]);
+              const int ks = (int)(nd % kKSlots);
+              issue_dq(tDQ, tmem + C::kColDP + 128u * (nd & 1), kmn0 + ks * kSlotStep, idesc_q,
+                       started);
+              umma_commit(&ctrl->k_empty[ks]);
               ++nd;
               started = true;
               if (en < 0) break;
-              slot = slot_n;
             }
           } else if (ok) {
             umma_commit(&ctrl->q_free);
@@ -708,19 +722,21 @@ namespace kv {
 // Key/value-outer kernel: one CTA per 128 keys of a (sequence, key/value
 // head), 128-query steps.  Per step t the tensor core computes
 //   S^T(t) = K Q(t)^T and dP^T(t) = V dO(t)^T     (M = 128 keys, N = 128)
-// into tensor memory; the gradient warps turn them into P^T and dS^T, which
-// they write as 16-bit over the scores they have read (two queries per
-// column); then
-//   dV += P^T(t) dO(t) and dK += dS^T(t) Q(t)     (A from tensor memory)
-// and S^T(t+1), dP^T(t+1) follow from the same issuing thread.  The tensor
-// core runs one thread's MMAs in issue order, so S^T(t+1) and dP^T(t+1)
-// overwrite the P^T(t), dS^T(t) columns only after dV and dK have read
-// them; the commit announcing S^T(t+1) also covers dV(t) and dK(t).
+// into tensor memory; the gradient warps read dP^T first (its columns are
+// then free: dp_free), then the scores chunk by chunk, and write P^T and
+// dS^T as 16-bit pairs over the score columns they have just read; then
+//   dV += P^T(t) dO(t) and dK += dS^T(t) Q(t)     (A from tensor memory).
+// dP^T(t+1) is issued as soon as dP^T(t) has been read, so it runs while
+// the gradient warps compute; S^T(t+1) follows dV(t) and dK(t) from the
+// same issuing thread (the tensor core runs one thread's MMAs in issue
+// order, so it overwrites P^T(t), dS^T(t) only after they have been read),
+// and the commit announcing step t+1 covers both of its products.
 // Gradient warp w works on key rows 32 (w % 4) .. + 31 (its TMEM lane
-// quadrant) and query columns 64 (w / 4) .. + 63; it writes P^T of its 64
-// queries into the first 32 columns of its own 64-column range, so the two
-// halves never overwrite scores the other has not read yet (each MMA step
-// takes its 16 queries' 8 columns from the half that holds them).
+// quadrant) and query columns 64 (w / 4) .. + 63, in two chunks of 32
+// queries: chunk c's P^T goes to the first 16 of the 32 score columns it
+// came from, its dS^T to the other 16, so no warp writes a column another
+// has not read yet (an MMA step takes its 16 queries' 8 columns from the
+// chunk that holds them).
 constexpr int BK = 128;  // keys per CTA
 constexpr int BQ = 128;  // query rows per step
 constexpr int kMma = 9;
@@ -749,7 +765,7 @@ struct Cfg {
 struct Ctrl {
   uint64_t kv_full, kv_free;
   uint64_t q_full[kQStages], q_empty[kQStages];
-  uint64_t s_full, pds_full;
+  uint64_t s_full, dp_free, pds_full;
   uint64_t acc_full, acc_free;
   uint64_t list_full[kListBufs], list_empty[kListBufs];
   uint64_t drain;
@@ -781,15 +797,15 @@ __device__ __forceinline__ void issue_kq(uint32_t d_tmem, uint64_t adesc, uint64
   }
 }
 
-// acc (+)= A B with A (128 keys x 128 queries, 16-bit) in tensor memory --
-// queries 0-63 in columns [a, a + 32), 64-127 in [a + 64, a + 96) -- and B a
-// 128-query tile MN-major (N = D in panels kQPanel apart).  Step kk covers
-// 16 queries.
+// acc (+)= A B with A (128 keys x 128 queries, 16-bit pairs) in tensor
+// memory -- queries 32 c .. 32 c + 31 in columns [a + 32 c, a + 32 c + 16)
+// -- and B a 128-query tile MN-major (N = D in panels kQPanel apart).  P^T
+// sits at a = the score columns, dS^T at a + 16.  Step kk covers 16 queries.
 __device__ __forceinline__ void issue_acc(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
                                           uint32_t idesc, bool accumulate) {
 #pragma unroll
   for (int kk = 0; kk < BQ / 16; ++kk)
-    umma_ts(d_tmem, a_tmem + (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8),
+    umma_ts(d_tmem, a_tmem + (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8),
             bdesc + (uint64_t)(kk * 128), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
@@ -817,6 +833,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ctrl->q_empty[s], 1);
     }
     mbar_init(&ctrl->s_full, 1);
+    mbar_init(&ctrl->dp_free, 256);
     mbar_init(&ctrl->pds_full, 256);
     mbar_init(&ctrl->acc_full, 1);
     mbar_init(&ctrl->acc_free, 256);
@@ -993,9 +1010,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) tc_fence_after();
         return slot;
       };
-      auto issue_sdp = [&](int slot) {
-        issue_kq<D>(tS, kdesc, qk0 + slot * kSlotStep, idesc_s);
+      // an item's first step: its dP^T once the previous step's has been
+      // read (its S^T follows that step's dV and dK in issue order)
+      auto issue_first = [&](int slot) {
+        if (npd > 0) {
+          ok = mbar_wait(&ctrl->dp_free, (npd - 1) & 1, abort_flag);
+          if (!ok) return;
+          tc_fence_after();
+        }
         issue_kq<D>(tDP, vdesc, dok0 + slot * kSlotStep, idesc_s);
+        issue_kq<D>(tS, kdesc, qk0 + slot * kSlotStep, idesc_s);
         umma_commit(&ctrl->s_full);
         issued_any = true;
       };
@@ -1015,14 +1039,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok) ok = rd.next(&e, abort_flag);
           if (ok && e >= 0) {
             int slot = take();
-            if (ok) issue_sdp(slot);
+            if (ok) issue_first(slot);
             while (ok) {
               int en = -1;
               ok = rd.next(&en, abort_flag);
               if (!ok) break;
               const int slot_n = en >= 0 ? take() : -1;
               if (!ok) break;
-              if (en < 0) umma_commit(&ctrl->kv_free);  // every use of K, V is issued
+              if (en >= 0) {
+                // dP^T(t+1) as soon as the gradient warps have read dP^T(t)
+                ok = mbar_wait(&ctrl->dp_free, npd & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                issue_kq<D>(tDP, vdesc, dok0 + slot_n * kSlotStep, idesc_s);
+              }
               ok = mbar_wait(&ctrl->pds_full, npd & 1, abort_flag);
               if (!ok) break;
               tc_fence_after();
@@ -1032,13 +1062,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
               }
               issue_acc(tDV, tS, domn0 + slot * kSlotStep, idesc_a, started);
-              issue_acc(tDK, tDP, qmn0 + slot * kSlotStep, idesc_a, started);
+              issue_acc(tDK, tS + 16, qmn0 + slot * kSlotStep, idesc_a, started);
               umma_commit(&ctrl->q_empty[slot]);
               ++npd;
               started = true;
-              if (en < 0) break;
+              if (en < 0) {
+                umma_commit(&ctrl->kv_free);  // every use of K, V is issued
+                break;
+              }
               // in issue order after dV and dK, which read P^T and dS^T
-              issue_sdp(slot_n);
+              issue_kq<D>(tS, kdesc, qk0 + slot_n * kSlotStep, idesc_s);
+              umma_commit(&ctrl->s_full);
               slot = slot_n;
             }
           } else if (ok) {
@@ -1106,22 +1140,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         sphase ^= 1;
         if (!ok) break;
         tc_fence_after();
+        // dP^T of this warp's 64 queries first (with the first 32 scores):
+        // its columns then take the next step's dP^T while this step is
+        // computed
+        float dp[64], s[32];
+        {
+          uint32_t* dr = reinterpret_cast<uint32_t*>(dp);
+          uint32_t* sr = reinterpret_cast<uint32_t*>(s);
+          RA_TMEM_LD32(tDP, dr);
+          RA_TMEM_LD32(tDP + 32, (dr + 32));
+          RA_TMEM_LD32(tS, sr);
+          tmem_wait_ld();
+        }
+        tc_fence_before();
+        mbar_arrive(&ctrl->dp_free);
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          // 32 query columns: scores and dP^T, then lse (log2 units) and D
-          float s[32], dp[32], l2[32], dd[32];
-          {
+          if (c > 0) {
             uint32_t* sr = reinterpret_cast<uint32_t*>(s);
-            uint32_t* dr = reinterpret_cast<uint32_t*>(dp);
             RA_TMEM_LD32(tS + c * 32, sr);
-            RA_TMEM_LD32(tDP + c * 32, dr);
-            const int q0 = half * 64 + c * 32;
-            const uint32_t va = smem_u32(vec + q0), vb = smem_u32(vec + BQ + q0);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              ld_shared_f4(va + 16u * u, l2[4 * u], l2[4 * u + 1], l2[4 * u + 2], l2[4 * u + 3]);
-              ld_shared_f4(vb + 16u * u, dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
-            }
             tmem_wait_ld();
           }
           // allowed query columns of this key row as a bit word
@@ -1148,23 +1185,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           uint32_t pp[16], pd[16];
+          const int q0 = half * 64 + c * 32;
 #pragma unroll
-          for (int j2 = 0; j2 < 16; ++j2) {
-            float pv[2], dv2[2];
+          for (int sb = 0; sb < 2; ++sb) {
+            // lse (log2 units) and D of 16 query columns
+            float l2[16], dd[16];
+            const uint32_t va = smem_u32(vec + q0 + 16 * sb), vb = smem_u32(vec + BQ + q0 + 16 * sb);
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int j = 2 * j2 + u;
-              const float pj = ex2_approx(fmaf(s[j], p.scale_log2, -l2[j]));
-              const bool a = (am >> j) & 1u;
-              pv[u] = a ? pj : 0.f;
-              dv2[u] = a ? pj * (dp[j] - dd[j]) : 0.f;
+            for (int u = 0; u < 4; ++u) {
+              ld_shared_f4(va + 16u * u, l2[4 * u], l2[4 * u + 1], l2[4 * u + 2], l2[4 * u + 3]);
+              ld_shared_f4(vb + 16u * u, dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
             }
-            pp[j2] = pack_x2<kFmt>(pv[0], pv[1]);
-            pd[j2] = pack_x2<kFmt>(dv2[0], dv2[1]);
+#pragma unroll
+            for (int j2 = 0; j2 < 8; ++j2) {
+              float pv[2], dv2[2];
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+                const int jl = 2 * j2 + u, j = 16 * sb + jl;
+                const float pj = ex2_approx(fmaf(s[j], p.scale_log2, -l2[jl]));
+                const bool a = (am >> j) & 1u;
+                pv[u] = a ? pj : 0.f;
+                dv2[u] = a ? pj * (dp[32 * c + j] - dd[jl]) : 0.f;
+              }
+              pp[8 * sb + j2] = pack_x2<kFmt>(pv[0], pv[1]);
+              pd[8 * sb + j2] = pack_x2<kFmt>(dv2[0], dv2[1]);
+            }
           }
-          // over the columns this warp has already read
-          RA_TMEM_ST16(tS + c * 16, pp);
-          RA_TMEM_ST16(tDP + c * 16, pd);
+          // P^T and dS^T over the 32 score columns just read
+          RA_TMEM_ST16(tS + c * 32, pp);
+          RA_TMEM_ST16(tS + c * 32 + 16, pd);
         }
         tmem_wait_st();
         tc_fence_before();

@@ -151,6 +151,9 @@ ra::FwdParams make_params(const void* q, const void* k, const void* v, int64_t t
   p.step = 0;
   p.q_block = p.kv_block = p.step_rows = 0;
   p.accumulate = 0;
+  p.step_split = 0;
+  p.split_out = nullptr;
+  p.split_lse = nullptr;
   p.withhold_q = g_withhold_q.load(std::memory_order_relaxed);
   p.sched_dump = g_sched_dump.load(std::memory_order_relaxed);
   p.sched_dump_cap = g_sched_dump_cap.load(std::memory_order_relaxed);

@@ -17,7 +17,10 @@
 // (heaviest causal ranges first); the pipelines run across item boundaries:
 // the next item's Q is loaded as soon as the last S MMA of the current one is
 // done (q_free), and its first PV MMA waits only until the softmax warps have
-// read O out (o_free).
+// read O out (o_free).  Dense causal launches run one CTA per item instead;
+// key/value-outer ring steps take items by a static stride and split the
+// items of a mostly empty last wave into halves of their key tiles, the
+// second halves folded in afterwards by step_merge_kernel.
 // Warp roles:
 //   warps 0-3  softmax for query tile 0 (one TMEM lane = one query row each)
 //   warps 4-7  softmax for query tile 1
@@ -237,6 +240,13 @@ __device__ __forceinline__ void apply_mask(float* x, const FwdParams& p, int L, 
   for (int c = 0; c < kTcBN; ++c) x[c] = ((mw[c >> 5] >> (c & 31)) & 1u) ? x[c] : -INFINITY;
 }
 
+// Is the item announced by list header h the second half of a split ring
+// step item (launch items n_items - 2 * split .. n_items - 1 come in halves)?
+__device__ __forceinline__ bool split_half(int h, int n_items, int split) {
+  const int d = -h - 8 - (n_items - 2 * split);  // launch item from the header
+  return d >= 0 && (d & 1);
+}
+
 // Schedule-list entries of an item (ra_list.cuh): (kt << 4) | (class of
 // query tile 1 << 2) | class of query tile 0 for a visited kv tile.
 __device__ __forceinline__ int entry_tile(int e) { return e >> 4; }
@@ -346,7 +356,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) ok = put(kAllDone) && flush();
         break;
       }
-      const SeqWork it = find_work_item(p, kRows, item);
+      // the halves of a split ring-step item share the item's description
+      const int n_whole = n_items - 2 * p.step_split;
+      const bool split = item >= n_whole;
+      const SeqWork it =
+          find_work_item(p, kRows, split ? n_whole + ((item - n_whole) >> 1) : item);
       if (!it.live) continue;
       if (lane == 0) {
         // query rows of this sequence held in q: the sequence, or one ring block
@@ -383,13 +397,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           // general classify() divides by the block geometry several times
           // per call, which at one thread paced the whole step).
           const int qo = p.q_block * p.step_rows, ko = p.kv_block * p.step_rows;
+          // a split item's half walks half of the block's tiles
+          const int nkt = p.step_rows / kTcBN;
+          const int kt_lo = split ? (((item - n_whole) & 1) ? nkt / 2 : 0) : 0;
+          const int kt_hi = split ? (((item - n_whole) & 1) ? nkt : nkt / 2) : nkt;
           auto seg_class = [&](int a, int b, int c) -> int {
             if (a >= b) return CLS_EMPTY;
             bool any = false, all = true;
             classify_segment(g, p.q_block, a, b, p.kv_block, c, c + kTcBN, &any, &all);
             return any ? (all ? CLS_FULL : CLS_PARTIAL) : CLS_EMPTY;
           };
-          for (kt = 0; ok && kt < p.step_rows / kTcBN; ++kt) {
+          for (kt = kt_lo; ok && kt < kt_hi; ++kt) {
             const int k0 = ko + kt * kTcBN;
             c0 = seg_class(qo + q0, qo + qm, k0);
             c1 = seg_class(qo + qm, qo + q1, k0);
@@ -522,6 +540,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       h = __shfl_sync(0xffffffffu, h, 0);
       if (!ok || h == kAllDone) break;
+      // the second half of a split ring-step item starts from the empty state
+      const bool acc = p.accumulate && !split_half(h, n_items, p.step_split);
       if (lane == 0) {
         SeqWork skip;  // the item's description is not needed here
         ok = read_item<false>(rd, &skip, abort_flag);
@@ -569,7 +589,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (!ok) break;
                 // an accumulating ring step adds to the O loaded from the state
                 issue_pv<D, kFmt>(tmem + C::kColO + i * D, tmem + C::kColS + i * kTcBN,
-                            vdesc0 + slot_v * kSlotStep, idesc_o, started[i] || p.accumulate);
+                            vdesc0 + slot_v * kSlotStep, idesc_o, started[i] || acc);
                 started[i] = true;
               }
               if (has) issue_s_tile(e, i, slot_k);
@@ -646,8 +666,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       bool first = true;
       // A ring step that accumulates starts from the running state: m = lse
       // (log2 units) with l = 1 and O = the normalised output (O = 0 where
-      // nothing was folded yet); the first PV then adds to O.
-      const bool from_state = p.step && p.accumulate;
+      // nothing was folded yet); the first PV then adds to O.  The second
+      // half of a split item (split_half) starts from the empty state.
+      const bool from_state = p.step && p.accumulate && !split_half(h, n_items, p.step_split);
       if (from_state) {
         const float lp = valid ? p.lse[li] : -INFINITY;
         const bool has = lp > -INFINITY;
@@ -784,13 +805,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const int64_t orow_off = ((int64_t)(it.base + sq) * p.heads + it.h) * D;
+      // a ring step writes fp32: the running output, or (second half of a
+      // split item) the partial at row sp_row of the split buffers
+      const bool to_split = split_half(h, n_items, p.step_split);
+      const bool acc = p.accumulate && !to_split;
+      const int64_t sp_row =
+          (int64_t)((-h - 8 - (n_items - 2 * p.step_split)) >> 1) * kRows + tile * kTcBM + r;
+      float* const srow = to_split ? p.split_out + sp_row * D
+                                   : static_cast<float*>(p.out) + orow_off;
+      const int64_t sstride = to_split ? D : (int64_t)p.heads * D;
       if (!first && p.step) {
         // ring step: the running output stays fp32, written by the warp's
         // threads together in the 16x256b fragment shape (32 contiguous
         // bytes of a row per four threads, as the state was loaded)
         const float inv_l = valid ? p.out_scale / l : 0.f;
-        float* obase = static_cast<float*>(p.out) + orow_off - (int64_t)lane * p.heads * D;
-        const int64_t rstride = (int64_t)p.heads * D;
+        float* obase = srow - (int64_t)lane * sstride;
+        const int64_t rstride = sstride;
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           const int ra = 16 * hf + (lane >> 2), rb = ra + 8;  // rows of the warp
@@ -835,19 +865,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
           }
         }
-      } else if (p.step && !p.accumulate && valid) {
+      } else if (p.step && !acc && valid) {
         // no key of this block is visible to the row: the empty result
-        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow_off);
+        float4* dst = reinterpret_cast<float4*>(srow);
 #pragma unroll
         for (int j = 0; j < D / 4; ++j) dst[j] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
       tc_fence_before();
       mbar_arrive(&ctrl->o_free[tile]);
       if (valid) {
+        float* const lse_dst = to_split ? p.split_lse + sp_row : p.lse + li;
         if (!first) {
-          p.lse[li] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
-        } else if (p.step && !p.accumulate) {
-          p.lse[li] = -INFINITY;
+          *lse_dst = (m_ref + __log2f(l)) * 0.69314718055994530942f;
+        } else if (p.step && !acc) {
+          *lse_dst = -INFINITY;
         }
         // (an accumulating step without new keys leaves the state as it was)
       }
@@ -910,6 +941,47 @@ static bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int heads,
   return r == CUDA_SUCCESS;
 }
 
+// Folds the second-half partials of a split ring step into the running
+// state (one warp per query row): with a = the state after the first half and
+// b = the partial, O = (w_a O_a + w_b O_b) / (w_a + w_b) and lse = m + ln(w_a
+// + w_b), w = exp(lse - m), m = max(lse_a, lse_b) -- the same fold as
+// ring_attn_merge.  Rows whose partial saw no key keep the state; rows whose
+// state is empty take the partial (their O is not read).
+template <int D>
+__global__ void __launch_bounds__(256) step_merge_kernel(const FwdParams p, int first_item) {
+  constexpr int kRows = kTcBM * kTcQT;
+  const int wg = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  const int s = wg / kRows, t = wg - s * kRows;
+  if (s >= p.step_split) return;
+  const WorkItem it = decode_work(p, first_item + s);
+  const int sq = it.qr * kRows + t;
+  if (sq >= p.step_rows) return;
+  const float lb = p.split_lse[(int64_t)s * kRows + t];
+  if (lb == -INFINITY) return;
+  const int64_t li = (int64_t)it.b * p.lse_seq_stride + (int64_t)it.h * p.lse_head_stride + sq;
+  float* o = static_cast<float*>(p.out) +
+             ((int64_t)(it.b * p.step_rows + sq) * p.heads + it.h) * D;
+  const float* ob = p.split_out + ((int64_t)s * kRows + t) * D;
+  const float la = p.lse[li];
+  constexpr int kPer = D / 32;  // elements per lane
+  if (la == -INFINITY) {
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) o[lane * kPer + j] = ob[lane * kPer + j];
+    if (lane == 0) p.lse[li] = lb;
+    return;
+  }
+  const float m = fmaxf(la, lb);
+  const float wa = expf(la - m), wb = expf(lb - m);
+  const float inv = 1.f / (wa + wb);
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int c = lane * kPer + j;
+    o[c] = (wa * o[c] + wb * ob[c]) * inv;
+  }
+  if (lane == 0) p.lse[li] = m + logf(wa + wb);
+}
+
 template <int D, int kFmt>
 static cudaError_t launch_tc_t(const FwdParams& p, cudaStream_t stream) {
   using C = TcCfg<D, kFmt>;
@@ -939,17 +1011,49 @@ static cudaError_t launch_tc_t(const FwdParams& p, cudaStream_t stream) {
   // dependents of the previous launch, with no counter reset between) by a
   // static stride over the CTAs.
   const bool per_item = p.causal && !p.cu_seqlens && !p.step;
-  const int64_t grid = per_item ? items : (items < num_sms ? items : num_sms);
+  // A ring step whose items leave the last wave of CTAs at most half full
+  // splits those items in halves of their key tiles, so the last wave takes
+  // half as long; a merge kernel folds the second halves in afterwards.  The
+  // partials live in stream-ordered scratch (without it the step runs
+  // unsplit).
+  int split = 0;
+  float* scratch = nullptr;
+  if (p.step && p.step_rows / kTcBN >= 2) {
+    const int64_t r = items % num_sms;
+    if (r > 0 && 2 * r <= num_sms) {
+      const size_t bytes = (size_t)r * (kTcBM * kTcQT) * (D + 1) * sizeof(float);
+      if (cudaMallocAsync(reinterpret_cast<void**>(&scratch), bytes, stream) == cudaSuccess) {
+        split = (int)r;
+      } else {
+        (void)cudaGetLastError();
+        scratch = nullptr;
+      }
+    }
+  }
+  pp.step_split = split;
+  pp.split_out = scratch;
+  pp.split_lse = scratch ? scratch + (size_t)split * (kTcBM * kTcQT) * D : nullptr;
+  const int64_t launch_items = items + split;
+  const int64_t grid =
+      per_item ? items : (launch_items < num_sms ? launch_items : num_sms);
   const int claim_limit = per_item ? 1 : 0;
+  // the scratch goes back to the pool on every exit path below
+  auto release = [&](cudaError_t err) -> cudaError_t {
+    if (scratch) {
+      const cudaError_t f = cudaFreeAsync(scratch, stream);
+      if (err == cudaSuccess) err = f;
+    }
+    return err;
+  };
   TcMaps maps;
   if (!make_map(&maps.q, p.q, p.total_rows, p.heads, D, p.tok_stride, kFmt) ||
       !make_map(&maps.k, p.k, p.total_rows, p.heads_kv, D, p.kv_tok_stride, kFmt) ||
       !make_map(&maps.v, p.v, p.total_rows, p.heads_kv, D, p.kv_tok_stride, kFmt))
-    return cudaErrorInvalidValue;
+    return release(cudaErrorInvalidValue);
   cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D, kFmt>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess) return release(e);
   if (p.step) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
@@ -961,7 +1065,15 @@ static cudaError_t launch_tc_t(const FwdParams& p, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, fwd_tc_kernel<D, kFmt>, pp, maps, (int)items, claim_limit);
+    e = cudaLaunchKernelEx(&cfg, fwd_tc_kernel<D, kFmt>, pp, maps, (int)launch_items,
+                           claim_limit);
+    if (e == cudaSuccess && split > 0) {
+      const int warps = split * kTcBM * kTcQT;
+      step_merge_kernel<D><<<(unsigned)((warps + 7) / 8), 256, 0, stream>>>(
+          pp, (int)(items - split));
+      e = cudaGetLastError();
+    }
+    return release(e);
   }
   fwd_tc_kernel<D, kFmt><<<(unsigned)grid, kTcThreads, C::kSmemBytes, stream>>>(
       pp, maps, (int)items, claim_limit);

@@ -48,6 +48,17 @@ struct FwdParams {
   int step;                 // 0: whole-sequence call
   int q_block, kv_block, step_rows;
   int accumulate;
+  // Ring steps whose items do not fill the last wave of CTAs split the
+  // last step_split items in two halves of their key tiles: launch items
+  // [0, n - step_split) are whole, then item n - step_split + s comes as
+  // halves 0 and 1 (launch items n - step_split + 2s and + 2s + 1).  Half 0
+  // folds into (out, lse) like a whole item; half 1 starts from the empty
+  // state and writes its partial (normalised O, lse) to split_out [s][row]
+  // [d_head] and split_lse [s][row] (rows of the item, 256), which a merge
+  // kernel then folds into (out, lse).  0 and NULL otherwise.
+  int step_split;
+  float* split_out;
+  float* split_lse;
   // Failure-detection test hook (0 in normal use): the tensor-core kernel's
   // producer issues no query-tile load, so the MMA issuers' bounded wait for
   // Q expires and the launch unwinds with ST_TIMEOUT.

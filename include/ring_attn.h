@@ -231,7 +231,13 @@ ra_status ring_attn_fwd_fp8(const void* q, const void* k, const void* v,
  * Launch: one persistent thread block per SM, as a programmatic dependent of
  * the launch before it on the stream, so that its set-up overlaps that
  * launch's last blocks; it reads no input before that launch has completed,
- * so ordering on the stream is the same as for any kernel.
+ * so ordering on the stream is the same as for any kernel.  When the work
+ * items (256 query rows of one head) leave the last wave of thread blocks at
+ * most half full, those items are split in two halves of the block's key
+ * tiles: the second halves write partial results to scratch taken from the
+ * stream-ordered pool (cudaMallocAsync, returned with cudaFreeAsync on the
+ * same stream), and a second kernel folds them into (out, lse).  If the pool
+ * has no room the step runs unsplit.
  */
 ra_status ring_attn_fwd_step(const void* q, const void* k, const void* v,
                              float* out, float* lse, int batch, int heads,

@@ -113,3 +113,44 @@ def test_invisible_block_gives_the_empty_state_or_leaves_it():
     torch.cuda.synchronize()
     assert ra.ring_attn_status() == ra.RA_OK
     assert torch.equal(out2, o_keep) and torch.equal(lse2, l_keep)
+
+
+@pytest.mark.parametrize("i,j,accumulate", [(3, 1, True), (2, 2, False)])
+def test_step_whose_last_wave_is_split_matches_the_oracle_fold(i, j, accumulate):
+    """A step launch whose items leave the last wave of CTAs at most half
+    full splits those items in halves of their key tiles and merges the
+    second halves afterwards.  The head count is chosen from the SM count so
+    that the launch has whole items and split ones (8 items of 256 query rows
+    per head: 2048 rows per ring block)."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    H = -(-(sms + sms // 8) // 8)        # items = 8 H in (sms, 1.5 sms]
+    assert 0 < (8 * H) % sms <= sms // 2
+    B, N, D, layout = 1, 4, 128, 0
+    L = 2048 * N
+    q, k, v = draw(B, L, H, D, 74 + i + j, torch.bfloat16)
+    scale = 1.0 / np.sqrt(D)
+    qi, kj, vj = (t[:, oracle.block_rows(L, N, layout, r)].contiguous()
+                  for t, r in ((q, i), (k, j), (v, j)))
+    b = L // N
+    g = torch.Generator().manual_seed(75)
+    out0 = torch.randn(B, b, H, D, generator=g)
+    lse0 = torch.randn(B, H, b, generator=g) * 2
+    out, lse = out0.clone().to(DEV), lse0.clone().to(DEV)
+    ra.ring_attn_fwd_step(qi.to(DEV), kj.to(DEV), vj.to(DEV), out, lse, B, H, L, D, N, i, j,
+                          accumulate, layout, True, scale)
+    torch.cuda.synchronize()
+    assert ra.ring_attn_status() == ra.RA_OK
+    if accumulate:
+        prev_o, prev_l = out0[0].numpy(), lse0[0].numpy()
+    else:
+        prev_o = np.zeros((b, H, D))
+        prev_l = np.full((H, b), -np.inf)
+    ref_o, ref_l = oracle.ring_step(qi[0].float().numpy(), kj[0].float().numpy(),
+                                    vj[0].float().numpy(), prev_o, prev_l, L, N, layout, True,
+                                    scale, i, j)
+    got_o, got_l = out[0].cpu().numpy(), lse[0].cpu().numpy()
+    fin = np.isfinite(ref_l)
+    assert np.array_equal(fin, np.isfinite(got_l))
+    assert float(np.abs(got_l[fin] - ref_l[fin]).max()) <= TOL["bf16"][1]
+    seen = fin.T
+    assert float(np.abs(got_o[seen] - ref_o[seen]).max()) <= TOL["bf16"][0]

@@ -21,16 +21,18 @@
 //   the second kernel.
 //   warps 0-7   gradient warps: warp w owns query rows 32 (w % 4) .. + 31
 //               (its TMEM lane quadrant) and keys 64 (w / 4) .. + 63
-//   warp  8     TMA producer: Q, dO per item; (K, V) pairs into a ring
+//   warp  8     TMA producer: Q, dO per item; K and V tiles into rings of
+//               their own (V(t) is free after dP(t), K(t) only after dQ(t))
 //   warp  9     MMA issuer;  warp 10 schedule builder;  warp 11 idle
 //   TMEM: S 128 | dP_A 128 | dP_B 128 | dQ D.
 //
 //  bwd_dkdv_kernel (key/value-outer): a CTA owns 128 keys of one (sequence,
-//   key/value head), one TMEM lane each, and walks the 64-row query tiles
-//   of every query head of its group that see them, 128 queries a step:
+//   key/value head), one TMEM lane each, and walks the 128-row query tiles
+//   of every query head of its group that see them, one tile a step:
 //   S^T = K Q^T and dP^T = V dO^T into tensor memory, the gradient warps
-//   write P^T and dS^T = P^T (dP^T - D) as 16-bit over the columns they have
-//   read, then dV += P^T dO and dK += dS^T Q take them from tensor memory.
+//   write P^T and dS^T = P^T (dP^T - D) as 16-bit over the score columns
+//   they have read, then dV += P^T dO and dK += dS^T Q take them from tensor
+//   memory; the next step's dP^T is computed while the gradient warps work.
 //   warps 0-3 / 4-7  gradient warps for query columns 0-63 / 64-127
 //   warp  8          TMA producer (and the per-tile lse / D vectors)
 //   warp  9          MMA issuer;  warp 10 schedule builder;  warp 11 idle

@@ -25,13 +25,13 @@
 //   warps 0-3  softmax for query tile 0 (one TMEM lane = one query row each)
 //   warps 4-7  softmax for query tile 1
 //   warp  8    TMA producer: Q once per item; K and V tiles into one ring of
-//              shared-memory slots in the order K(0), K(1), V(0), K(2), V(1),
-//              ... (the order in which the MMA issuers consume them)
-//   warps 9,11 MMA issuers, one per query tile i: S_i = Q_i K^T into tensor
+//              shared-memory slots in the order K(0), V(0), K(1), V(1), ...
+//              (the issuer takes V(t) and K(t+1) for PV(t) and S(t+1))
+//   warp  9    MMA issuer for both query tiles: S_i = Q_i K^T into tensor
 //              memory and O_i += P_i V with P_i read from tensor memory, as
-//              tcgen05.mma; completion signalled with tcgen05.commit.  Two
-//              issuers keep the tensor pipe fed while one of them waits on a
-//              barrier (a tcgen05.mma group issues at about the rate it runs).
+//              tcgen05.mma; completion signalled with tcgen05.commit.  (With
+//              kTcIssuers = 2, warps 9 and 11 issue one query tile each; one
+//              issuer measured faster: the two tiles then stay out of phase.)
 //   warp  10   schedule builder: runs the ring-order tile walk (ra_sched.h)
 //              and publishes the visited kv tiles with their per-query-tile
 //              class into a shared-memory ring of small list chunks

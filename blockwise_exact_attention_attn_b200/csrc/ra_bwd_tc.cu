@@ -589,15 +589,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nk = min(64, L - k0);
         uint32_t mw[2];
         tile_mask(mw, p, L, valid, cls, rq, tq, k0, nk);
+        // P = ex2(S scale - lse) and dS = P (dP - D) in paired fp32
+        // instructions (the same roundings as the scalar forms)
+        const uint64_t sc2 = f32x2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t nl2 = f32x2_pack(-lse2, -lse2), nd2 = f32x2_pack(-dsum, -dsum);
         uint32_t pk[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int c0 = 2 * j, c1 = 2 * j + 1;
           const bool a0 = (mw[c0 >> 5] >> (c0 & 31)) & 1u;
           const bool a1 = (mw[c1 >> 5] >> (c1 & 31)) & 1u;
-          const float p0 = a0 ? ex2_approx(fmaf(s[c0], p.scale_log2, -lse2)) : 0.f;
-          const float p1 = a1 ? ex2_approx(fmaf(s[c1], p.scale_log2, -lse2)) : 0.f;
-          pk[j] = pack_x2<kFmt>(p0 * (dp[c0] - dsum), p1 * (dp[c1] - dsum));
+          float y0, y1;
+          ffma2(s[c0], s[c1], sc2, nl2, y0, y1);
+          const float p0 = a0 ? ex2_approx(y0) : 0.f;
+          const float p1 = a1 ? ex2_approx(y1) : 0.f;
+          const uint64_t r2 = mul2(f32x2_pack(p0, p1), add2(f32x2_pack(dp[c0], dp[c1]), nd2));
+          pk[j] = pack_x2<kFmt>(f32x2_lo(r2), f32x2_hi(r2));
         }
         // dS over the first 32 of this warp's dP columns (already read)
         RA_TMEM_ST32(tDP, pk);
@@ -971,8 +978,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               l2 = p.lse[li] * 1.4426950408889634f;
               dd = bp.dsum[li];
             }
-            vec[j] = l2;
-            vec[BQ + j] = dd;
+            // stored negated: the gradient warps add them
+            vec[j] = -l2;
+            vec[BQ + j] = -dd;
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(&ctrl->q_full[slot]);
@@ -1190,27 +1198,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int q0 = half * 64 + c * 32;
 #pragma unroll
           for (int sb = 0; sb < 2; ++sb) {
-            // lse (log2 units) and D of 16 query columns
-            float l2[16], dd[16];
+            // -lse (log2 units) and -D of 16 query columns
+            float nl[16], nd[16];
             const uint32_t va = smem_u32(vec + q0 + 16 * sb), vb = smem_u32(vec + BQ + q0 + 16 * sb);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-              ld_shared_f4(va + 16u * u, l2[4 * u], l2[4 * u + 1], l2[4 * u + 2], l2[4 * u + 3]);
-              ld_shared_f4(vb + 16u * u, dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
+              ld_shared_f4(va + 16u * u, nl[4 * u], nl[4 * u + 1], nl[4 * u + 2], nl[4 * u + 3]);
+              ld_shared_f4(vb + 16u * u, nd[4 * u], nd[4 * u + 1], nd[4 * u + 2], nd[4 * u + 3]);
             }
+            // P = ex2(S scale - lse) and dS = P (dP - D) in paired fp32
+            // instructions (the same roundings as the scalar forms); masked
+            // entries are selected to zero after the products
+            const uint64_t sc2 = f32x2_pack(p.scale_log2, p.scale_log2);
 #pragma unroll
             for (int j2 = 0; j2 < 8; ++j2) {
-              float pv[2], dv2[2];
-#pragma unroll
-              for (int u = 0; u < 2; ++u) {
-                const int jl = 2 * j2 + u, j = 16 * sb + jl;
-                const float pj = ex2_approx(fmaf(s[j], p.scale_log2, -l2[jl]));
-                const bool a = (am >> j) & 1u;
-                pv[u] = a ? pj : 0.f;
-                dv2[u] = a ? pj * (dp[32 * c + j] - dd[jl]) : 0.f;
-              }
-              pp[8 * sb + j2] = pack_x2<kFmt>(pv[0], pv[1]);
-              pd[8 * sb + j2] = pack_x2<kFmt>(dv2[0], dv2[1]);
+              const int jl = 2 * j2, j = 16 * sb + jl;
+              float y0, y1;
+              ffma2(s[j], s[j + 1], sc2, f32x2_pack(nl[jl], nl[jl + 1]), y0, y1);
+              const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
+              const uint64_t r2 = mul2(f32x2_pack(p0, p1),
+                                       add2(f32x2_pack(dp[32 * c + j], dp[32 * c + j + 1]),
+                                            f32x2_pack(nd[jl], nd[jl + 1])));
+              const bool a0 = (am >> j) & 1u, a1 = (am >> (j + 1)) & 1u;
+              pp[8 * sb + j2] = pack_x2<kFmt>(a0 ? p0 : 0.f, a1 ? p1 : 0.f);
+              pd[8 * sb + j2] = pack_x2<kFmt>(a0 ? f32x2_lo(r2) : 0.f, a1 ? f32x2_hi(r2) : 0.f);
             }
           }
           // P^T and dS^T over the 32 score columns just read

@@ -529,35 +529,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t li = (int64_t)it.b * p.lse_seq_stride + (int64_t)it.h * p.lse_head_stride +
                          (p.cu_seqlens ? it.base : 0) + sq;
       const int64_t roff = ((int64_t)(it.base + sq) * bp.heads_q + it.h) * D;
-      // D = <dO, O> for this row, fp32 over the 16-bit inputs (both warps of
-      // the row form it; the first writes it for the dK/dV kernel)
+      // D = <dO, O> for the warp's 32 rows, fp32 over the 16-bit inputs.  The
+      // lanes read them together: an instruction covers two rows, 16 bytes
+      // per lane (whole lines), and each row is summed over its 16 lanes by
+      // shuffles and handed to the row's own lane.  Both warps of a row form
+      // it; the first writes it for the dK/dV kernel.
       float dsum = 0.f, lse2 = 0.f;
-      if (valid) {
-        const uint4* dorow = reinterpret_cast<const uint4*>(
-            static_cast<const uint16_t*>(bp.dout) + roff);
-        const uint4* orow =
-            reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(bp.o) + roff);
+      {
+        const int sub = lane >> 4, ch = lane & 15;  // row of the pair, 16-byte chunk
+        const int row0 = sq - lane;                  // the warp's first row
 #pragma unroll 4
-        for (int c = 0; c < D / 8; ++c) {
-          const uint4 a = dorow[c], b = orow[c];
-          const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+        for (int i = 0; i < 16; ++i) {
+          const int sr = row0 + 2 * i + sub;
+          float part = 0.f;
+          if (sr < L && ch < D / 8) {
+            const int64_t ro = ((int64_t)(it.base + sr) * bp.heads_q + it.h) * D;
+            const uint4 a = reinterpret_cast<const uint4*>(
+                static_cast<const uint16_t*>(bp.dout) + ro)[ch];
+            const uint4 b =
+                reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(bp.o) + ro)[ch];
+            const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float a0, a1, b0, b1;
-            if (kFmt == kFmtBF16) {
-              a0 = __uint_as_float(av[j] << 16);
-              a1 = __uint_as_float(av[j] & 0xffff0000u);
-              b0 = __uint_as_float(bv[j] << 16);
-              b1 = __uint_as_float(bv[j] & 0xffff0000u);
-            } else {
-              const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&av[j]));
-              const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&bv[j]));
-              a0 = fa.x; a1 = fa.y; b0 = fb.x; b1 = fb.y;
+            for (int j = 0; j < 4; ++j) {
+              float a0, a1, b0, b1;
+              if (kFmt == kFmtBF16) {
+                a0 = __uint_as_float(av[j] << 16);
+                a1 = __uint_as_float(av[j] & 0xffff0000u);
+                b0 = __uint_as_float(bv[j] << 16);
+                b1 = __uint_as_float(bv[j] & 0xffff0000u);
+              } else {
+                const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&av[j]));
+                const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&bv[j]));
+                a0 = fa.x; a1 = fa.y; b0 = fb.x; b1 = fb.y;
+              }
+              part = fmaf(a0, b0, part);
+              part = fmaf(a1, b1, part);
             }
-            dsum = fmaf(a0, b0, dsum);
-            dsum = fmaf(a1, b1, dsum);
           }
+#pragma unroll
+          for (int off = 8; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+          const float t0 = __shfl_sync(0xffffffffu, part, 0);
+          const float t1 = __shfl_sync(0xffffffffu, part, 16);
+          if (lane == 2 * i) dsum = t0;
+          if (lane == 2 * i + 1) dsum = t1;
         }
+      }
+      if (valid) {
         lse2 = p.lse[li] * 1.4426950408889634f;
         if (bp.dsum && half == 0) bp.dsum[li] = dsum;
       }

@@ -888,37 +888,48 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_dec<kRegsControl>();
     if (warp == kBuilder) {
       // ---------------------------------------------------------- schedule
-      // One item per CTA (grid = items): its header, then for every query
-      // head of the key/value head's group every query tile that sees the
-      // key tile, with its class.
+      // Per item: its header, then for every query head of the key/value
+      // head's group every query tile that sees the key tile, with its
+      // class.  The CTAs take the items in waves of one per CTA, every other
+      // wave in reverse CTA order (one wave when the grid has a CTA per item).
       ListWriter wr;
       wr.list = smem_u32(list);
       wr.full = ctrl->list_full;
       wr.empty = ctrl->list_empty;
       wr.abort = abort_flag;
       bool ok = true;
-      const int item = blockIdx.x;
-      const SeqWork it = find_work_item(p, BK, item);
-      if (lane == 0) {
-        if (it.live && item < n_items) {
-          const int k_lo = it.qr * BK, k_hi = min(k_lo + BK, it.L);
-          const RingGeom g = make_geom(it.L, p.n_ring, p.layout, p.causal, p.passes);
-          ok = put_item(wr, item, it);
-          const int nqt = (it.L + BQ - 1) / BQ;
-          // contiguous causal: the query tiles that end before the first key
-          // see none of it (query and key positions are the stored rows), so
-          // the walk starts at the tile that holds row k_lo; every other
-          // tile is classified exactly (a few divisions per call, which the
-          // leading empty tiles would otherwise spend before the first entry)
-          const int qt0 = (g.causal && g.layout == LAYOUT_CONTIGUOUS) ? k_lo / BQ : 0;
-          for (int gq = 0; ok && gq < p.kv_group; ++gq)
-            for (int qt = qt0; ok && qt < nqt; ++qt) {
-              const int q_lo = qt * BQ, q_hi = min(q_lo + BQ, it.L);
-              const int cls = classify(g, q_lo, q_hi, k_lo, k_hi);
-              if (cls != CLS_EMPTY) ok = wr.put((gq << 24) | (qt << 2) | cls);
-            }
-          if (ok) ok = wr.put(kItemEnd);
+      int claims = 0;
+      while (ok) {
+        const int wave_pos =
+            (claims & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x;
+        const int item = claims * (int)gridDim.x + wave_pos;
+        ++claims;
+        if (item >= n_items) break;
+        const SeqWork it = find_work_item(p, BK, item);
+        if (lane == 0) {
+          if (it.live) {
+            const int k_lo = it.qr * BK, k_hi = min(k_lo + BK, it.L);
+            const RingGeom g = make_geom(it.L, p.n_ring, p.layout, p.causal, p.passes);
+            ok = put_item(wr, item, it);
+            const int nqt = (it.L + BQ - 1) / BQ;
+            // contiguous causal: the query tiles that end before the first key
+            // see none of it (query and key positions are the stored rows), so
+            // the walk starts at the tile that holds row k_lo; every other
+            // tile is classified exactly (a few divisions per call, which the
+            // leading empty tiles would otherwise spend before the first entry)
+            const int qt0 = (g.causal && g.layout == LAYOUT_CONTIGUOUS) ? k_lo / BQ : 0;
+            for (int gq = 0; ok && gq < p.kv_group; ++gq)
+              for (int qt = qt0; ok && qt < nqt; ++qt) {
+                const int q_lo = qt * BQ, q_hi = min(q_lo + BQ, it.L);
+                const int cls = classify(g, q_lo, q_hi, k_lo, k_hi);
+                if (cls != CLS_EMPTY) ok = wr.put((gq << 24) | (qt << 2) | cls);
+              }
+            if (ok) ok = wr.put(kItemEnd);
+          }
         }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      }
+      if (lane == 0) {
         if (ok) ok = wr.put(kAllDone);
         if (ok) ok = wr.flush();
         if (!ok) {
@@ -1300,7 +1311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D, int kFmt>
-static cudaError_t launch_t(const Params& bp_in, cudaStream_t stream) {
+static cudaError_t launch_t(const Params& bp_in, cudaStream_t stream, int num_sms) {
   using C = Cfg<D>;
   Params bp = bp_in;
   FwdParams& p = bp.f;
@@ -1320,7 +1331,12 @@ static cudaError_t launch_t(const Params& bp_in, cudaStream_t stream) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  bwd_dkdv_kernel<D, kFmt><<<(unsigned)items, kThreads, C::kSmemBytes, stream>>>(
+  // Dense causal items differ in length: one CTA per item, balanced by the
+  // hardware block scheduler (persistent CTAs measured 11 % slower there).
+  // Otherwise persistent CTAs, one per SM (1.6-2.3 % faster non-causal).
+  const bool per_item = p.causal && !p.cu_seqlens;
+  const int64_t grid = per_item ? items : (items < num_sms ? items : num_sms);
+  bwd_dkdv_kernel<D, kFmt><<<(unsigned)grid, kThreads, C::kSmemBytes, stream>>>(
       bp, maps, (int)items);
   return cudaGetLastError();
 }
@@ -1334,7 +1350,7 @@ static cudaError_t launch_both(const Params& bp, int num_sms, cudaStream_t strea
   // dK/dV: the work decode runs over the key/value heads
   Params kvp = bp;
   kvp.f.heads = bp.f.heads_kv;
-  return kv::launch_t<D, kFmt>(kvp, stream);
+  return kv::launch_t<D, kFmt>(kvp, stream, num_sms);
 }
 
 }  // namespace tcb

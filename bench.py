@@ -608,6 +608,9 @@ def main():
     ap.add_argument("--backward", action="store_true",
                     help="time only the backward (ring_attn_bwd) workload and print its "
                          "object (for profiling captures)")
+    ap.add_argument("--ring-steps", action="store_true",
+                    help="time only the key/value-outer ring-step workload and print its "
+                         "object (for profiling captures)")
     ap.add_argument("--heads", type=int, default=0,
                     help="run the workload with this many heads (a reduced copy for "
                          "profiling captures); 0 keeps the workload's own")
@@ -618,15 +621,18 @@ def main():
         if args.impl == "reference":
             run_reference(args, dist)
             return
-        if args.backward:
+        if args.backward or args.ring_steps:
             import blockwise_exact_attention_attn_b200 as ra
             dev = torch.device("cuda", dist.local)
             torch.cuda.set_device(dev)
             ra.load_library()
             peaks, _ = load_peaks()
-            r = measure_backward(args.steps, args.warmup, dist, dev, peaks)
+            if args.backward:
+                r = {"backward": measure_backward(args.steps, args.warmup, dist, dev, peaks)}
+            else:
+                r = {"ring_steps": measure_ring_steps(args.steps, args.warmup, dist, dev, peaks)}
             if dist.rank == 0:
-                print(json.dumps({"backward": r}), flush=True)
+                print(json.dumps(r), flush=True)
             return
         run_ours(args, dist)
     finally:

@@ -191,8 +191,9 @@ ra_status run_fwd(const ra::FwdParams& params, int dtype, void* stream, bool for
   if (st != RA_OK) return st;
   p.status = status;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // (ring steps need no counter: one CTA per item, and no memset between
-  // consecutive step launches, which run as programmatic dependents)
+  // (ring steps need no counter: their CTAs take items by a static stride,
+  // so no memset runs between consecutive step launches, which are
+  // programmatic dependents of each other)
   if (uses_tc(p, dtype, force_simt) && !p.step) {
     p.work_counter = next_counter(status);
     if (cudaMemsetAsync(p.work_counter, 0, sizeof(int), s) != cudaSuccess) return RA_ERR_CUDA;

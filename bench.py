@@ -164,10 +164,12 @@ def source_hash(names) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(workload: str, path: str = None):
     """DRAM bytes per launch of the tensor-core kernel from the committed ncu
-    summary, if it was taken on the current kernel source."""
-    path = os.path.join(ROOT, "profiles", "fwd_tc_traffic.txt")
+    summary (or the summary at `path`), if it was taken on the current kernel
+    source and on this workload."""
+    if path is None:
+        path = os.path.join(ROOT, "profiles", "fwd_tc_traffic.txt")
     if not os.path.exists(path):
         return None
     kv = {}
